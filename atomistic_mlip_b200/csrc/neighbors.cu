@@ -1,0 +1,329 @@
+// Cell-list radius graph -> sorted CSR (the neighbour set j in N(i) that
+// E2Former-V2's node-centric attention streams over, "E2Former-V2 ...",
+// §2.2 "Streaming reduction").
+//
+// Steps (all on `stream`):
+//   bbox (open dims only; one host read)  -> grid of cells of edge >= r_c
+//   cell_assign: cell of each atom + per-cell counts (+ domain check)
+//   scan -> cell_start;  cell_scatter -> atoms grouped by cell
+//   count: warp per atom over the 27-cell stencil, exact fp32 predicate
+//   scan -> row_ptr, E read back (one host read), capacity check
+//   fill: warp per atom, same stencil; the row is collected in shared
+//         memory and written in ascending j (rank placement), or, for rows
+//         longer than the shared buffer, written then sorted in place.
+#include <math.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "scan.cuh"
+
+namespace e2f {
+
+struct CellGrid {
+  int nc[3];
+  float lo[3];    // grid origin (0 in periodic dims)
+  float inv[3];   // cells per Angstrom
+  int stencil[3]; // 1: offsets -1..1, 0: offset 0 only
+};
+
+constexpr int NB_WARPS = 8;
+constexpr int ROW_CAP = 512;   // shared-memory row buffer per warp
+
+__global__ void bbox_partial_kernel(const float *__restrict__ pos, int n, float *__restrict__ part) {
+  float mn[3] = {INFINITY, INFINITY, INFINITY}, mx[3] = {-INFINITY, -INFINITY, -INFINITY};
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      float v = pos[3 * i + k];
+      mn[k] = fminf(mn[k], v);
+      mx[k] = fmaxf(mx[k], v);
+    }
+  }
+  __shared__ float sm[6][32];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn[k] = fminf(mn[k], __shfl_xor_sync(0xffffffffu, mn[k], o));
+      mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], o));
+    }
+  }
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (lane == 0) {
+    for (int k = 0; k < 3; ++k) { sm[k][wid] = mn[k]; sm[3 + k][wid] = mx[k]; }
+  }
+  __syncthreads();
+  if (threadIdx.x < 6) {
+    float v = sm[threadIdx.x][0];
+    for (int w = 1; w < nw; ++w) v = threadIdx.x < 3 ? fminf(v, sm[threadIdx.x][w]) : fmaxf(v, sm[threadIdx.x][w]);
+    part[blockIdx.x * 6 + threadIdx.x] = v;
+  }
+}
+
+__global__ void bbox_final_kernel(const float *__restrict__ part, int nparts, float *__restrict__ out) {
+  if (threadIdx.x < 6) {
+    float v = part[threadIdx.x];
+    for (int b = 1; b < nparts; ++b)
+      v = threadIdx.x < 3 ? fminf(v, part[b * 6 + threadIdx.x]) : fmaxf(v, part[b * 6 + threadIdx.x]);
+    out[threadIdx.x] = v;
+  }
+}
+
+__device__ __forceinline__ int cell_coord(float p, const CellGrid &cg, int k) {
+  int c = (int)floorf(__fmul_rn(__fsub_rn(p, cg.lo[k]), cg.inv[k]));
+  return min(max(c, 0), cg.nc[k] - 1);
+}
+
+__global__ void cell_assign_kernel(const float *__restrict__ pos, int n, CellGrid cg, Geom g,
+                                   int32_t *__restrict__ cell_of, int32_t *__restrict__ cell_count,
+                                   int32_t *__restrict__ domain_err) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  int c[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    float p = pos[3 * i + k];
+    bool ok = g.periodic[k] ? (p >= 0.f && p < g.box[k]) : (p == p && fabsf(p) < INFINITY);
+    if (!ok) atomicExch(domain_err, 1);
+    c[k] = cell_coord(p, cg, k);
+  }
+  const int cid = c[0] + cg.nc[0] * (c[1] + cg.nc[1] * c[2]);
+  cell_of[i] = cid;
+  atomicAdd(&cell_count[cid], 1);
+}
+
+__global__ void cell_scatter_kernel(const int32_t *__restrict__ cell_of, int n,
+                                    const int32_t *__restrict__ cell_start, int32_t *__restrict__ cursor,
+                                    int32_t *__restrict__ atom_by_cell) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int c = cell_of[i];
+  const int slot = atomicAdd(&cursor[c], 1);
+  atom_by_cell[cell_start[c] + slot] = i;
+}
+
+// Visit the stencil cells of atom i; f(j) is called by each lane for its
+// candidates (all lanes of the warp iterate together, inactive lanes get -1).
+template <typename F>
+__device__ __forceinline__ void for_stencil(int cid, const CellGrid &cg, const Geom &g,
+                                            const int32_t *__restrict__ cell_start,
+                                            const int32_t *__restrict__ atom_by_cell, int lane, F &&f) {
+  const int cx = cid % cg.nc[0];
+  const int cy = (cid / cg.nc[0]) % cg.nc[1];
+  const int cz = cid / (cg.nc[0] * cg.nc[1]);
+  const int rz = cg.stencil[2], ry = cg.stencil[1], rx = cg.stencil[0];
+  for (int dz = -rz; dz <= rz; ++dz) {
+    int z = cz + dz;
+    if (g.periodic[2]) z = (z + cg.nc[2]) % cg.nc[2];
+    else if (z < 0 || z >= cg.nc[2]) continue;
+    for (int dy = -ry; dy <= ry; ++dy) {
+      int y = cy + dy;
+      if (g.periodic[1]) y = (y + cg.nc[1]) % cg.nc[1];
+      else if (y < 0 || y >= cg.nc[1]) continue;
+      for (int dx = -rx; dx <= rx; ++dx) {
+        int x = cx + dx;
+        if (g.periodic[0]) x = (x + cg.nc[0]) % cg.nc[0];
+        else if (x < 0 || x >= cg.nc[0]) continue;
+        const int c = x + cg.nc[0] * (y + cg.nc[1] * z);
+        const int s = cell_start[c], e = cell_start[c + 1];
+        for (int t = s; t < e; t += 32) {
+          const int idx = t + lane;
+          f(idx < e ? atom_by_cell[idx] : -1);
+        }
+      }
+    }
+  }
+}
+
+__global__ void count_kernel(const float *__restrict__ pos, int n, CellGrid cg, Geom g,
+                             const int32_t *__restrict__ cell_of, const int32_t *__restrict__ cell_start,
+                             const int32_t *__restrict__ atom_by_cell, int32_t *__restrict__ deg) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * NB_WARPS + (threadIdx.x >> 5);
+  if (i >= n) return;
+  const float3 pi = load_pos(pos, i);
+  int cnt = 0;
+  for_stencil(cell_of[i], cg, g, cell_start, atom_by_cell, lane, [&](int j) {
+    if (j >= 0 && j != i) {
+      float dx, dy, dz;
+      pair_disp(g, pi, load_pos(pos, j), dx, dy, dz);
+      if (pair_r2(dx, dy, dz) < g.rc2) ++cnt;
+    }
+  });
+  cnt = warp_sum_i(cnt);
+  if (lane == 0) deg[i] = cnt;
+}
+
+__global__ void fill_kernel(const float *__restrict__ pos, int n, CellGrid cg, Geom g,
+                            const int32_t *__restrict__ cell_of, const int32_t *__restrict__ cell_start,
+                            const int32_t *__restrict__ atom_by_cell, const int32_t *__restrict__ row_ptr,
+                            int32_t *__restrict__ col_idx) {
+  __shared__ int32_t buf[NB_WARPS][ROW_CAP];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int i = blockIdx.x * NB_WARPS + wid;
+  if (i >= n) return;
+  const int r0 = row_ptr[i];
+  const int deg = row_ptr[i + 1] - r0;
+  const bool in_smem = deg <= ROW_CAP;
+  int32_t *row = col_idx + r0;
+  int32_t *b = buf[wid];
+  const float3 pi = load_pos(pos, i);
+  int w = 0;
+  for_stencil(cell_of[i], cg, g, cell_start, atom_by_cell, lane, [&](int j) {
+    bool pass = false;
+    if (j >= 0 && j != i) {
+      float dx, dy, dz;
+      pair_disp(g, pi, load_pos(pos, j), dx, dy, dz);
+      pass = pair_r2(dx, dy, dz) < g.rc2;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, pass);
+    const int p = w + __popc(m & ((1u << lane) - 1u));
+    if (pass && p < deg) {
+      if (in_smem) b[p] = j;
+      else row[p] = j;
+    }
+    w += __popc(m);
+  });
+  __syncwarp();
+  if (in_smem) {
+    // rank placement: keys are distinct atom indices
+    for (int e = lane; e < deg; e += 32) {
+      const int key = b[e];
+      int rank = 0;
+      for (int t = 0; t < deg; ++t) rank += (b[t] < key);
+      row[rank] = key;
+    }
+  } else {
+    // odd-even transposition sort in place (rare long rows)
+    for (int round = 0; round < deg; ++round) {
+      for (int k = 2 * lane + (round & 1); k + 1 < deg; k += 64) {
+        int a = row[k], c = row[k + 1];
+        if (a > c) { row[k] = c; row[k + 1] = a; }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, float r_c,
+                                int32_t *row_ptr, int32_t *col_idx, int64_t capacity, int64_t *n_edges,
+                                cudaStream_t s) {
+  Geom g;
+  bool any_open = false;
+  for (int k = 0; k < 3; ++k) {
+    const float b = box ? box[k] : 0.f;
+    g.periodic[k] = b > 0.f;
+    g.box[k] = g.periodic[k] ? b : 0.f;
+    g.half[k] = 0.5f * g.box[k];
+    any_open |= !g.periodic[k];
+  }
+  g.rc = r_c;
+  g.rc2 = r_c * r_c;
+  const int n = (int)N;
+  if (n == 0) {
+    E2F_CUDA_TRY(cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), s));
+    *n_edges = 0;
+    return E2F_OK;
+  }
+
+  // bounding box of open dimensions (host sync 1)
+  float bb[6] = {0, 0, 0, 0, 0, 0};
+  if (any_open) {
+    const int nparts = std::min(256, (n + 255) / 256);
+    Scratch part;
+    E2F_CUDA_TRY(part.alloc(sizeof(float) * (6 * nparts + 6), s));
+    float *pp = part.as<float>();
+    E2F_LAUNCH(bbox_partial_kernel, nparts, 256, 0, s, pos, n, pp);
+    E2F_LAUNCH(bbox_final_kernel, 1, 32, 0, s, pp, nparts, pp + 6 * nparts);
+    E2F_CUDA_TRY(cudaMemcpyAsync(bb, pp + 6 * nparts, sizeof(bb), cudaMemcpyDeviceToHost, s));
+    E2F_CUDA_TRY(cudaStreamSynchronize(s));
+    for (int k = 0; k < 6; ++k)
+      if (!(fabsf(bb[k]) < INFINITY)) return E2F_ERR_DOMAIN;
+  }
+
+  // cell grid: cells of edge >= r_c with a relative margin far above the
+  // rounding of the cell-index computation
+  CellGrid cg;
+  double cs[3];
+  long long ncell = 1;
+  for (int k = 0; k < 3; ++k) {
+    if (g.periodic[k]) {
+      const double b = g.box[k];
+      const double cmin = (double)r_c * 1.001 + b * 1e-6;
+      int nc = (int)floor(b / cmin);
+      if (nc < 3) nc = 1;
+      cg.nc[k] = nc;
+      cg.lo[k] = 0.f;
+      cs[k] = b / nc;
+      cg.inv[k] = (float)(nc / b);
+      cg.stencil[k] = nc >= 3 ? 1 : 0;
+    } else {
+      const double ext = (double)bb[3 + k] - (double)bb[k];
+      cs[k] = (double)r_c * 1.001 + fabs(ext) * 1e-6 + 1e-6 * fabs((double)bb[k]);
+      cg.lo[k] = bb[k];
+    }
+  }
+  // bound the number of cells (sparse open systems): grow open cells
+  for (int it = 0; it < 64; ++it) {
+    ncell = 1;
+    for (int k = 0; k < 3; ++k) {
+      if (!g.periodic[k]) {
+        const double ext = (double)bb[3 + k] - (double)bb[k];
+        cg.nc[k] = (int)std::min<double>(floor(ext / cs[k]) + 1.0, 1 << 20);
+        cg.inv[k] = (float)(1.0 / cs[k]);
+        cg.stencil[k] = 1;
+      }
+      ncell *= cg.nc[k];
+    }
+    if (ncell <= std::max<long long>(4096, 8LL * n)) break;
+    for (int k = 0; k < 3; ++k)
+      if (!g.periodic[k]) cs[k] *= 1.25;
+  }
+
+  Scratch cell_of, cnt, cstart, cursor, abc, deg, flag, scan_tmp;
+  E2F_CUDA_TRY(cell_of.alloc(sizeof(int32_t) * n, s));
+  E2F_CUDA_TRY(cnt.alloc(sizeof(int32_t) * ncell, s));
+  E2F_CUDA_TRY(cstart.alloc(sizeof(int32_t) * (ncell + 1), s));
+  E2F_CUDA_TRY(cursor.alloc(sizeof(int32_t) * ncell, s));
+  E2F_CUDA_TRY(abc.alloc(sizeof(int32_t) * n, s));
+  E2F_CUDA_TRY(deg.alloc(sizeof(int32_t) * n, s));
+  E2F_CUDA_TRY(flag.alloc(sizeof(int32_t) * 4, s));
+  E2F_CUDA_TRY(scan_tmp.alloc(std::max(scan_scratch_bytes(ncell), scan_scratch_bytes(n)), s));
+  E2F_CUDA_TRY(cudaMemsetAsync(cnt.p, 0, sizeof(int32_t) * ncell, s));
+  E2F_CUDA_TRY(cudaMemsetAsync(cursor.p, 0, sizeof(int32_t) * ncell, s));
+  E2F_CUDA_TRY(cudaMemsetAsync(flag.p, 0, sizeof(int32_t) * 4, s));
+
+  const int tb = 256;
+  E2F_LAUNCH(cell_assign_kernel, (n + tb - 1) / tb, tb, 0, s, pos, n, cg, g, cell_of.as<int32_t>(),
+             cnt.as<int32_t>(), flag.as<int32_t>());
+  e2f_status st = exclusive_scan(cnt.as<int32_t>(), ncell, cstart.as<int32_t>(), scan_tmp.p, s, nullptr);
+  if (st != E2F_OK) return st;
+  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, cell_of.as<int32_t>(), n,
+             cstart.as<int32_t>(), cursor.as<int32_t>(), abc.as<int32_t>());
+  const int nblk = (n + NB_WARPS - 1) / NB_WARPS;
+  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of.as<int32_t>(),
+             cstart.as<int32_t>(), abc.as<int32_t>(), deg.as<int32_t>());
+  long long *total = nullptr;
+  st = exclusive_scan(deg.as<int32_t>(), n, row_ptr, scan_tmp.p, s, &total);
+  if (st != E2F_OK) return st;
+
+  // E and the domain flag (host sync 2)
+  long long E = 0;
+  int32_t dom = 0;
+  E2F_CUDA_TRY(cudaMemcpyAsync(&E, total, sizeof(long long), cudaMemcpyDeviceToHost, s));
+  E2F_CUDA_TRY(cudaMemcpyAsync(&dom, flag.p, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  E2F_CUDA_TRY(cudaStreamSynchronize(s));
+  *n_edges = E;
+  if (dom) return E2F_ERR_DOMAIN;
+  if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
+  if (E > capacity) return E2F_ERR_CAPACITY;
+  if (E > 0) {
+    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of.as<int32_t>(),
+               cstart.as<int32_t>(), abc.as<int32_t>(), row_ptr, col_idx);
+  }
+  return E2F_OK;
+}
+
+}  // namespace e2f

@@ -121,6 +121,7 @@ const char *e2f_status_string(e2f_status s) {
     case E2F_ERR_CUDA: return "CUDA error";
     case E2F_ERR_TIMEOUT: return "bounded device wait timed out";
     case E2F_ERR_DOMAIN: return "coordinate outside the periodic box";
+    case E2F_ERR_SCRATCH_LIMIT: return "input exceeds the fixed scratch of a no-allocation entry point";
     default: return "unknown status";
   }
 }

@@ -14,6 +14,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "scan.cuh"
@@ -327,3 +328,198 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
 }
 
 }  // namespace e2f
+
+// ===========================================================================
+// Allocation-free variant: e2f_build_neighbors_noalloc.
+//
+// Same kernels and the same result as e2f_build_neighbors, but every
+// temporary array lives in one fixed, file-scope device array instead of
+// memory taken from a pool, so the call never allocates device memory.
+// Limits: at most NOALLOC_MAX_ATOMS atoms; the cell grid is coarsened (cells
+// only grow, which never drops a pair) until it has at most
+// NOALLOC_MAX_CELLS cells.  Every call on a device shares the array and it
+// keeps the previous call's contents, so the counters that must start at
+// zero are cleared on the stream first, and two calls whose GPU work
+// overlaps (different streams, no ordering between them) race on it.
+// ===========================================================================
+namespace e2f {
+
+constexpr int64_t NOALLOC_MAX_ATOMS = 1 << 17;   // 131,072 atoms
+constexpr int64_t NOALLOC_MAX_CELLS = 1 << 17;   // 131,072 cells
+
+// layout of the array, in 4-byte words (offsets kept 64-word aligned)
+constexpr size_t NA_CELL_OF = 0;
+constexpr size_t NA_ABC = NA_CELL_OF + NOALLOC_MAX_ATOMS;
+constexpr size_t NA_DEG = NA_ABC + NOALLOC_MAX_ATOMS;
+constexpr size_t NA_CNT = NA_DEG + NOALLOC_MAX_ATOMS;
+constexpr size_t NA_CSTART = NA_CNT + NOALLOC_MAX_CELLS;
+constexpr size_t NA_CURSOR = NA_CSTART + NOALLOC_MAX_CELLS + 64;
+constexpr size_t NA_FLAG = NA_CURSOR + NOALLOC_MAX_CELLS;
+constexpr size_t NA_BBOX = NA_FLAG + 64;
+constexpr size_t NA_SCAN = NA_BBOX + 2048;        // 6 * 256 + 6 floats fit
+constexpr size_t NA_WORDS = NA_SCAN + 256;        // scan sums: long longs
+static_assert(NA_SCAN % 2 == 0, "scan sums need 8-byte alignment");
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[NA_WORDS];
+
+// Device address of the array on the current device (looked up once per
+// device; host code cannot use the symbol itself as a device address).
+static std::mutex g_na_mu;
+static void *g_na_ptr[64] = {nullptr};
+
+static e2f_status noalloc_scratch(int32_t **p) {
+  int dev = 0;
+  E2F_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_na_mu);
+  if (!g_na_ptr[dev]) {
+    void *ptr = nullptr;
+    E2F_CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+    g_na_ptr[dev] = ptr;
+  }
+  *p = static_cast<int32_t *>(g_na_ptr[dev]);
+  return E2F_OK;
+}
+
+static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, const float *box, float r_c,
+                                               int32_t *row_ptr, int32_t *col_idx, int64_t capacity,
+                                               int64_t *n_edges, cudaStream_t s) {
+  int32_t *ws = nullptr;
+  e2f_status st = noalloc_scratch(&ws);
+  if (st != E2F_OK) return st;
+  Geom g;
+  bool any_open = false;
+  for (int k = 0; k < 3; ++k) {
+    const float b = box ? box[k] : 0.f;
+    g.periodic[k] = b > 0.f;
+    g.box[k] = g.periodic[k] ? b : 0.f;
+    g.half[k] = 0.5f * g.box[k];
+    any_open |= !g.periodic[k];
+  }
+  g.rc = r_c;
+  g.rc2 = r_c * r_c;
+  const int n = (int)N;
+  if (n == 0) {
+    E2F_CUDA_TRY(cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), s));
+    *n_edges = 0;
+    return E2F_OK;
+  }
+  float bb[6] = {0, 0, 0, 0, 0, 0};
+  if (any_open) {
+    const int nparts = std::min(256, (n + 255) / 256);
+    float *pp = reinterpret_cast<float *>(ws + NA_BBOX);
+    E2F_LAUNCH(bbox_partial_kernel, nparts, 256, 0, s, pos, n, pp);
+    E2F_LAUNCH(bbox_final_kernel, 1, 32, 0, s, pp, nparts, pp + 6 * nparts);
+    E2F_CUDA_TRY(cudaMemcpyAsync(bb, pp + 6 * nparts, sizeof(bb), cudaMemcpyDeviceToHost, s));
+    E2F_CUDA_TRY(cudaStreamSynchronize(s));
+    for (int k = 0; k < 6; ++k)
+      if (!(fabsf(bb[k]) < INFINITY)) return E2F_ERR_DOMAIN;
+  }
+  CellGrid cg;
+  double cs[3];
+  for (int k = 0; k < 3; ++k) {
+    if (g.periodic[k]) {
+      const double b = g.box[k];
+      const double cmin = (double)r_c * 1.001 + b * 1e-6;
+      int nc = (int)floor(b / cmin);
+      if (nc < 3) nc = 1;
+      cg.nc[k] = nc;
+      cg.lo[k] = 0.f;
+    } else {
+      const double ext = (double)bb[3 + k] - (double)bb[k];
+      cs[k] = (double)r_c * 1.001 + fabs(ext) * 1e-6 + 1e-6 * fabs((double)bb[k]);
+      cg.lo[k] = bb[k];
+    }
+  }
+  const long long cap = std::min<long long>(std::max<long long>(4096, 8LL * n), NOALLOC_MAX_CELLS);
+  long long ncell = 1;
+  for (int it = 0; it < 256; ++it) {
+    ncell = 1;
+    for (int k = 0; k < 3; ++k) {
+      if (!g.periodic[k]) {
+        const double ext = (double)bb[3 + k] - (double)bb[k];
+        cg.nc[k] = (int)std::min<double>(floor(ext / cs[k]) + 1.0, 1 << 20);
+        cg.inv[k] = (float)(1.0 / cs[k]);
+        cg.stencil[k] = 1;
+      }
+      ncell *= cg.nc[k];
+    }
+    if (ncell <= cap) break;
+    // coarsen: fewer, larger cells (periodic dims below 3 cells use 1)
+    int kmax = 0;
+    for (int k = 1; k < 3; ++k)
+      if (cg.nc[k] > cg.nc[kmax]) kmax = k;
+    if (g.periodic[kmax]) {
+      cg.nc[kmax] = cg.nc[kmax] - 1 < 3 ? 1 : cg.nc[kmax] - 1;
+    } else {
+      cs[kmax] *= 1.25;
+    }
+  }
+  if (ncell > NOALLOC_MAX_CELLS) return E2F_ERR_SCRATCH_LIMIT;
+  for (int k = 0; k < 3; ++k) {
+    if (g.periodic[k]) {
+      cg.inv[k] = (float)(cg.nc[k] / (double)g.box[k]);
+      cg.stencil[k] = cg.nc[k] >= 3 ? 1 : 0;
+    }
+  }
+  int32_t *cell_of = ws + NA_CELL_OF, *abc = ws + NA_ABC, *deg = ws + NA_DEG;
+  int32_t *cnt = ws + NA_CNT, *cstart = ws + NA_CSTART, *cursor = ws + NA_CURSOR, *flag = ws + NA_FLAG;
+  void *scan_tmp = ws + NA_SCAN;
+  E2F_CUDA_TRY(cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ncell, s));
+  E2F_CUDA_TRY(cudaMemsetAsync(cursor, 0, sizeof(int32_t) * ncell, s));
+  E2F_CUDA_TRY(cudaMemsetAsync(flag, 0, sizeof(int32_t) * 4, s));
+  const int tb = 256;
+  E2F_LAUNCH(cell_assign_kernel, (n + tb - 1) / tb, tb, 0, s, pos, n, cg, g, cell_of, cnt, flag);
+  st = exclusive_scan(cnt, ncell, cstart, scan_tmp, s, nullptr);
+  if (st != E2F_OK) return st;
+  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, cell_of, n, cstart, cursor, abc);
+  const int nblk = (n + NB_WARPS - 1) / NB_WARPS;
+  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of, cstart, abc, deg);
+  long long *total = nullptr;
+  st = exclusive_scan(deg, n, row_ptr, scan_tmp, s, &total);
+  if (st != E2F_OK) return st;
+  long long E = 0;
+  int32_t dom = 0;
+  E2F_CUDA_TRY(cudaMemcpyAsync(&E, total, sizeof(long long), cudaMemcpyDeviceToHost, s));
+  E2F_CUDA_TRY(cudaMemcpyAsync(&dom, flag, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  E2F_CUDA_TRY(cudaStreamSynchronize(s));
+  *n_edges = E;
+  if (dom) return E2F_ERR_DOMAIN;
+  if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
+  if (E > capacity) return E2F_ERR_CAPACITY;
+  if (E > 0) {
+    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of, cstart, abc, row_ptr, col_idx);
+  }
+  return E2F_OK;
+}
+
+}  // namespace e2f
+
+extern "C" e2f_status e2f_build_neighbors_noalloc(const float *pos, int64_t N, const float *box, float r_c,
+                                                  int32_t *row_ptr, int32_t *col_idx, int64_t capacity,
+                                                  int64_t *n_edges, e2f_csr *out_csr, void *stream) {
+  using namespace e2f;
+  if (N < 0 || !n_edges || !row_ptr || capacity < 0) return E2F_ERR_INVALID_ARG;
+  if (N > NOALLOC_MAX_ATOMS) return E2F_ERR_SCRATCH_LIMIT;
+  if (N > 0 && !pos) return E2F_ERR_INVALID_ARG;
+  if (capacity > 0 && !col_idx) return E2F_ERR_INVALID_ARG;
+  if (!(r_c > 0.f) || !(r_c < INFINITY)) return E2F_ERR_INVALID_ARG;
+  if (box) {
+    for (int k = 0; k < 3; ++k) {
+      if (!(box[k] >= 0.f) || !(box[k] < INFINITY)) return E2F_ERR_INVALID_ARG;
+      if (box[k] > 0.f && !(r_c < 0.5f * box[k])) return E2F_ERR_CUTOFF_TOO_LARGE;
+    }
+  }
+  e2f_status st = build_neighbors_noalloc_impl(pos, N, box, r_c, row_ptr, col_idx, capacity, n_edges,
+                                               static_cast<cudaStream_t>(stream));
+  if (st != E2F_OK && st != E2F_ERR_CAPACITY) return st;
+  if (out_csr) {
+    out_csr->row_ptr = row_ptr;
+    out_csr->col_idx = col_idx;
+    out_csr->n_nodes = N;
+    out_csr->n_edges = *n_edges;
+    for (int k = 0; k < 3; ++k) out_csr->box[k] = box ? box[k] : 0.f;
+    out_csr->r_c = r_c;
+  }
+  return st;
+}

@@ -21,7 +21,7 @@ MAX_L = 6
 F32, BF16 = 0, 1
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "cutoff too large", 3: "capacity",
-          4: "unsupported", 5: "CUDA error", 6: "timeout", 7: "domain"}
+          4: "unsupported", 5: "CUDA error", 6: "timeout", 7: "domain", 8: "scratch limit"}
 
 
 class E2FError(RuntimeError):
@@ -54,6 +54,10 @@ SIGNATURES = {
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                              ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(Csr),
                                              ctypes.c_void_p]),
+    "e2f_build_neighbors_noalloc": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                                     ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                                     ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                                                     ctypes.POINTER(Csr), ctypes.c_void_p]),
     "e2f_attention_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
                                                ctypes.POINTER(Weights), ctypes.c_void_p, ctypes.c_void_p]),
     "e2f_stream_status": (ctypes.c_int32, [ctypes.c_void_p]),

@@ -56,6 +56,7 @@ typedef int32_t e2f_status;
 #define E2F_ERR_CUDA             5  /* a CUDA runtime call failed (e2f_last_cuda_error) */
 #define E2F_ERR_TIMEOUT          6  /* a bounded device-side wait gave up */
 #define E2F_ERR_DOMAIN           7  /* a coordinate outside [0, box[k]) in a periodic dim */
+#define E2F_ERR_SCRATCH_LIMIT    8  /* input larger than a fixed-scratch entry point allows */
 
 #define E2F_F32  0
 #define E2F_BF16 1
@@ -108,6 +109,34 @@ typedef struct e2f_csr {
 E2F_API e2f_status e2f_build_neighbors(const float *pos, int64_t N, const float *box, float r_c,
                                int32_t *row_ptr, int32_t *col_idx, int64_t capacity,
                                int64_t *n_edges, e2f_csr *out_csr, void *stream);
+
+/*
+ * e2f_build_neighbors_noalloc -- the same CSR as e2f_build_neighbors,
+ * computed without allocating any device memory.  The pages describe no
+ * such call; it is an interface addition for callers that cannot allocate:
+ * MD engines and plugin hosts that reserve the device memory budget once
+ * at start-up and own every later allocation, and step loops that must not
+ * meet an allocation (its failure mode, its implicit synchronisation) in
+ * the middle of a step.
+ *
+ * All temporary arrays live in one fixed array of about 3.2 MB that is part
+ * of the library's device image, so every GPU that loads the library holds
+ * it until the process exits.  The caller still passes pos, row_ptr and
+ * col_idx; arguments, result and status codes are those of
+ * e2f_build_neighbors, plus E2F_ERR_SCRATCH_LIMIT when N > 131072.  The
+ * cell grid is coarsened to at most 131072 cells when needed (same result,
+ * more candidate pairs tested).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call on a device uses the same array and finds the previous call's
+ * contents in it (the call clears what must start at zero); calls whose GPU
+ * work can overlap, e.g. on two streams with no ordering between them,
+ * race on the array and must be serialised by the caller.
+ */
+E2F_API e2f_status e2f_build_neighbors_noalloc(const float *pos, int64_t N, const float *box, float r_c,
+                                               int32_t *row_ptr, int32_t *col_idx, int64_t capacity,
+                                               int64_t *n_edges, e2f_csr *out_csr, void *stream);
 
 /* ---------------------------------------------------------------------------
  * Attention weights.

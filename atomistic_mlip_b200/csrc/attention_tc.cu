@@ -1,14 +1,1050 @@
-// Tensor-core (tcgen05 / TMEM) fused attention -- not built yet; the bf16
-// path runs on the SIMT kernel until this reports availability.
+// Fused on-the-fly equivariant attention on the tensor cores (tcgen05/TMEM).
+//
+// What it computes is the operator of e2f_attention_forward ("E2Former-V2
+// ...", §2.1 EAAS change of basis, §2.2 node-centric streaming with no edge
+// materialisation; "EquiformerV3 ...", §2B.3 envelope in the softmax).
+//
+// Structure (one persistent CTA per SM, 512 threads, contiguous edge range
+// per CTA, tiles of <= 64 edges covering <= 4 destination nodes):
+//
+//   producers (warps 8-15)  per tile: edge geometry, Wigner blocks of the
+//                           y-rotation in the two-angle frame (parity blocks),
+//                           envelope, radial MLP, logits -> alpha (exact
+//                           softmax: per-node max / denominator come from
+//                           a pre-pass, so nothing is rescaled later); then,
+//                           block by block, the rotated neighbour features
+//                           v~ = D v_j written as bf16 MMA operands (one
+//                           64 x 128 "unit" per (degree, +-m)).
+//   loaders (warps 1-2)     stream pre-packed weight tiles (Wr|Wi, or W0)
+//                           from L2 with 1-D bulk copies.
+//   MMA (warp 0)            SO(2) block products as tcgen05.mma (M = 64
+//                           edges, N = 128 channels of one output degree,
+//                           K streamed over the block's units), complex form:
+//                           y+ += v+ Wr^T - v- Wi^T,  y- += v- Wr^T + v+ Wi^T,
+//                           y+ / y- accumulate in the two lane halves of a TMEM
+//                           buffer; then the back-rotation + per-node sum as a
+//                           second GEMM per (l, +-m) group:
+//                           Out_l[c, (slot, m')] += sum_e A[c, e] R[(slot,m'), e]
+//                           with A = alpha g y (bf16) and R = D^l[+-m][m'].
+//   epilogue (warps 4-7)    TMEM y -> A (scaled bf16, shared memory), builds R,
+//                           reads finished nodes' Out columns -> o_i.
+//
+// All waits are bounded; a timeout raises a CTA-wide abort flag and the
+// device error word (E2F_ERR_TIMEOUT) and every role exits its loops.
+#include <algorithm>
+
 #include "common.cuh"
+#include "tc_common.cuh"
+#include "wigner.cuh"
 
 namespace e2f {
+namespace tca {
 
-e2f_status attention_tc_available(const e2f_weights *) { return E2F_ERR_UNSUPPORTED; }
+using namespace tc;
 
-e2f_status attention_tc_impl(const void *, const void *, const void *, const float *, const e2f_csr *,
-                             const e2f_weights *, float *, cudaStream_t, cudaEvent_t, cudaEvent_t) {
-  return E2F_ERR_UNSUPPORTED;
+constexpr int CH = 128;            // channels on this path
+constexpr int TE = 64;             // edges per tile (MMA M)
+constexpr int S = 4;               // destination-node slots per tile
+constexpr int NSTAGE = 2;          // weight ring stages
+constexpr int STAGE_BYTES = 16384;
+constexpr int UNIT_BYTES = TE * CH * 2;
+constexpr int A2_BYTES = CH * TE * 2;
+constexpr int NTHREADS = 512;
+constexpr int HMAX = 16;
+constexpr uint32_t WAIT_LIMIT = 1u << 25;
+
+template <int L> struct Cfg {
+  static constexpr int Q = (L + 1) * (L + 1);
+  static constexpr int P = (L + 1) * (L + 2) / 2;
+  static constexpr int NUNIT = (L + 1 > 2 * L) ? L + 1 : 2 * L;
+  static constexpr int NDYE = (L + 1) * (L + 2) * (2 * L + 3) / 6;   // sum (l+1)^2
+  static constexpr int NDYO = L * (L + 1) * (2 * L + 1) / 6;         // sum l^2
+  static constexpr int NDYP = ((NDYE + NDYO) + 1) & ~1;
+  static constexpr int WIG = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  static __host__ __device__ constexpr int NL(int l) { return ((S * (2 * l + 1) + 15) / 16) * 16; }
+  static __host__ __device__ constexpr int OCB(int l) {
+    int s = 0;
+    for (int k = 0; k < l; ++k) s += NL(k);
+    return s;
+  }
+  static constexpr int NLMAX = NL(L);
+  static constexpr int OUT_COLS = OCB(L + 1);
+  // shared-memory carve-up (bytes)
+  static constexpr size_t OFF_UNIT = 0;
+  static constexpr size_t OFF_W = OFF_UNIT + (size_t)NUNIT * UNIT_BYTES;
+  static constexpr size_t OFF_A2 = OFF_W + (size_t)NSTAGE * STAGE_BYTES;
+  static constexpr size_t OFF_R = OFF_A2 + 2 * (size_t)A2_BYTES;
+  static constexpr size_t OFF_AL = OFF_R + (size_t)NLMAX * TE * 2;
+  static constexpr size_t OFF_DY = OFF_AL + (size_t)TE * HMAX * 4;
+  static constexpr size_t OFF_CS = OFF_DY + (size_t)TE * NDYP * 2;
+  static constexpr size_t OFF_G = OFF_CS + 2 * (size_t)TE * (L > 0 ? L : 1) * 4;
+  static constexpr size_t OFF_GEO = OFF_G + (size_t)TE * P * 4;     // float [TE][4]: ct, st, u, pad
+  static constexpr size_t OFF_J = OFF_GEO + (size_t)TE * 4 * 4;      // int [TE] j, node
+  static constexpr size_t OFF_TILE = OFF_J + 2 * (size_t)TE * 4;     // 8 ints
+  static constexpr size_t OFF_BAR = (OFF_TILE + 32 + 7) & ~(size_t)7;
+  static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 5;
+  static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert((size_t)WIG * 4 * 8 <= UNIT_BYTES, "IR scratch fits one unit");
+  // weight stages per tile
+  static __host__ __device__ constexpr int stages_per_tile() {
+    int s = 0;
+    for (int m = 0; m <= L; ++m) s += (L - m + 1) * (L - m + 1) * 4;
+    return s;
+  }
+};
+
+struct TcArgs {
+  const __nv_bfloat16 *q, *k, *v;
+  const float *pos;
+  Geom g;
+  const int32_t *row_ptr, *col_idx;
+  int N;
+  int64_t E;
+  int H;
+  float inv_sqrt_d;
+  float2 *stats;
+  const uint8_t *wpack;
+  const float *W1, *W2;
+  float *out;
+  int *err;
+};
+
+// ---------------------------------------------------------------------------
+// helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also ORs a predicate over the participating threads, so
+// that every thread of a role takes the same branch (no thread may leave a
+// loop that others still synchronise in).
+__device__ __forceinline__ bool bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+struct Waiter {
+  volatile int *abort_flag;
+  int *err;
+  __device__ bool wait(uint64_t *bar, uint32_t parity) {
+    for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((it & 255) == 255 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicExch(err, E2F_ERR_TIMEOUT);
+    return false;
+  }
+  __device__ bool aborted() const { return *abort_flag != 0; }
+};
+
+struct TileIter {
+  const int32_t *rp;
+  int N;
+  int64_t ebeg, eend;
+  int64_t e0, e1;
+  int n0;
+  __device__ void bounds() {
+    const int nlim = min(n0 + S, N);
+    int64_t e = e0 + TE;
+    if (eend < e) e = eend;
+    if ((int64_t)rp[nlim] < e) e = rp[nlim];
+    e1 = e;
+  }
+  __device__ bool start() {
+    e0 = ebeg;
+    if (e0 >= eend) return false;
+    int lo = 0, hi = N - 1;   // largest n with rp[n] <= e0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((int64_t)rp[mid] <= e0) lo = mid;
+      else hi = mid - 1;
+    }
+    n0 = lo;
+    while ((int64_t)rp[n0 + 1] <= e0) ++n0;
+    bounds();
+    return true;
+  }
+  __device__ bool next() {
+    e0 = e1;
+    if (e0 >= eend) return false;
+    while ((int64_t)rp[n0 + 1] <= e0) ++n0;
+    bounds();
+    return true;
+  }
+};
+
+// D^l of the y-rotation in parity blocks: even rows/cols m >= 0, odd m < 0.
+template <int L> __device__ __forceinline__ int dye_off(int l) { return l * (l + 1) * (2 * l + 1) / 6; }
+template <int L> __device__ __forceinline__ int dyo_off(int l) {
+  return Cfg<L>::NDYE + (l - 1) * l * (2 * l - 1) / 6;
+}
+
+// ---------------------------------------------------------------------------
+// weight packing: per (m, l, lp, kk) stage, 128 x 32 K-major core-matrix
+// tiles (W0 for m = 0; Wr then Wi for m >= 1), in the order the kernel uses.
+// ---------------------------------------------------------------------------
+struct PackArgs {
+  const __nv_bfloat16 *W0;
+  const __nv_bfloat16 *Wr[E2F_MAX_L + 1];
+  const __nv_bfloat16 *Wi[E2F_MAX_L + 1];
+  uint8_t *dst;
+  int L;
+};
+
+__global__ void pack_w_kernel(PackArgs a) {
+  // blockIdx.x = stage index; threadIdx.x = row (128)
+  int stage = blockIdx.x;
+  const int L = a.L;
+  size_t off = 0;
+  int m = 0, l = 0, lp = 0, kk = 0;
+  {
+    int s = stage;
+    bool found = false;
+    for (m = 0; m <= L && !found; ++m) {
+      for (l = m; l <= L && !found; ++l) {
+        for (lp = m; lp <= L && !found; ++lp) {
+          for (kk = 0; kk < 4; ++kk) {
+            if (s == 0) { found = true; break; }
+            off += (m == 0) ? 8192 : 16384;
+            --s;
+          }
+          if (found) break;
+        }
+        if (found) break;
+      }
+      if (found) break;
+    }
+  }
+  const int row = threadIdx.x;
+  const int n = (L - m + 1) * CH;
+  const int srow = (m == 0 ? l : (l - m)) * CH + row;
+  const int scol = (m == 0 ? lp : (lp - m)) * CH + kk * 32;
+  const int ntile = (m == 0) ? 1 : 2;
+  for (int t = 0; t < ntile; ++t) {
+    const __nv_bfloat16 *src = (m == 0) ? a.W0 : (t == 0 ? a.Wr[m] : a.Wi[m]);
+    uint8_t *tile = a.dst + off + (size_t)t * 8192;
+    for (int k = 0; k < 32; ++k)
+      *reinterpret_cast<__nv_bfloat16 *>(tile + kmajor_off(row, k, 32)) = src[(size_t)srow * n + scol + k];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// per-node softmax statistics (max, envelope-weighted denominator) per head
+// ---------------------------------------------------------------------------
+template <int L>
+__device__ __forceinline__ void norm_sh_row0(float ux, float uy, float uz, float *y0) {
+  // Y'_l^m = sqrt(4 pi / (2l+1)) Y_l^m: P_l(z) at m = 0, and
+  // sqrt(2 (l-m)!/(l+m)!) P_l^m(z) {cos, sin}(m phi), no Condon-Shortley phase.
+  const float rho = sqrtf(ux * ux + uy * uy);
+  float cp = 1.f, sp = 0.f;
+  if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
+  float cm[L + 1], sm[L + 1];
+  cm[0] = 1.f; sm[0] = 0.f;
+  for (int m = 1; m <= L; ++m) {
+    cm[m] = cm[m - 1] * cp - sm[m - 1] * sp;
+    sm[m] = sm[m - 1] * cp + cm[m - 1] * sp;
+  }
+  float pmm = 1.f;   // P_m^m
+  for (int m = 0; m <= L; ++m) {
+    if (m > 0) pmm *= (float)(2 * m - 1) * rho;
+    float p_lm2 = 0.f, p_lm1 = pmm;
+    // normalisation sqrt(2 (l-m)!/(l+m)!) built incrementally in l
+    for (int l = m; l <= L; ++l) {
+      float p;
+      if (l == m) p = pmm;
+      else if (l == m + 1) p = uz * (2 * m + 1) * pmm;
+      else p = ((2 * l - 1) * uz * p_lm1 - (l + m - 1) * p_lm2) / (float)(l - m);
+      if (l > m) { p_lm2 = p_lm1; p_lm1 = p; }
+      float nrm = 1.f;
+      if (m > 0) {
+        double f = 2.0;
+        for (int t = l - m + 1; t <= l + m; ++t) f /= (double)t;
+        nrm = (float)sqrt(f);
+      }
+      if (m == 0) y0[l * l + l] = p;
+      else {
+        y0[l * l + l + m] = nrm * p * cm[m];
+        y0[l * l + l - m] = nrm * p * sm[m];
+      }
+    }
+  }
+}
+
+template <int L>
+__global__ void __launch_bounds__(128) node_stats_kernel(TcArgs a) {
+  constexpr int Q = (L + 1) * (L + 1);
+  __shared__ float y0s[32][Q];
+  __shared__ float us[32];
+  __shared__ float sv[32][HMAX];
+  __shared__ float stat_m[HMAX], stat_l[HMAX];
+  const int c = threadIdx.x;
+  const int H = a.H, Ch = CH / H;
+  for (int i = blockIdx.x; i < a.N; i += gridDim.x) {
+    const int r0 = a.row_ptr[i], r1 = a.row_ptr[i + 1];
+    float qreg[Q];
+#pragma unroll
+    for (int t = 0; t < Q; ++t) qreg[t] = __bfloat162float(a.q[((size_t)i * Q + t) * CH + c]);
+    if (c < HMAX) { stat_m[c] = -INFINITY; stat_l[c] = 0.f; }
+    const float3 pi = load_pos(a.pos, i);
+    for (int e0 = r0; e0 < r1; e0 += 32) {
+      const int nb = min(32, r1 - e0);
+      __syncthreads();
+      if (c < nb) {
+        const int j = a.col_idx[e0 + c];
+        float dx, dy, dz;
+        pair_disp(a.g, pi, load_pos(a.pos, j), dx, dy, dz);
+        const float r = sqrtf(dx * dx + dy * dy + dz * dz);
+        float ux = 0.f, uy = 0.f, uz = 1.f;
+        if (r > 0.f) { ux = dx / r; uy = dy / r; uz = dz / r; }
+        norm_sh_row0<L>(ux, uy, uz, y0s[c]);
+        us[c] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+      }
+      __syncthreads();
+      for (int e = 0; e < nb; ++e) {
+        const int j = a.col_idx[e0 + e];
+        const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c;
+        float s = 0.f;
+#pragma unroll
+        for (int l = 0; l <= L; ++l) {
+          float qh = 0.f, kh = 0.f;
+#pragma unroll
+          for (int mp = 0; mp < 2 * l + 1; ++mp) {
+            const float yv = y0s[e][l * l + mp];
+            qh = fmaf(yv, qreg[l * l + mp], qh);
+            kh = fmaf(yv, __bfloat162float(kr[(size_t)(l * l + mp) * CH]), kh);
+          }
+          s = fmaf(qh, kh, s);
+        }
+        for (int o = 1; o < Ch; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (c % Ch == 0) sv[e][c / Ch] = s * a.inv_sqrt_d;
+      }
+      __syncthreads();
+      if (c < H) {
+        float mx = stat_m[c];
+        for (int e = 0; e < nb; ++e) mx = fmaxf(mx, sv[e][c]);
+        const float scale = (stat_m[c] == -INFINITY) ? 0.f : expf(stat_m[c] - mx);
+        float sum = 0.f;
+        for (int e = 0; e < nb; ++e) sum += us[e] * expf(sv[e][c] - mx);
+        stat_l[c] = stat_l[c] * scale + sum;
+        stat_m[c] = mx;
+      }
+    }
+    __syncthreads();
+    if (c < H) a.stats[(size_t)i * H + c] = make_float2(stat_m[c] == -INFINITY ? 0.f : stat_m[c], stat_l[c]);
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the fused kernel
+// ---------------------------------------------------------------------------
+template <int L>
+__global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
+  using Cf = Cfg<L>;
+  constexpr int Q = Cf::Q, P = Cf::P, NUNIT = Cf::NUNIT;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cf::OFF_BAR);
+  uint64_t *unit_full = bars;
+  uint64_t *unit_empty = unit_full + NUNIT;
+  uint64_t *w_full = unit_empty + NUNIT;
+  uint64_t *w_empty = w_full + NSTAGE;
+  uint64_t *y_full = w_empty + NSTAGE;
+  uint64_t *y_empty = y_full + 2;
+  uint64_t *a2r_full = y_empty + 2;
+  uint64_t *rg_done = a2r_full + 2;
+  uint64_t *tile_done = rg_done + 2;
+  uint64_t *slots_clean = tile_done + 1;
+  uint64_t *geo_full = slots_clean + 1;
+  uint64_t *geo_empty = geo_full + 1;
+  uint64_t *mma_drain = geo_empty + 1;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + Cf::NBAR);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+
+  uint8_t *units = smem + Cf::OFF_UNIT;
+  uint8_t *wst = smem + Cf::OFF_W;
+  uint8_t *A2 = smem + Cf::OFF_A2;
+  uint8_t *Rb = smem + Cf::OFF_R;
+  float *al = reinterpret_cast<float *>(smem + Cf::OFF_AL);          // [TE][HMAX]
+  __half *dy = reinterpret_cast<__half *>(smem + Cf::OFF_DY);        // [TE][NDYP]
+  float *csb = reinterpret_cast<float *>(smem + Cf::OFF_CS);         // cos [TE][L], sin [TE][L]
+  float *snb = csb + TE * (L > 0 ? L : 1);
+  float *gs = reinterpret_cast<float *>(smem + Cf::OFF_G);           // [TE][P]
+  float *geo = reinterpret_cast<float *>(smem + Cf::OFF_GEO);        // [TE][4]
+  int *jj = reinterpret_cast<int *>(smem + Cf::OFF_J);               // [TE]
+  int *nodeof = jj + TE;                                             // [TE]
+
+  if (tid == 0) {
+    for (int s = 0; s < NUNIT; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], 1); }
+    for (int s = 0; s < NSTAGE; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&y_full[b], 1); mbar_init(&y_empty[b], 4);
+      mbar_init(&a2r_full[b], 1); mbar_init(&rg_done[b], 1);
+    }
+    mbar_init(tile_done, 1); mbar_init(slots_clean, 4);
+    mbar_init(geo_full, 1); mbar_init(geo_empty, 4);
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) { tmem_alloc(tslot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  Waiter W{abort_flag, a.err};
+
+  TileIter ti;
+  ti.rp = a.row_ptr; ti.N = a.N;
+  ti.ebeg = a.E * (int64_t)blockIdx.x / gridDim.x;
+  ti.eend = a.E * (int64_t)(blockIdx.x + 1) / gridDim.x;
+  const int H = a.H, Ch = CH / H;
+
+  if (warp == 0) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      constexpr uint32_t ID_MAIN = idesc_bf16(64, 128, 0, 0);
+      constexpr uint32_t ID_NEGB = ID_MAIN | (1u << 14);
+      uint32_t st = 0, pc = 0;
+      uint32_t fills[NUNIT];
+      for (int s = 0; s < NUNIT; ++s) fills[s] = 0;
+      uint32_t rgm[2] = {0, 0};
+      const uint32_t s_units = smem_addr(units), s_w = smem_addr(wst), s_a2 = smem_addr(A2), s_r = smem_addr(Rb);
+      int t = 0;
+      bool ok = ti.start();
+      auto rgemm = [&](int m, int l, bool first_in_tile) -> bool {
+        const int ng = (m == 0) ? 1 : 2;
+        for (int sg = 0; sg < ng; ++sg) {
+          if (!W.wait(&a2r_full[sg], rgm[sg] & 1)) return false;
+          if (first_in_tile && sg == 0 && t > 0)
+            if (!W.wait(slots_clean, (t - 1) & 1)) return false;
+          tc_fence_after();
+          const uint32_t id = idesc_bf16(128, Cf::NL(l), 1, 0);
+          const uint32_t d = tbase + 256 + Cf::OCB(l);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc(s_a2 + sg * A2_BYTES + mnmajor_off(0, 16 * kk, 64), 128, 64 * 16);
+            const uint64_t bd = smem_desc(s_r + kmajor_off(0, 16 * kk, 64), 128, 64 * 16);
+            mma_bf16_ss(d, ad, bd, id, 1);
+          }
+          mma_commit(&rg_done[sg]);
+          ++rgm[sg];
+        }
+        return true;
+      };
+      while (ok && !W.aborted()) {
+        int pm = -1, pl = -1;
+        bool first_rg = true;
+        for (int m = 0; m <= L && !W.aborted(); ++m) {
+          for (int l = m; l <= L; ++l) {
+            const uint32_t b = pc & 1;
+            if (!W.wait(&y_empty[b], ((pc >> 1) & 1) ^ 1)) break;
+            tc_fence_after();
+            const bool first_pass = (l == m), last_pass = (l == L);
+            const uint32_t dp = tbase + 128 * b, dmn = tbase + (16u << 16) + 128 * b;
+            bool bad = false;
+            for (int lp = m; lp <= L && !bad; ++lp) {
+              const int sp = (m == 0) ? lp : 2 * (lp - m);
+              if (first_pass) {
+                if (!W.wait(&unit_full[sp], fills[sp] & 1)) { bad = true; break; }
+                if (m > 0 && !W.wait(&unit_full[sp + 1], fills[sp + 1] & 1)) { bad = true; break; }
+                tc_fence_after();
+              }
+              const uint32_t ap = s_units + sp * UNIT_BYTES, am = ap + UNIT_BYTES;
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t s = st % NSTAGE;
+                if (!W.wait(&w_full[s], (st / NSTAGE) & 1)) { bad = true; break; }
+                tc_fence_after();
+                const uint32_t wb = s_w + s * STAGE_BYTES;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                  const int k = kk * 32 + sub * 16;
+                  const uint32_t acc = (lp > m || kk > 0 || sub > 0) ? 1u : 0u;
+                  const uint64_t adp = smem_desc(ap + kmajor_off(0, k, 128), 128, 128 * 16);
+                  const uint64_t bdr = smem_desc(wb + kmajor_off(0, sub * 16, 32), 128, 32 * 16);
+                  if (m == 0) {
+                    mma_bf16_ss(dp, adp, bdr, ID_MAIN, acc);
+                  } else {
+                    const uint64_t adm = smem_desc(am + kmajor_off(0, k, 128), 128, 128 * 16);
+                    const uint64_t bdi = smem_desc(wb + 8192 + kmajor_off(0, sub * 16, 32), 128, 32 * 16);
+                    mma_bf16_ss(dp, adp, bdr, ID_MAIN, acc);
+                    mma_bf16_ss(dp, adm, bdi, ID_NEGB, 1);
+                    mma_bf16_ss(dmn, adm, bdr, ID_MAIN, acc);
+                    mma_bf16_ss(dmn, adp, bdi, ID_MAIN, 1);
+                  }
+                }
+                mma_commit(&w_empty[s]);
+                ++st;
+              }
+              if (bad) break;
+              if (last_pass) {
+                mma_commit(&unit_empty[sp]);
+                ++fills[sp];
+                if (m > 0) { mma_commit(&unit_empty[sp + 1]); ++fills[sp + 1]; }
+              }
+            }
+            if (bad) break;
+            mma_commit(&y_full[b]);
+            ++pc;
+            if (pm >= 0) {
+              if (!rgemm(pm, pl, first_rg)) break;
+              first_rg = false;
+            }
+            pm = m; pl = l;
+          }
+        }
+        if (W.aborted()) break;
+        if (!rgemm(pm, pl, first_rg)) break;
+        mma_commit(tile_done);
+        ++t;
+        ok = ti.next();
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(mma_drain);
+      for (uint32_t it = 0; it < WAIT_LIMIT; ++it)
+        if (mbar_try_wait(mma_drain, 0)) break;
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ======================= weight loaders =======================
+    if (lane == 0) {
+      const int me = warp - 1;
+      constexpr int SPT = Cf::stages_per_tile();
+      uint32_t st = 0;
+      bool ok = ti.start();
+      while (ok && !W.aborted()) {
+        size_t off = 0;
+        int idx = 0;
+        for (int m = 0; m <= L; ++m) {
+          const uint32_t bytes = (m == 0) ? 8192u : 16384u;
+          const int nst = (L - m + 1) * (L - m + 1) * 4;
+          for (int i = 0; i < nst; ++i, ++idx, ++st, off += bytes) {
+            if ((int)(st % 2) != me) continue;
+            const uint32_t s = st % NSTAGE;
+            if (!W.wait(&w_empty[s], ((st / NSTAGE) & 1) ^ 1)) break;
+            mbar_arrive_expect_tx(&w_full[s], bytes);
+            bulk_g2s(wst + s * STAGE_BYTES, a.wpack + off, bytes, &w_full[s]);
+          }
+          if (W.aborted()) break;
+        }
+        (void)SPT;
+        ok = ti.next();
+      }
+      // drain: wait for this loader's last copy so no bulk write lands after exit
+      if (st > 0) {
+        for (uint32_t back = 1; back <= 2 && back <= st; ++back) {
+          const uint32_t s_last = st - back;
+          if ((int)(s_last % 2) != me) continue;
+          const uint32_t s = s_last % NSTAGE;
+          for (uint32_t it = 0; it < WAIT_LIMIT; ++it)
+            if (mbar_try_wait(&w_full[s], (s_last / NSTAGE) & 1)) break;
+        }
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ======================= epilogue =======================
+    const int ew = warp - 4;
+    const int et = tid - 128;   // 0..127
+    const uint32_t lane_base = (uint32_t)(32 * ew) << 16;
+    // zero the Out accumulators
+    {
+      float z[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z[i] = 0.f;
+      for (int c = 0; c < Cf::OUT_COLS; c += 16) tmem_st_32x32b_x16(tbase + lane_base + 256 + c, z);
+      tmem_st_wait();
+      tc_fence_before();
+    }
+    named_bar(1, 128);
+    uint32_t pc = 0, nA[2] = {0, 0};
+    int t = 0;
+    bool dead = false;
+    bool ok = ti.start();
+    while (ok && !dead) {
+      dead = bar_or(1, 128, !W.wait(geo_full, t & 1));
+      if (dead) break;
+      const int ne = (int)(ti.e1 - ti.e0);
+      for (int m = 0; m <= L && !dead; ++m) {
+        for (int l = m; l <= L && !dead; ++l) {
+          const uint32_t b = pc & 1;
+          bool f = !W.wait(&y_full[b], (pc >> 1) & 1);
+          // A2 / R buffers free: the latest R-GEMM of each sign has completed
+          if (!f && nA[0] > 0) f = !W.wait(&rg_done[0], (nA[0] - 1) & 1);
+          if (!f && nA[1] > 0) f = !W.wait(&rg_done[1], (nA[1] - 1) & 1);
+          dead = bar_or(1, 128, f);
+          if (dead) break;
+          tc_fence_after();
+          // ---- y -> A2 (scaled by alpha g, bf16, MN-major [c][e])
+          const int sg = lane >> 4;                // 0: y+ rows, 1: y- rows
+          const int e = 16 * ew + (lane & 15);
+          const bool act = (m > 0 || sg == 0);
+          const int p_ml = m * (L + 1) - m * (m - 1) / 2 + (l - m);
+          const float ge = (e < ne) ? gs[e * P + p_ml] : 0.f;
+          uint8_t *a2 = A2 + sg * A2_BYTES;
+          for (int i = 0; i < 8; ++i) {
+            float v[16];
+            tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i, v);
+            tmem_ld_wait();
+            if (act) {
+              __align__(16) __nv_bfloat16 o[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int c = 16 * i + j;
+                const float sc = (e < ne) ? al[e * HMAX + c / Ch] * ge : 0.f;
+                o[j] = __float2bfloat16_rn(v[j] * sc);
+              }
+              *reinterpret_cast<uint4 *>(a2 + mnmajor_off(16 * i, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
+              *reinterpret_cast<uint4 *>(a2 + mnmajor_off(16 * i + 8, e, 64)) = *reinterpret_cast<uint4 *>(&o[8]);
+            }
+          }
+          fence_async_smem();
+          tc_fence_before();
+          named_bar(1, 128);
+          if (lane == 0) mbar_arrive(&y_empty[b]);
+          // ---- R for each sign, then hand over to the MMA warp
+          const int ng = (m == 0) ? 1 : 2;
+          const int w2 = 2 * l + 1;
+          const int nrow = Cf::NL(l);
+          for (int s2 = 0; s2 < ng; ++s2) {
+            if (s2 == 1) {
+              dead = bar_or(1, 128, !W.wait(&rg_done[0], (nA[0] - 1) & 1));
+              if (dead) break;
+            }
+            // rows (slot, m'), columns edges; entry D^l[sm][m'] for the edge's slot
+            for (int item = et; item < nrow * 8; item += 128) {
+              const int row = item >> 3, e8 = (item & 7) * 8;
+              const int slot = row / w2, mp = row % w2 - l;
+              __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+              for (int t8 = 0; t8 < 8; ++t8) {
+                const int ee = e8 + t8;
+                float val = 0.f;
+                if (row < S * w2 && ee < ne && (nodeof[ee] % S) == slot) {
+                  const __half *d = dy + ee * Cf::NDYP;
+                  const int amp = mp < 0 ? -mp : mp;
+                  if (s2 == 0) {
+                    const float de = __half2float(d[dye_off<L>(l) + m * (l + 1) + amp]);
+                    val = (mp == 0) ? de : (mp > 0 ? de * csb[ee * L + amp - 1] : de * snb[ee * L + amp - 1]);
+                  } else if (mp != 0) {
+                    const float dd = __half2float(d[dyo_off<L>(l) + (m - 1) * l + (amp - 1)]);
+                    val = (mp > 0) ? -dd * snb[ee * L + amp - 1] : dd * csb[ee * L + amp - 1];
+                  }
+                }
+                o[t8] = __float2bfloat16_rn(val);
+              }
+              *reinterpret_cast<uint4 *>(Rb + kmajor_off(row, e8, 64)) = *reinterpret_cast<uint4 *>(o);
+            }
+            fence_async_smem();
+            named_bar(1, 128);
+            if (et == 0) mbar_arrive(&a2r_full[s2]);
+            ++nA[s2];
+          }
+          ++pc;
+        }
+      }
+      if (dead) break;
+      // ---- tile end: read out the nodes that finished here
+      dead = bar_or(1, 128, !W.wait(tile_done, t & 1));
+      if (dead) break;
+      tc_fence_after();
+      {
+        const int n0 = ti.n0;
+        int n1 = ti.n0;
+        while ((int64_t)a.row_ptr[n1 + 1] < ti.e1) ++n1;
+        for (int i = n0; i <= n1; ++i) {
+          const int64_t rb = a.row_ptr[i], re = a.row_ptr[i + 1];
+          if (re == rb) continue;
+          const int64_t reff = re < ti.eend ? re : ti.eend;
+          if (reff > ti.e1) continue;   // continues in the next tile of this CTA
+          const bool shared_node = (rb < ti.ebeg) || (re > ti.eend);
+          const int slot = i % S;
+          float *orow = a.out + (size_t)i * Q * CH + 32 * ew + lane;
+          for (int l = 0; l <= L; ++l) {
+            for (int mp = 0; mp < 2 * l + 1; ++mp) {
+              const uint32_t col = 256 + Cf::OCB(l) + slot * (2 * l + 1) + mp;
+              uint32_t r;
+              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(tbase + lane_base + col));
+              tmem_ld_wait();
+              const float val = __uint_as_float(r);
+              float *dst = orow + (size_t)(l * l + mp) * CH;
+              if (shared_node) atomicAdd(dst, val);
+              else *dst = val;
+              asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col), "r"(0u)
+                           : "memory");
+            }
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      named_bar(1, 128);
+      if (lane == 0) { mbar_arrive(slots_clean); mbar_arrive(geo_empty); }
+      ++t;
+      ok = ti.next();
+    }
+  } else if (warp >= 8) {
+    // ======================= producers =======================
+    const int pt = tid - 256;        // 0..255
+    const int pw = pt >> 5;          // 0..7
+    uint32_t pfill[NUNIT];
+    for (int s = 0; s < NUNIT; ++s) pfill[s] = 0;
+    int t = 0;
+    bool dead = false;
+    bool ok = ti.start();
+    while (ok && !dead) {
+      {
+        bool f = false;
+        if (pt == 0) f = !W.wait(geo_empty, (t & 1) ^ 1);
+        dead = bar_or(2, 256, f || W.aborted());
+        if (dead) break;
+      }
+      const int64_t e0 = ti.e0;
+      const int ne = (int)(ti.e1 - e0);
+      // ---- per-edge basics (thread per edge)
+      if (pt < TE) {
+        const int e = pt;
+        if (e < ne) {
+          const int64_t E = e0 + e;
+          int i = ti.n0;
+          while ((int64_t)a.row_ptr[i + 1] <= E) ++i;
+          const int j = a.col_idx[E];
+          jj[e] = j;
+          nodeof[e] = i;
+          float dx, dyv, dz;
+          pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dyv, dz);
+          const float r = sqrtf(dx * dx + dyv * dyv + dz * dz);
+          float ux = 0.f, uy = 0.f, uz = 1.f;
+          if (r > 0.f) { ux = dx / r; uy = dyv / r; uz = dz / r; }
+          const float rho = sqrtf(ux * ux + uy * uy);
+          float cp = 1.f, sp = 0.f;
+          if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
+          float cm = 1.f, sm = 0.f;
+          for (int mm = 1; mm <= L; ++mm) {
+            const float c2 = cm * cp - sm * sp, s2 = sm * cp + cm * sp;
+            cm = c2; sm = s2;
+            csb[e * L + mm - 1] = cm;
+            snb[e * L + mm - 1] = sm;
+          }
+          geo[e * 4 + 0] = uz;
+          geo[e * 4 + 1] = rho;
+          geo[e * 4 + 2] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+          // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5), 16 SiLU, P outputs
+          float phi[8];
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const float dd = r - (float)kk * (a.g.rc / 7.f);
+            phi[kk] = expf(-dd * dd * 2.f);
+          }
+          float hid[16];
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            float z = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) z = fmaf(a.W1[h * 8 + kk], phi[kk], z);
+            hid[h] = z / (1.f + expf(-z));
+          }
+          for (int p = 0; p < P; ++p) {
+            float gv = 0.f;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) gv = fmaf(a.W2[p * 16 + h], hid[h], gv);
+            gs[e * P + p] = gv;
+          }
+        } else {
+          jj[e] = -1;
+          nodeof[e] = -1;
+          for (int mm = 0; mm < L; ++mm) { csb[e * L + mm] = 1.f; snb[e * L + mm] = 0.f; }
+          geo[e * 4 + 0] = 1.f; geo[e * 4 + 1] = 0.f; geo[e * 4 + 2] = 0.f;
+          for (int p = 0; p < P; ++p) gs[e * P + p] = 0.f;
+        }
+      }
+      named_bar(2, 256);
+      // ---- Wigner blocks of Ry(-theta), lane-parallel per edge, parity blocks -> fp16
+      {
+        float *scr = reinterpret_cast<float *>(units + (size_t)(NUNIT - 1) * UNIT_BYTES) + pw * Cf::WIG;
+        for (int e = pw; e < TE; e += 8) {
+          const float ct = geo[e * 4 + 0], stt = geo[e * 4 + 1];
+          if (lane == 0) {
+            scr[0] = 1.f;
+            // Ry(-theta) = [[ct, 0, -st], [0, 1, 0], [st, 0, ct]] in (x, y, z)
+            const float R[9] = {ct, 0.f, -stt, 0.f, 1.f, 0.f, stt, 0.f, ct};
+            wig_l1_from_rotation(R, scr + 1);
+          }
+          __syncwarp();
+          for (int l = 2; l <= L; ++l) {
+            const int w = 2 * l + 1;
+            for (int x = lane; x < w * w; x += 32)
+              scr[wig_offset(l) + x] = wig_entry(l, x / w - l, x % w - l, scr + 1, scr + wig_offset(l - 1));
+            __syncwarp();
+          }
+          __half *d = dy + e * Cf::NDYP;
+          for (int l = 0; l <= L; ++l) {
+            const int w = 2 * l + 1;
+            const float *Dl = scr + wig_offset(l);
+            for (int x = lane; x < (l + 1) * (l + 1); x += 32) {
+              const int ra = x / (l + 1), cb = x % (l + 1);   // rows/cols m = 0..l
+              d[dye_off<L>(l) + x] = __float2half_rn(Dl[(ra + l) * w + (cb + l)]);
+            }
+            for (int x = lane; x < l * l; x += 32) {
+              const int ra = x / l + 1, cb = x % l + 1;       // rows/cols -m, m = 1..l
+              d[dyo_off<L>(l) + x] = __float2half_rn(Dl[(l - ra) * w + (l - cb)]);
+            }
+          }
+          __syncwarp();
+        }
+      }
+      named_bar(2, 256);
+      // ---- logits -> alpha (warp per edge, lane per 4 channels)
+      for (int e = pw; e < TE; e += 8) {
+        if (e >= ne) {
+          if (lane < HMAX) al[e * HMAX + lane] = 0.f;
+          continue;
+        }
+        const int i = nodeof[e], j = jj[e];
+        const __half *d = dy + e * Cf::NDYP;
+        const int c0 = 4 * lane;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int l = 0; l <= L; ++l) {
+          float qh[4] = {0.f, 0.f, 0.f, 0.f}, kh[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int mp = -l; mp <= l; ++mp) {
+            const int amp = mp < 0 ? -mp : mp;
+            const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
+            const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[e * L + amp - 1] : de * snb[e * L + amp - 1]);
+            const size_t off = (size_t)(l * l + l + mp) * CH + c0;
+            const uint2 qa = *reinterpret_cast<const uint2 *>(a.q + (size_t)i * Q * CH + off);
+            const uint2 ka = *reinterpret_cast<const uint2 *>(a.k + (size_t)j * Q * CH + off);
+            const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qa);
+            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&ka);
+            const float2 qf0 = __bfloat1622float2(q2[0]), qf1 = __bfloat1622float2(q2[1]);
+            const float2 kf0 = __bfloat1622float2(k2[0]), kf1 = __bfloat1622float2(k2[1]);
+            qh[0] = fmaf(coef, qf0.x, qh[0]); qh[1] = fmaf(coef, qf0.y, qh[1]);
+            qh[2] = fmaf(coef, qf1.x, qh[2]); qh[3] = fmaf(coef, qf1.y, qh[3]);
+            kh[0] = fmaf(coef, kf0.x, kh[0]); kh[1] = fmaf(coef, kf0.y, kh[1]);
+            kh[2] = fmaf(coef, kf1.x, kh[2]); kh[3] = fmaf(coef, kf1.y, kh[3]);
+          }
+#pragma unroll
+          for (int x = 0; x < 4; ++x) acc[x] = fmaf(qh[x], kh[x], acc[x]);
+        }
+        float sv = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const int lpg = Ch / 4;   // lanes per head
+        for (int o = 1; o < lpg; o <<= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
+        if (lane % lpg == 0) {
+          const int h = lane / lpg;
+          const float2 stt = a.stats[(size_t)i * H + h];
+          const float u = geo[e * 4 + 2];
+          al[e * HMAX + h] = (stt.y > 0.f) ? u * expf(sv * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
+        }
+      }
+      named_bar(2, 256);
+      if (pt == 0) mbar_arrive(geo_full);
+      // ---- rotate in, block by block
+      for (int m = 0; m <= L && !dead; ++m) {
+        for (int lp = m; lp <= L; ++lp) {
+          const int sp = (m == 0) ? lp : 2 * (lp - m);
+          {
+            bool f = false;
+            if (pt == 0) {
+              f = !W.wait(&unit_empty[sp], (pfill[sp] & 1) ^ 1);
+              if (!f && m > 0) f = !W.wait(&unit_empty[sp + 1], (pfill[sp + 1] & 1) ^ 1);
+            }
+            dead = bar_or(2, 256, f || W.aborted());
+            if (dead) break;
+          }
+          uint8_t *up = units + (size_t)sp * UNIT_BYTES;
+          uint8_t *um = up + UNIT_BYTES;
+          for (int item = pt; item < TE * 8; item += 256) {
+            const int e = item >> 3, cb = (item & 7) * 16;
+            __align__(16) __nv_bfloat16 op[16], om[16];
+            if (e < ne) {
+              const int j = jj[e];
+              const __half *d = dy + e * Cf::NDYP;
+              const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(lp * lp + lp) * CH + cb;
+              float accp[16], accm[16];
+#pragma unroll
+              for (int x = 0; x < 16; ++x) { accp[x] = 0.f; accm[x] = 0.f; }
+              {
+                // k = 0 term (cos-type rows only)
+                const uint4 *src = reinterpret_cast<const uint4 *>(vr);
+                const uint4 r0 = src[0], r1 = src[1];
+                const __nv_bfloat16 *b0 = reinterpret_cast<const __nv_bfloat16 *>(&r0);
+                const __nv_bfloat16 *b1 = reinterpret_cast<const __nv_bfloat16 *>(&r1);
+                const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + 0]);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                  accp[x] = fmaf(de, __bfloat162float(b0[x]), accp[x]);
+                  accp[x + 8] = fmaf(de, __bfloat162float(b1[x]), accp[x + 8]);
+                }
+              }
+              for (int kq = 1; kq <= lp; ++kq) {
+                const uint4 *sp4 = reinterpret_cast<const uint4 *>(vr + (size_t)kq * CH);
+                const uint4 *sm4 = reinterpret_cast<const uint4 *>(vr - (size_t)kq * CH);
+                const uint4 p0 = sp4[0], p1 = sp4[1], n0v = sm4[0], n1v = sm4[1];
+                const __nv_bfloat16 *bp0 = reinterpret_cast<const __nv_bfloat16 *>(&p0);
+                const __nv_bfloat16 *bp1 = reinterpret_cast<const __nv_bfloat16 *>(&p1);
+                const __nv_bfloat16 *bn0 = reinterpret_cast<const __nv_bfloat16 *>(&n0v);
+                const __nv_bfloat16 *bn1 = reinterpret_cast<const __nv_bfloat16 *>(&n1v);
+                const float ck = csb[e * L + kq - 1], sk = snb[e * L + kq - 1];
+                const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + kq]);
+                const float dd = (m > 0) ? __half2float(d[dyo_off<L>(lp) + (m - 1) * lp + (kq - 1)]) : 0.f;
+                // u+ = c v+ + s v-,  u- = -s v+ + c v-
+                const float a_pp = de * ck, a_pm = de * sk;      // into v~(+m)
+                const float a_mp = -dd * sk, a_mm = dd * ck;     // into v~(-m)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                  const float vp0 = __bfloat162float(bp0[x]), vm0 = __bfloat162float(bn0[x]);
+                  const float vp1 = __bfloat162float(bp1[x]), vm1 = __bfloat162float(bn1[x]);
+                  accp[x] = fmaf(a_pp, vp0, fmaf(a_pm, vm0, accp[x]));
+                  accp[x + 8] = fmaf(a_pp, vp1, fmaf(a_pm, vm1, accp[x + 8]));
+                  accm[x] = fmaf(a_mp, vp0, fmaf(a_mm, vm0, accm[x]));
+                  accm[x + 8] = fmaf(a_mp, vp1, fmaf(a_mm, vm1, accm[x + 8]));
+                }
+              }
+#pragma unroll
+              for (int x = 0; x < 16; ++x) { op[x] = __float2bfloat16_rn(accp[x]); om[x] = __float2bfloat16_rn(accm[x]); }
+            } else {
+#pragma unroll
+              for (int x = 0; x < 16; ++x) { op[x] = __float2bfloat16_rn(0.f); om[x] = __float2bfloat16_rn(0.f); }
+            }
+            *reinterpret_cast<uint4 *>(up + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(&op[0]);
+            *reinterpret_cast<uint4 *>(up + kmajor_off(e, cb + 8, 128)) = *reinterpret_cast<uint4 *>(&op[8]);
+            if (m > 0) {
+              *reinterpret_cast<uint4 *>(um + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(&om[0]);
+              *reinterpret_cast<uint4 *>(um + kmajor_off(e, cb + 8, 128)) = *reinterpret_cast<uint4 *>(&om[8]);
+            }
+          }
+          fence_async_smem();
+          named_bar(2, 256);
+          if (pt == 0) {
+            mbar_arrive(&unit_full[sp]);
+            if (m > 0) mbar_arrive(&unit_full[sp + 1]);
+          }
+          ++pfill[sp];
+          if (m > 0) ++pfill[sp + 1];
+        }
+      }
+      if (dead) break;
+      ++t;
+      ok = ti.next();
+    }
+  }
+  // warp 3 idles
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+template <int L>
+static e2f_status launch_tc(const TcArgs &args, int grid, cudaStream_t s) {
+  using Cf = Cfg<L>;
+  E2F_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM));
+  E2F_LAUNCH(attn_tc_kernel<L>, grid, NTHREADS, Cf::SMEM, s, args);
+  return E2F_OK;
+}
+
+template <int L>
+static e2f_status launch_stats(const TcArgs &args, cudaStream_t s) {
+  const int grid = (int)std::min<int64_t>(args.N, 148 * 16);
+  E2F_LAUNCH(node_stats_kernel<L>, grid, 128, 0, s, args);
+  return E2F_OK;
+}
+
+}  // namespace tca
+
+e2f_status attention_tc_available(const e2f_weights *w) {
+  if (w->dtype != E2F_BF16 || w->C != tca::CH) return E2F_ERR_UNSUPPORTED;
+  if (w->L_max < 1 || w->L_max > 4) return E2F_ERR_UNSUPPORTED;
+  // heads of 8..32 channels (the head reductions run inside one warp)
+  if (w->H < 4 || w->H > tca::HMAX || tca::CH % w->H != 0) return E2F_ERR_UNSUPPORTED;
+  return E2F_OK;
+}
+
+e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const float *pos, const e2f_csr *csr,
+                             const e2f_weights *w, float *out, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1) {
+  using namespace tca;
+  const int L = w->L_max;
+  const int64_t N = csr->n_nodes, E = csr->n_edges;
+  const size_t Q = (size_t)(L + 1) * (L + 1);
+  E2F_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)N * Q * CH * sizeof(float), s));
+  if (E == 0) return E2F_OK;
+  // pack weights
+  int nst = 0;
+  size_t wbytes = 0;
+  for (int m = 0; m <= L; ++m) {
+    const int n = (L - m + 1) * (L - m + 1) * 4;
+    nst += n;
+    wbytes += (size_t)n * (m == 0 ? 8192 : 16384);
+  }
+  Scratch wp, st;
+  E2F_CUDA_TRY(wp.alloc(wbytes, s));
+  E2F_CUDA_TRY(st.alloc((size_t)N * w->H * sizeof(float2), s));
+  PackArgs pa;
+  pa.W0 = static_cast<const __nv_bfloat16 *>(w->W0);
+  for (int m = 0; m <= E2F_MAX_L; ++m) {
+    pa.Wr[m] = (m >= 1 && m <= L) ? static_cast<const __nv_bfloat16 *>(w->Wr[m]) : nullptr;
+    pa.Wi[m] = (m >= 1 && m <= L) ? static_cast<const __nv_bfloat16 *>(w->Wi[m]) : nullptr;
+  }
+  pa.dst = wp.as<uint8_t>();
+  pa.L = L;
+  E2F_LAUNCH(pack_w_kernel, nst, 128, 0, s, pa);
+
+  TcArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q);
+  a.k = static_cast<const __nv_bfloat16 *>(k);
+  a.v = static_cast<const __nv_bfloat16 *>(v);
+  a.pos = pos;
+  for (int kk = 0; kk < 3; ++kk) {
+    a.g.box[kk] = csr->box[kk] > 0.f ? csr->box[kk] : 0.f;
+    a.g.half[kk] = 0.5f * a.g.box[kk];
+    a.g.periodic[kk] = csr->box[kk] > 0.f;
+  }
+  a.g.rc = csr->r_c;
+  a.g.rc2 = csr->r_c * csr->r_c;
+  a.row_ptr = csr->row_ptr;
+  a.col_idx = csr->col_idx;
+  a.N = (int)N;
+  a.E = E;
+  a.H = w->H;
+  a.inv_sqrt_d = 1.f / sqrtf((float)((L + 1) * (CH / w->H)));
+  a.stats = st.as<float2>();
+  a.wpack = wp.as<uint8_t>();
+  a.W1 = w->rad_W1;
+  a.W2 = w->rad_W2;
+  a.out = out;
+  a.err = device_error_flag();
+  if (!a.err) return E2F_ERR_CUDA;
+  e2f_status r = E2F_OK;
+  switch (L) {
+    case 1: r = launch_stats<1>(a, s); break;
+    case 2: r = launch_stats<2>(a, s); break;
+    case 3: r = launch_stats<3>(a, s); break;
+    case 4: r = launch_stats<4>(a, s); break;
+    default: return E2F_ERR_UNSUPPORTED;
+  }
+  if (r != E2F_OK) return r;
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(nsm, (E + TE - 1) / TE));
+  if (ev0) E2F_CUDA_TRY(cudaEventRecord(ev0, s));
+  switch (L) {
+    case 1: r = launch_tc<1>(a, grid, s); break;
+    case 2: r = launch_tc<2>(a, grid, s); break;
+    case 3: r = launch_tc<3>(a, grid, s); break;
+    case 4: r = launch_tc<4>(a, grid, s); break;
+    default: return E2F_ERR_UNSUPPORTED;
+  }
+  if (ev1) E2F_CUDA_TRY(cudaEventRecord(ev1, s));
+  return r;
 }
 
 }  // namespace e2f

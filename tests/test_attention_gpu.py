@@ -79,6 +79,28 @@ def test_full_size_sampled_rows(cuda_ok, cfg, prec, n):
     _compare(wl, nodes=nodes)
 
 
+@pytest.mark.parametrize("L", [1, 2, 3, 4])
+def test_tensor_core_path_small(cuda_ok, L):
+    """bf16, C = 128, H = 8 takes the tcgen05 kernel: 24-atom cluster (7 edge
+    tiles, ragged last tile) for every supported degree."""
+    wl0 = wlmod.make_workload(0)
+    wl = wlmod.make_custom(wl0.pos, None, wl0.r_c, L=L, C=128, H=8, precision="bf16", seed=3 + L)
+    _compare(wl)
+
+
+def test_tensor_core_path_isolated_and_low_degree(cuda_ok):
+    """Isolated atoms (empty rows), degree-1 rows and a dense clump in one
+    batch: tiles bounded by the node-slot limit, nodes spanning tiles."""
+    rng = np.random.default_rng(8)
+    clump = rng.uniform(0, 4.0, (90, 3))
+    pairs = np.array([[20, 20, 20], [21, 20, 20], [40, 40, 40], [60, 5, 5]], float)
+    chain = np.stack([np.arange(12) * 1.4 + 80, np.full(12, 80.0), np.full(12, 80.0)], 1)
+    pos = np.concatenate([clump, pairs, chain]).astype(np.float32)
+    wl = wlmod.make_custom(pos, None, 5.0, L=3, C=128, H=4, precision="bf16", seed=9)
+    out, _ = _compare(wl)
+    assert np.all(out[92] == 0) and np.all(out[93] == 0)
+
+
 def test_isolated_atoms_and_coincident(cuda_ok):
     pos = np.array([[0, 0, 0], [50, 50, 50], [1.0, 0.5, 0.2], [1.0, 0.5, 0.2], [0.3, 1.2, 2.0]], np.float32)
     wl = wlmod.make_custom(pos, None, 3.0, L=3, C=16, H=4, precision="fp32", seed=4)

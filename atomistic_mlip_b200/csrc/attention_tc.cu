@@ -74,7 +74,7 @@ template <int L> struct Cfg {
   static constexpr size_t OFF_W = OFF_UNIT + (size_t)NUNIT * UNIT_BYTES;
   static constexpr size_t OFF_A2 = OFF_W + (size_t)NSTAGE * STAGE_BYTES;
   static constexpr size_t OFF_R = OFF_A2 + 2 * (size_t)A2_BYTES;
-  static constexpr size_t OFF_AL = OFF_R + (size_t)NLMAX * TE * 2;
+  static constexpr size_t OFF_AL = OFF_R + 2 * (size_t)NLMAX * TE * 2;
   static constexpr size_t OFF_DY = OFF_AL + (size_t)TE * HMAX * 4;
   static constexpr size_t OFF_CS = OFF_DY + (size_t)TE * NDYP * 2;
   static constexpr size_t OFF_G = OFF_CS + 2 * (size_t)TE * (L > 0 ? L : 1) * 4;
@@ -85,7 +85,8 @@ template <int L> struct Cfg {
   static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 5;
   static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert((size_t)WIG * 4 * 8 <= UNIT_BYTES, "IR scratch fits one unit");
+  static_assert(NUNIT < 3 || (size_t)WIG * 4 * TE <= 3 * (size_t)UNIT_BYTES, "Wigner scratch fits three units");
+  static_assert(NUNIT >= 3 || (size_t)WIG * 4 * TE <= (size_t)NUNIT * UNIT_BYTES, "Wigner scratch fits the units");
   // weight stages per tile
   static __host__ __device__ constexpr int stages_per_tile() {
     int s = 0;
@@ -411,6 +412,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   ti.ebeg = a.E * (int64_t)blockIdx.x / gridDim.x;
   ti.eend = a.E * (int64_t)(blockIdx.x + 1) / gridDim.x;
   const int H = a.H, Ch = CH / H;
+  const int hshift = 31 - __clz(Ch);   // Ch is a power of two
 
   if (warp == 0) {
     // ======================= MMA issuer =======================
@@ -436,7 +438,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = smem_desc(s_a2 + sg * A2_BYTES + mnmajor_off(0, 16 * kk, 64), 128, 64 * 16);
-            const uint64_t bd = smem_desc(s_r + kmajor_off(0, 16 * kk, 64), 128, 64 * 16);
+            const uint64_t bd = smem_desc(s_r + sg * Cf::NLMAX * TE * 2 + kmajor_off(0, 16 * kk, 64), 128, 64 * 16);
             mma_bf16_ss(d, ad, bd, id, 1);
           }
           mma_commit(&rg_done[sg]);
@@ -601,7 +603,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const int c = 16 * i + j;
-                const float sc = (e < ne) ? al[e * HMAX + c / Ch] * ge : 0.f;
+                const float sc = (e < ne) ? al[e * HMAX + (c >> hshift)] * ge : 0.f;
                 o[j] = __float2bfloat16_rn(v[j] * sc);
               }
               *reinterpret_cast<uint4 *>(a2 + mnmajor_off(16 * i, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
@@ -617,10 +619,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const int w2 = 2 * l + 1;
           const int nrow = Cf::NL(l);
           for (int s2 = 0; s2 < ng; ++s2) {
-            if (s2 == 1) {
-              dead = bar_or(1, 128, !W.wait(&rg_done[0], (nA[0] - 1) & 1));
-              if (dead) break;
-            }
+            uint8_t *Rs = Rb + (size_t)s2 * Cf::NLMAX * TE * 2;
             // rows (slot, m'), columns edges; entry D^l[sm][m'] for the edge's slot
             for (int item = et; item < nrow * 8; item += 128) {
               const int row = item >> 3, e8 = (item & 7) * 8;
@@ -643,7 +642,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 }
                 o[t8] = __float2bfloat16_rn(val);
               }
-              *reinterpret_cast<uint4 *>(Rb + kmajor_off(row, e8, 64)) = *reinterpret_cast<uint4 *>(o);
+              *reinterpret_cast<uint4 *>(Rs + kmajor_off(row, e8, 64)) = *reinterpret_cast<uint4 *>(o);
             }
             fence_async_smem();
             named_bar(1, 128);
@@ -654,6 +653,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         }
       }
       if (dead) break;
+      if (lane == 0) mbar_arrive(geo_empty);   // geometry of this tile no longer needed
       // ---- tile end: read out the nodes that finished here
       dead = bar_or(1, 128, !W.wait(tile_done, t & 1));
       if (dead) break;
@@ -670,14 +670,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const bool shared_node = (rb < ti.ebeg) || (re > ti.eend);
           const int slot = i % S;
           float *orow = a.out + (size_t)i * Q * CH + 32 * ew + lane;
+          uint32_t r[Q];
+#pragma unroll
           for (int l = 0; l <= L; ++l) {
+#pragma unroll
             for (int mp = 0; mp < 2 * l + 1; ++mp) {
               const uint32_t col = 256 + Cf::OCB(l) + slot * (2 * l + 1) + mp;
-              uint32_t r;
-              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(tbase + lane_base + col));
-              tmem_ld_wait();
-              const float val = __uint_as_float(r);
+              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
+                           : "=r"(r[l * l + mp])
+                           : "r"(tbase + lane_base + col));
+            }
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int l = 0; l <= L; ++l) {
+#pragma unroll
+            for (int mp = 0; mp < 2 * l + 1; ++mp) {
+              const uint32_t col = 256 + Cf::OCB(l) + slot * (2 * l + 1) + mp;
               float *dst = orow + (size_t)(l * l + mp) * CH;
+              const float val = __uint_as_float(r[l * l + mp]);
               if (shared_node) atomicAdd(dst, val);
               else *dst = val;
               asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col), "r"(0u)
@@ -689,7 +700,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         tc_fence_before();
       }
       named_bar(1, 128);
-      if (lane == 0) { mbar_arrive(slots_clean); mbar_arrive(geo_empty); }
+      if (lane == 0) mbar_arrive(slots_clean);
       ++t;
       ok = ti.next();
     }
@@ -769,77 +780,115 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         }
       }
       named_bar(2, 256);
-      // ---- Wigner blocks of Ry(-theta), lane-parallel per edge, parity blocks -> fp16
+      // ---- Wigner blocks of Ry(-theta): lane = edge, warp = group of entries
+      // (no divergence); entries of opposite parity are zero for a y-rotation.
+      // Scratch: entry-major [entry][edge] floats in the last units (free now).
       {
-        float *scr = reinterpret_cast<float *>(units + (size_t)(NUNIT - 1) * UNIT_BYTES) + pw * Cf::WIG;
-        for (int e = pw; e < TE; e += 8) {
+        const int u0 = NUNIT >= 3 ? NUNIT - 3 : 0;
+        float *scr = reinterpret_cast<float *>(units + (size_t)u0 * UNIT_BYTES);
+        if (pt < TE) {
+          const int e = pt;
           const float ct = geo[e * 4 + 0], stt = geo[e * 4 + 1];
-          if (lane == 0) {
-            scr[0] = 1.f;
-            // Ry(-theta) = [[ct, 0, -st], [0, 1, 0], [st, 0, ct]] in (x, y, z)
-            const float R[9] = {ct, 0.f, -stt, 0.f, 1.f, 0.f, stt, 0.f, ct};
-            wig_l1_from_rotation(R, scr + 1);
-          }
-          __syncwarp();
-          for (int l = 2; l <= L; ++l) {
-            const int w = 2 * l + 1;
-            for (int x = lane; x < w * w; x += 32)
-              scr[wig_offset(l) + x] = wig_entry(l, x / w - l, x % w - l, scr + 1, scr + wig_offset(l - 1));
-            __syncwarp();
-          }
-          __half *d = dy + e * Cf::NDYP;
-          for (int l = 0; l <= L; ++l) {
-            const int w = 2 * l + 1;
-            const float *Dl = scr + wig_offset(l);
-            for (int x = lane; x < (l + 1) * (l + 1); x += 32) {
-              const int ra = x / (l + 1), cb = x % (l + 1);   // rows/cols m = 0..l
-              d[dye_off<L>(l) + x] = __float2half_rn(Dl[(ra + l) * w + (cb + l)]);
-            }
-            for (int x = lane; x < l * l; x += 32) {
-              const int ra = x / l + 1, cb = x % l + 1;       // rows/cols -m, m = 1..l
-              d[dyo_off<L>(l) + x] = __float2half_rn(Dl[(l - ra) * w + (l - cb)]);
+          // Ry(-theta) = [[ct, 0, -st], [0, 1, 0], [st, 0, ct]] in (x, y, z); D^1 in (y, z, x)
+          const float R[9] = {ct, 0.f, -stt, 0.f, 1.f, 0.f, stt, 0.f, ct};
+          float D1[9];
+          wig_l1_from_rotation(R, D1);
+          scr[0 * TE + e] = 1.f;
+#pragma unroll
+          for (int k = 0; k < 9; ++k) scr[(1 + k) * TE + e] = D1[k];
+        }
+        named_bar(2, 256);
+#pragma unroll 1
+        for (int l = 2; l <= L; ++l) {
+          const int w = 2 * l + 1;
+          const float *D1 = scr + 1 * TE;
+          const float *Dp = scr + wig_offset(l - 1) * TE;
+          for (int x = pw; x < w * w; x += 8) {
+            const int m = x / w - l, mp = x % w - l;
+            const bool zero = (m < 0) != (mp < 0);
+            for (int e = lane; e < TE; e += 32) {
+              const float val = zero ? 0.f : wig_entry_s(l, m, mp, D1 + e, Dp + e, TE);
+              scr[(wig_offset(l) + x) * TE + e] = val;
             }
           }
-          __syncwarp();
+          named_bar(2, 256);
+        }
+        // parity blocks -> fp16, thread per (edge, entry)
+        for (int item = pt; item < TE * (Cf::NDYE + Cf::NDYO); item += 256) {
+          const int e = item % TE, x = item / TE;
+          int l = 0, off = 0, val_idx;
+          if (x < Cf::NDYE) {
+            while (off + (l + 1) * (l + 1) <= x) { off += (l + 1) * (l + 1); ++l; }
+            const int r = (x - off) / (l + 1), c = (x - off) % (l + 1);
+            val_idx = wig_offset(l) + (r + l) * (2 * l + 1) + (c + l);
+          } else {
+            const int y = x - Cf::NDYE;
+            l = 1;
+            while (off + l * l <= y) { off += l * l; ++l; }
+            const int r = (y - off) / l + 1, c = (y - off) % l + 1;
+            val_idx = wig_offset(l) + (l - r) * (2 * l + 1) + (l - c);
+          }
+          dy[e * Cf::NDYP + x] = __float2half_rn(scr[val_idx * TE + e]);
         }
       }
       named_bar(2, 256);
-      // ---- logits -> alpha (warp per edge, lane per 4 channels)
-      for (int e = pw; e < TE; e += 8) {
-        if (e >= ne) {
-          if (lane < HMAX) al[e * HMAX + lane] = 0.f;
-          continue;
-        }
-        const int i = nodeof[e], j = jj[e];
-        const __half *d = dy + e * Cf::NDYP;
-        const int c0 = 4 * lane;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int l = 0; l <= L; ++l) {
-          float qh[4] = {0.f, 0.f, 0.f, 0.f}, kh[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int mp = -l; mp <= l; ++mp) {
-            const int amp = mp < 0 ? -mp : mp;
-            const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
-            const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[e * L + amp - 1] : de * snb[e * L + amp - 1]);
-            const size_t off = (size_t)(l * l + l + mp) * CH + c0;
-            const uint2 qa = *reinterpret_cast<const uint2 *>(a.q + (size_t)i * Q * CH + off);
-            const uint2 ka = *reinterpret_cast<const uint2 *>(a.k + (size_t)j * Q * CH + off);
-            const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qa);
-            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&ka);
-            const float2 qf0 = __bfloat1622float2(q2[0]), qf1 = __bfloat1622float2(q2[1]);
-            const float2 kf0 = __bfloat1622float2(k2[0]), kf1 = __bfloat1622float2(k2[1]);
-            qh[0] = fmaf(coef, qf0.x, qh[0]); qh[1] = fmaf(coef, qf0.y, qh[1]);
-            qh[2] = fmaf(coef, qf1.x, qh[2]); qh[3] = fmaf(coef, qf1.y, qh[3]);
-            kh[0] = fmaf(coef, kf0.x, kh[0]); kh[1] = fmaf(coef, kf0.y, kh[1]);
-            kh[2] = fmaf(coef, kf1.x, kh[2]); kh[3] = fmaf(coef, kf1.y, kh[3]);
-          }
+      // ---- logits -> alpha: item = (edge, 8-channel block); loads of one
+      // degree are issued together; partial sums per block go through smem
+      {
+        float *part = reinterpret_cast<float *>(units + (size_t)(NUNIT >= 3 ? NUNIT - 3 : 0) * UNIT_BYTES);  // [TE][16]
+        for (int item = pt; item < TE * 16; item += 256) {
+          const int e = item >> 4, c0 = (item & 15) * 8;
+          float acc = 0.f;
+          if (e < ne) {
+            const int i = nodeof[e], j = jj[e];
+            const __half *d = dy + e * Cf::NDYP;
+            const __nv_bfloat16 *qr = a.q + (size_t)i * Q * CH + c0;
+            const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c0;
+            float accv[8];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) acc[x] = fmaf(qh[x], kh[x], acc[x]);
+            for (int x = 0; x < 8; ++x) accv[x] = 0.f;
+#pragma unroll
+            for (int l = 0; l <= L; ++l) {
+              uint4 qv[2 * L + 1], kv[2 * L + 1];
+#pragma unroll
+              for (int t = 0; t < 2 * l + 1; ++t) {
+                qv[t] = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + t) * CH);
+                kv[t] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + t) * CH);
+              }
+              float qh[8], kh[8];
+#pragma unroll
+              for (int x = 0; x < 8; ++x) { qh[x] = 0.f; kh[x] = 0.f; }
+#pragma unroll
+              for (int t = 0; t < 2 * l + 1; ++t) {
+                const int mp = t - l, amp = mp < 0 ? -mp : mp;
+                const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
+                const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[e * L + amp - 1] : de * snb[e * L + amp - 1]);
+                const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv[t]);
+                const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv[t]);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                  qh[x] = fmaf(coef, __bfloat162float(qb[x]), qh[x]);
+                  kh[x] = fmaf(coef, __bfloat162float(kb[x]), kh[x]);
+                }
+              }
+#pragma unroll
+              for (int x = 0; x < 8; ++x) accv[x] = fmaf(qh[x], kh[x], accv[x]);
+            }
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc += accv[x];
+          }
+          part[e * 16 + (item & 15)] = acc;
         }
-        float sv = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        const int lpg = Ch / 4;   // lanes per head
-        for (int o = 1; o < lpg; o <<= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
-        if (lane % lpg == 0) {
-          const int h = lane / lpg;
+        named_bar(2, 256);
+        // heads: Ch / 8 channel blocks per head
+        for (int item = pt; item < TE * HMAX; item += 256) {
+          const int e = item / HMAX, h = item % HMAX;
+          if (h >= H) continue;
+          if (e >= ne) { al[e * HMAX + h] = 0.f; continue; }
+          const int nb = Ch / 8;
+          float sv = 0.f;
+          for (int x = 0; x < nb; ++x) sv += part[e * 16 + h * nb + x];
+          const int i = nodeof[e];
           const float2 stt = a.stats[(size_t)i * H + h];
           const float u = geo[e * 4 + 2];
           al[e * HMAX + h] = (stt.y > 0.f) ? u * expf(sv * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
@@ -862,65 +911,57 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           }
           uint8_t *up = units + (size_t)sp * UNIT_BYTES;
           uint8_t *um = up + UNIT_BYTES;
-          for (int item = pt; item < TE * 8; item += 256) {
-            const int e = item >> 3, cb = (item & 7) * 16;
-            __align__(16) __nv_bfloat16 op[16], om[16];
+          for (int item = pt; item < TE * 16; item += 256) {
+            const int e = item >> 4, cb = (item & 15) * 8;
+            __align__(16) __nv_bfloat16 op[8], om[8];
             if (e < ne) {
               const int j = jj[e];
               const __half *d = dy + e * Cf::NDYP;
               const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(lp * lp + lp) * CH + cb;
-              float accp[16], accm[16];
+              uint4 vz, vp[L > 0 ? L : 1], vn[L > 0 ? L : 1];
+              vz = *reinterpret_cast<const uint4 *>(vr);
 #pragma unroll
-              for (int x = 0; x < 16; ++x) { accp[x] = 0.f; accm[x] = 0.f; }
+              for (int kq = 1; kq <= L; ++kq) {
+                if (kq <= lp) {
+                  vp[kq - 1] = *reinterpret_cast<const uint4 *>(vr + (size_t)kq * CH);
+                  vn[kq - 1] = *reinterpret_cast<const uint4 *>(vr - (size_t)kq * CH);
+                }
+              }
+              float accp[8], accm[8];
               {
                 // k = 0 term (cos-type rows only)
-                const uint4 *src = reinterpret_cast<const uint4 *>(vr);
-                const uint4 r0 = src[0], r1 = src[1];
-                const __nv_bfloat16 *b0 = reinterpret_cast<const __nv_bfloat16 *>(&r0);
-                const __nv_bfloat16 *b1 = reinterpret_cast<const __nv_bfloat16 *>(&r1);
+                const __nv_bfloat16 *b0 = reinterpret_cast<const __nv_bfloat16 *>(&vz);
                 const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + 0]);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                  accp[x] = fmaf(de, __bfloat162float(b0[x]), accp[x]);
-                  accp[x + 8] = fmaf(de, __bfloat162float(b1[x]), accp[x + 8]);
-                }
+                for (int x = 0; x < 8; ++x) { accp[x] = de * __bfloat162float(b0[x]); accm[x] = 0.f; }
               }
-              for (int kq = 1; kq <= lp; ++kq) {
-                const uint4 *sp4 = reinterpret_cast<const uint4 *>(vr + (size_t)kq * CH);
-                const uint4 *sm4 = reinterpret_cast<const uint4 *>(vr - (size_t)kq * CH);
-                const uint4 p0 = sp4[0], p1 = sp4[1], n0v = sm4[0], n1v = sm4[1];
-                const __nv_bfloat16 *bp0 = reinterpret_cast<const __nv_bfloat16 *>(&p0);
-                const __nv_bfloat16 *bp1 = reinterpret_cast<const __nv_bfloat16 *>(&p1);
-                const __nv_bfloat16 *bn0 = reinterpret_cast<const __nv_bfloat16 *>(&n0v);
-                const __nv_bfloat16 *bn1 = reinterpret_cast<const __nv_bfloat16 *>(&n1v);
-                const float ck = csb[e * L + kq - 1], sk = snb[e * L + kq - 1];
-                const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + kq]);
-                const float dd = (m > 0) ? __half2float(d[dyo_off<L>(lp) + (m - 1) * lp + (kq - 1)]) : 0.f;
-                // u+ = c v+ + s v-,  u- = -s v+ + c v-
-                const float a_pp = de * ck, a_pm = de * sk;      // into v~(+m)
-                const float a_mp = -dd * sk, a_mm = dd * ck;     // into v~(-m)
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                  const float vp0 = __bfloat162float(bp0[x]), vm0 = __bfloat162float(bn0[x]);
-                  const float vp1 = __bfloat162float(bp1[x]), vm1 = __bfloat162float(bn1[x]);
-                  accp[x] = fmaf(a_pp, vp0, fmaf(a_pm, vm0, accp[x]));
-                  accp[x + 8] = fmaf(a_pp, vp1, fmaf(a_pm, vm1, accp[x + 8]));
-                  accm[x] = fmaf(a_mp, vp0, fmaf(a_mm, vm0, accm[x]));
-                  accm[x + 8] = fmaf(a_mp, vp1, fmaf(a_mm, vm1, accm[x + 8]));
+              for (int kq = 1; kq <= L; ++kq) {
+                if (kq <= lp) {
+                  const __nv_bfloat16 *bp = reinterpret_cast<const __nv_bfloat16 *>(&vp[kq - 1]);
+                  const __nv_bfloat16 *bn = reinterpret_cast<const __nv_bfloat16 *>(&vn[kq - 1]);
+                  const float ck = csb[e * L + kq - 1], sk = snb[e * L + kq - 1];
+                  const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + kq]);
+                  const float dd = (m > 0) ? __half2float(d[dyo_off<L>(lp) + (m - 1) * lp + (kq - 1)]) : 0.f;
+                  // u+ = c v+ + s v-,  u- = -s v+ + c v-
+                  const float a_pp = de * ck, a_pm = de * sk;      // into v~(+m)
+                  const float a_mp = -dd * sk, a_mm = dd * ck;     // into v~(-m)
+#pragma unroll
+                  for (int x = 0; x < 8; ++x) {
+                    const float vpx = __bfloat162float(bp[x]), vmx = __bfloat162float(bn[x]);
+                    accp[x] = fmaf(a_pp, vpx, fmaf(a_pm, vmx, accp[x]));
+                    accm[x] = fmaf(a_mp, vpx, fmaf(a_mm, vmx, accm[x]));
+                  }
                 }
               }
 #pragma unroll
-              for (int x = 0; x < 16; ++x) { op[x] = __float2bfloat16_rn(accp[x]); om[x] = __float2bfloat16_rn(accm[x]); }
+              for (int x = 0; x < 8; ++x) { op[x] = __float2bfloat16_rn(accp[x]); om[x] = __float2bfloat16_rn(accm[x]); }
             } else {
 #pragma unroll
-              for (int x = 0; x < 16; ++x) { op[x] = __float2bfloat16_rn(0.f); om[x] = __float2bfloat16_rn(0.f); }
+              for (int x = 0; x < 8; ++x) { op[x] = __float2bfloat16_rn(0.f); om[x] = __float2bfloat16_rn(0.f); }
             }
-            *reinterpret_cast<uint4 *>(up + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(&op[0]);
-            *reinterpret_cast<uint4 *>(up + kmajor_off(e, cb + 8, 128)) = *reinterpret_cast<uint4 *>(&op[8]);
-            if (m > 0) {
-              *reinterpret_cast<uint4 *>(um + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(&om[0]);
-              *reinterpret_cast<uint4 *>(um + kmajor_off(e, cb + 8, 128)) = *reinterpret_cast<uint4 *>(&om[8]);
-            }
+            *reinterpret_cast<uint4 *>(up + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(op);
+            if (m > 0) *reinterpret_cast<uint4 *>(um + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(om);
           }
           fence_async_smem();
           named_bar(2, 256);

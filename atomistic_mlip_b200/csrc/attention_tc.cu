@@ -32,6 +32,7 @@
 // All waits are bounded; a timeout raises a CTA-wide abort flag and the
 // device error word (E2F_ERR_TIMEOUT) and every role exits its loops.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "tc_common.cuh"
@@ -46,36 +47,50 @@ constexpr int CH = 128;            // channels on this path
 constexpr int TE = 64;             // edges per tile (MMA M)
 constexpr int S = 4;               // destination-node slots per tile
 constexpr int NSTAGE = 2;          // weight ring stages
-constexpr int STAGE_BYTES = 16384;
+constexpr int STAGE_BYTES = 32768; // one weight stage: W0 128 x 128, or Wr|Wi 128 x 64 each
 constexpr int UNIT_BYTES = TE * CH * 2;
 constexpr int A2_BYTES = CH * TE * 2;
 constexpr int NTHREADS = 512;
 constexpr int HMAX = 16;
+constexpr int ALS = HMAX + 1;     // alpha row stride (odd: conflict-free per-edge rows)
 constexpr uint32_t WAIT_LIMIT = 1u << 25;
+// TMEM columns: [0, 256) two y buffers (y+ in lanes 0-15, y- in lanes 16-31 of
+// each 32-lane subpartition), [256, 256 + OUT_COLS) the per-node output sums,
+// [384, 512) one rotated-feature unit pair used as the MMA A operand.
+constexpr uint32_t TM_OUT = 256;
+constexpr uint32_t TM_UNIT = 384;
 
 template <int L> struct Cfg {
   static constexpr int Q = (L + 1) * (L + 1);
   static constexpr int P = (L + 1) * (L + 2) / 2;
   static constexpr int NUNIT = (L + 1 > 2 * L) ? L + 1 : 2 * L;
+  // From L = 3 on, the unit pair of (m = 1, l' = L) lives in TMEM: those two
+  // units are used by the m = 1 passes only, and shared memory is tight.
+  static constexpr bool TMU = (L >= 3);
+  static constexpr int TMU_SP = 2 * L - 2;                 // first TMEM unit index
+  static constexpr int NSU = TMU ? NUNIT - 2 : NUNIT;      // units in shared memory
   static constexpr int NDYE = (L + 1) * (L + 2) * (2 * L + 3) / 6;   // sum (l+1)^2
   static constexpr int NDYO = L * (L + 1) * (2 * L + 1) / 6;         // sum l^2
   static constexpr int NDYP = ((NDYE + NDYO) + 1) & ~1;
   static constexpr int WIG = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  // Output-sum columns: the R-GEMM of degree l writes NL(l) columns from
+  // OB(l); its S (2l+1) real columns start RO(l) into that block, the rest of
+  // the block only ever receives exact zeros (zero rows of R), so real
+  // columns of another degree may sit there.
   static __host__ __device__ constexpr int NL(int l) { return ((S * (2 * l + 1) + 15) / 16) * 16; }
-  static __host__ __device__ constexpr int OCB(int l) {
-    int s = 0;
-    for (int k = 0; k < l; ++k) s += NL(k);
-    return s;
+  static __host__ __device__ constexpr int OB(int l) {
+    return l <= 1 ? 0 : (l == 2 ? (L >= 3 ? 32 : 16) : (l == 3 ? 16 : 64));
   }
+  static __host__ __device__ constexpr int RO(int l) { return l == 0 ? 12 : (l == 2 && L >= 3 ? 12 : 0); }
+  static constexpr int OUT_COLS = L == 1 ? 16 : (L == 2 ? 48 : (L == 3 ? 64 : 112));
   static constexpr int NLMAX = NL(L);
-  static constexpr int OUT_COLS = OCB(L + 1);
   // shared-memory carve-up (bytes)
   static constexpr size_t OFF_UNIT = 0;
-  static constexpr size_t OFF_W = OFF_UNIT + (size_t)NUNIT * UNIT_BYTES;
+  static constexpr size_t OFF_W = OFF_UNIT + (size_t)NSU * UNIT_BYTES;
   static constexpr size_t OFF_A2 = OFF_W + (size_t)NSTAGE * STAGE_BYTES;
   static constexpr size_t OFF_R = OFF_A2 + 2 * (size_t)A2_BYTES;
   static constexpr size_t OFF_AL = OFF_R + 2 * (size_t)NLMAX * TE * 2;
-  static constexpr size_t OFF_DY = OFF_AL + (size_t)TE * HMAX * 4;
+  static constexpr size_t OFF_DY = OFF_AL + (size_t)TE * ALS * 4;
   static constexpr size_t OFF_CS = OFF_DY + (size_t)TE * NDYP * 2;
   static constexpr size_t OFF_G = OFF_CS + 2 * (size_t)TE * (L > 0 ? L : 1) * 4;
   static constexpr size_t OFF_GEO = OFF_G + (size_t)TE * P * 4;     // float [TE][4]: ct, st, u, pad
@@ -85,12 +100,12 @@ template <int L> struct Cfg {
   static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 5;
   static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(NUNIT < 3 || (size_t)WIG * 4 * TE <= 3 * (size_t)UNIT_BYTES, "Wigner scratch fits three units");
-  static_assert(NUNIT >= 3 || (size_t)WIG * 4 * TE <= (size_t)NUNIT * UNIT_BYTES, "Wigner scratch fits the units");
+  static_assert(TM_OUT + OUT_COLS <= TM_UNIT, "TMEM budget");
   // weight stages per tile
+  static __host__ __device__ constexpr int stages_of_m(int m) { return (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2); }
   static __host__ __device__ constexpr int stages_per_tile() {
     int s = 0;
-    for (int m = 0; m <= L; ++m) s += (L - m + 1) * (L - m + 1) * 4;
+    for (int m = 0; m <= L; ++m) s += stages_of_m(m);
     return s;
   }
 };
@@ -136,10 +151,14 @@ __device__ __forceinline__ bool bar_or(int id, int nthreads, bool pred) {
 struct Waiter {
   volatile int *abort_flag;
   int *err;
-  __device__ bool wait(uint64_t *bar, uint32_t parity) {
+  // sleep_ns > 0: back off between polls, so that a waiting warp leaves the
+  // issue slots of its scheduler to the warps that share it (the MMA issuer
+  // polls without sleeping).
+  __device__ bool wait(uint64_t *bar, uint32_t parity, uint32_t sleep_ns = 0) {
     for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
       if (mbar_try_wait(bar, parity)) return true;
       if ((it & 255) == 255 && *abort_flag) return false;
+      if (sleep_ns) __nanosleep(sleep_ns);
     }
     *abort_flag = 1;
     atomicExch(err, E2F_ERR_TIMEOUT);
@@ -191,8 +210,10 @@ template <int L> __device__ __forceinline__ int dyo_off(int l) {
 }
 
 // ---------------------------------------------------------------------------
-// weight packing: per (m, l, lp, kk) stage, 128 x 32 K-major core-matrix
-// tiles (W0 for m = 0; Wr then Wi for m >= 1), in the order the kernel uses.
+// weight packing: one 32 KB stage per (m, l, l', half), in the order the MMA
+// warp consumes them.  m = 0: W0 rows of degree l, columns of degree l'
+// (128 x 128, K-major core matrices, Kc = 128).  m >= 1: Wr then Wi rows of
+// degree l, columns of degree l', K half `kh` (128 x 64 each, Kc = 64).
 // ---------------------------------------------------------------------------
 struct PackArgs {
   const __nv_bfloat16 *W0;
@@ -204,39 +225,125 @@ struct PackArgs {
 
 __global__ void pack_w_kernel(PackArgs a) {
   // blockIdx.x = stage index; threadIdx.x = row (128)
-  int stage = blockIdx.x;
   const int L = a.L;
-  size_t off = 0;
-  int m = 0, l = 0, lp = 0, kk = 0;
-  {
-    int s = stage;
-    bool found = false;
-    for (m = 0; m <= L && !found; ++m) {
-      for (l = m; l <= L && !found; ++l) {
-        for (lp = m; lp <= L && !found; ++lp) {
-          for (kk = 0; kk < 4; ++kk) {
-            if (s == 0) { found = true; break; }
-            off += (m == 0) ? 8192 : 16384;
-            --s;
-          }
-          if (found) break;
-        }
-        if (found) break;
-      }
-      if (found) break;
-    }
+  int s = blockIdx.x;
+  int m = 0;
+  for (;; ++m) {
+    const int n = (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
+    if (s < n) break;
+    s -= n;
   }
+  const int nk = (m == 0) ? 1 : 2;
+  const int kh = s % nk;
+  const int l = m + (s / nk) / (L - m + 1), lp = m + (s / nk) % (L - m + 1);
+  uint8_t *stage = a.dst + (size_t)blockIdx.x * STAGE_BYTES;
   const int row = threadIdx.x;
   const int n = (L - m + 1) * CH;
-  const int srow = (m == 0 ? l : (l - m)) * CH + row;
-  const int scol = (m == 0 ? lp : (lp - m)) * CH + kk * 32;
-  const int ntile = (m == 0) ? 1 : 2;
-  for (int t = 0; t < ntile; ++t) {
-    const __nv_bfloat16 *src = (m == 0) ? a.W0 : (t == 0 ? a.Wr[m] : a.Wi[m]);
-    uint8_t *tile = a.dst + off + (size_t)t * 8192;
-    for (int k = 0; k < 32; ++k)
-      *reinterpret_cast<__nv_bfloat16 *>(tile + kmajor_off(row, k, 32)) = src[(size_t)srow * n + scol + k];
+  const size_t srow = (size_t)(l - m) * CH + row;
+  if (m == 0) {
+    const int scol = lp * CH;
+    for (int k = 0; k < 128; ++k)
+      *reinterpret_cast<__nv_bfloat16 *>(stage + kmajor_off(row, k, 128)) = a.W0[srow * n + scol + k];
+  } else {
+    const int scol = (lp - m) * CH + kh * 64;
+    for (int t = 0; t < 2; ++t) {
+      const __nv_bfloat16 *src = (t == 0) ? a.Wr[m] : a.Wi[m];
+      for (int k = 0; k < 64; ++k)
+        *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = src[srow * n + scol + k];
+    }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Wigner blocks of the y-rotation Ry(-theta) as polynomials.  In the real
+// basis, D^l(Ry(-theta))[m][m'] is zero unless m and m' have the same sign
+// (m = 0 counting as cos-type), and otherwise equals
+//   sin(theta)^eps * sum_j c_j cos(theta)^j,   eps = (|m| + |m'|) mod 2,
+// a polynomial of degree l - eps (the half-angle powers of the Wigner
+// small-d sum pair up into cos and sin of the full angle).  The coefficients
+// are fitted once on the host, in double, to the Ivanic-Ruedenberg recursion
+// of the same rotation (exact up to rounding: the fit is interpolation of a
+// polynomial of known degree) and kept in constant memory; a residual above
+// 1e-9 at any sample aborts the fit.
+// Table entry of (l, m, m'): DYP_STRIDE floats at
+// DYP_STRIDE * (wig_offset(l) + (m + l)(2l + 1) + (m' + l)): [eps, c_0, .., c_l].
+// ---------------------------------------------------------------------------
+constexpr int DYP_STRIDE = E2F_MAX_L + 2;
+constexpr int DYP_ENTRIES = (E2F_MAX_L + 1) * (2 * E2F_MAX_L + 1) * (2 * E2F_MAX_L + 3) / 3;  // sum (2l+1)^2
+__constant__ float c_dypoly[DYP_ENTRIES * DYP_STRIDE];
+
+static bool fit_dy_poly(float *tab) {
+  constexpr int L = E2F_MAX_L, K = 4 * (L + 1);
+  static double D[K][DYP_ENTRIES];
+  double ct[K], st[K];
+  for (int k = 0; k < K; ++k) {
+    const double th = 3.14159265358979323846 * (k + 0.5) / K;
+    ct[k] = cos(th); st[k] = sin(th);
+    const double R[9] = {ct[k], 0.0, -st[k], 0.0, 1.0, 0.0, st[k], 0.0, ct[k]};
+    wig_all_serial<double>(R, L, D[k]);
+  }
+  for (int l = 0; l <= L; ++l) {
+    const int w = 2 * l + 1;
+    for (int m = -l; m <= l; ++m)
+      for (int mp = -l; mp <= l; ++mp) {
+        const int idx = wig_offset(l) + (m + l) * w + (mp + l);
+        float *out = tab + (size_t)DYP_STRIDE * idx;
+        for (int j = 0; j < DYP_STRIDE; ++j) out[j] = 0.f;
+        if ((m < 0) != (mp < 0)) continue;
+        const int eps = ((m < 0 ? -m : m) + (mp < 0 ? -mp : mp)) & 1;
+        const int nc = l - eps + 1;
+        // normal equations of the least-squares fit (nc <= 7), solved by
+        // Gaussian elimination with partial pivoting
+        double A[8][9] = {};
+        for (int k = 0; k < K; ++k) {
+          double basis[8];
+          double pw = eps ? st[k] : 1.0;
+          for (int j = 0; j < nc; ++j) { basis[j] = pw; pw *= ct[k]; }
+          for (int i = 0; i < nc; ++i) {
+            for (int j = 0; j < nc; ++j) A[i][j] += basis[i] * basis[j];
+            A[i][nc] += basis[i] * D[k][idx];
+          }
+        }
+        for (int c = 0; c < nc; ++c) {
+          int piv = c;
+          for (int r = c + 1; r < nc; ++r)
+            if (fabs(A[r][c]) > fabs(A[piv][c])) piv = r;
+          for (int j = 0; j <= nc; ++j) { const double t = A[c][j]; A[c][j] = A[piv][j]; A[piv][j] = t; }
+          for (int r = 0; r < nc; ++r) {
+            if (r == c) continue;
+            const double f = A[r][c] / A[c][c];
+            for (int j = c; j <= nc; ++j) A[r][j] -= f * A[c][j];
+          }
+        }
+        double coef[8];
+        for (int j = 0; j < nc; ++j) coef[j] = A[j][nc] / A[j][j];
+        for (int k = 0; k < K; ++k) {
+          double pw = eps ? st[k] : 1.0, v = 0.0;
+          for (int j = 0; j < nc; ++j) { v += coef[j] * pw; pw *= ct[k]; }
+          if (fabs(v - D[k][idx]) > 1e-9) return false;
+        }
+        out[0] = (float)eps;
+        for (int j = 0; j < nc; ++j) out[1 + j] = (float)coef[j];
+      }
+  }
+  return true;
+}
+
+// Uploads the table to the current device once.
+static e2f_status ensure_dy_poly() {
+  static float tab[DYP_ENTRIES * DYP_STRIDE];
+  static int fitted = 0;   // 0: not yet, 1: ok, -1: failed
+  static bool uploaded[64] = {};
+  if (fitted == 0) fitted = fit_dy_poly(tab) ? 1 : -1;
+  if (fitted < 0) return E2F_ERR_CUDA;
+  int dev = 0;
+  E2F_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
+  if (!uploaded[dev]) {
+    E2F_CUDA_TRY(cudaMemcpyToSymbol(c_dypoly, tab, sizeof(tab)));
+    uploaded[dev] = true;
+  }
+  return E2F_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -377,7 +484,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   uint8_t *wst = smem + Cf::OFF_W;
   uint8_t *A2 = smem + Cf::OFF_A2;
   uint8_t *Rb = smem + Cf::OFF_R;
-  float *al = reinterpret_cast<float *>(smem + Cf::OFF_AL);          // [TE][HMAX]
+  float *al = reinterpret_cast<float *>(smem + Cf::OFF_AL);          // [TE][ALS]
   __half *dy = reinterpret_cast<__half *>(smem + Cf::OFF_DY);        // [TE][NDYP]
   float *csb = reinterpret_cast<float *>(smem + Cf::OFF_CS);         // cos [TE][L], sin [TE][L]
   float *snb = csb + TE * (L > 0 ? L : 1);
@@ -420,36 +527,41 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       constexpr uint32_t ID_MAIN = idesc_bf16(64, 128, 0, 0);
       constexpr uint32_t ID_NEGB = ID_MAIN | (1u << 14);
       uint32_t st = 0, pc = 0;
-      uint32_t fills[NUNIT];
-      for (int s = 0; s < NUNIT; ++s) fills[s] = 0;
-      uint32_t rgm[2] = {0, 0};
+      uint32_t fillpar = 0;        // bit sp: parity of unit sp's fill count
+      uint32_t rgpar = 0;          // bit sg: parity of the R-GEMMs issued for sign sg
       const uint32_t s_units = smem_addr(units), s_w = smem_addr(wst), s_a2 = smem_addr(A2), s_r = smem_addr(Rb);
+      const uint64_t ud0 = smem_desc(s_units, 128, 128 * 16);   // unit 0, K-major, Kc = 128
+      const uint64_t wd128 = smem_desc(s_w, 128, 128 * 16);     // stage 0 as 128 x 128 (m = 0)
+      const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 2 x 128 x 64 (m >= 1)
+      const uint64_t a2d = smem_desc(s_a2, 128, 64 * 16);       // A2, MN-major, K = 64 edges
+      const uint64_t rd = smem_desc(s_r, 128, 64 * 16);         // R, K-major, K = 64 edges
       int t = 0;
       bool ok = ti.start();
       auto rgemm = [&](int m, int l, bool first_in_tile) -> bool {
         const int ng = (m == 0) ? 1 : 2;
+        #pragma unroll 1
         for (int sg = 0; sg < ng; ++sg) {
-          if (!W.wait(&a2r_full[sg], rgm[sg] & 1)) return false;
+          if (!W.wait(&a2r_full[sg], (rgpar >> sg) & 1)) return false;
           if (first_in_tile && sg == 0 && t > 0)
             if (!W.wait(slots_clean, (t - 1) & 1)) return false;
           tc_fence_after();
           const uint32_t id = idesc_bf16(128, Cf::NL(l), 1, 0);
-          const uint32_t d = tbase + 256 + Cf::OCB(l);
+          const uint32_t d = tbase + TM_OUT + Cf::OB(l);
+          const uint64_t ad = a2d + (uint64_t)sg * (A2_BYTES >> 4);
+          const uint64_t bd = rd + (uint64_t)sg * ((Cf::NLMAX * TE * 2) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(s_a2 + sg * A2_BYTES + mnmajor_off(0, 16 * kk, 64), 128, 64 * 16);
-            const uint64_t bd = smem_desc(s_r + sg * Cf::NLMAX * TE * 2 + kmajor_off(0, 16 * kk, 64), 128, 64 * 16);
-            mma_bf16_ss(d, ad, bd, id, 1);
-          }
+          for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, ad + 16 * kk, bd + 16 * kk, id, 1u);
           mma_commit(&rg_done[sg]);
-          ++rgm[sg];
+          rgpar ^= 1u << sg;
         }
         return true;
       };
       while (ok && !W.aborted()) {
         int pm = -1, pl = -1;
         bool first_rg = true;
+        #pragma unroll 1
         for (int m = 0; m <= L && !W.aborted(); ++m) {
+          #pragma unroll 1
           for (int l = m; l <= L; ++l) {
             const uint32_t b = pc & 1;
             if (!W.wait(&y_empty[b], ((pc >> 1) & 1) ^ 1)) break;
@@ -457,34 +569,52 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             const bool first_pass = (l == m), last_pass = (l == L);
             const uint32_t dp = tbase + 128 * b, dmn = tbase + (16u << 16) + 128 * b;
             bool bad = false;
+            #pragma unroll 1
             for (int lp = m; lp <= L && !bad; ++lp) {
               const int sp = (m == 0) ? lp : 2 * (lp - m);
               if (first_pass) {
-                if (!W.wait(&unit_full[sp], fills[sp] & 1)) { bad = true; break; }
-                if (m > 0 && !W.wait(&unit_full[sp + 1], fills[sp + 1] & 1)) { bad = true; break; }
+                if (!W.wait(&unit_full[sp], (fillpar >> sp) & 1)) { bad = true; break; }
+                if (m > 0 && !W.wait(&unit_full[sp + 1], (fillpar >> (sp + 1)) & 1)) { bad = true; break; }
                 tc_fence_after();
               }
-              const uint32_t ap = s_units + sp * UNIT_BYTES, am = ap + UNIT_BYTES;
-              for (int kk = 0; kk < 4; ++kk) {
+              const bool in_tmem = Cf::TMU && sp >= Cf::NSU;
+              // descriptors advance by (byte offset >> 4): 16 per 16-wide K step
+              const uint64_t adp = ud0 + (uint64_t)sp * (UNIT_BYTES >> 4), adm = adp + (UNIT_BYTES >> 4);
+              const int nk = (m == 0) ? 1 : 2;
+              #pragma unroll 1
+              for (int kh = 0; kh < nk; ++kh) {
                 const uint32_t s = st % NSTAGE;
                 if (!W.wait(&w_full[s], (st / NSTAGE) & 1)) { bad = true; break; }
                 tc_fence_after();
-                const uint32_t wb = s_w + s * STAGE_BYTES;
+                const uint32_t acc0 = (lp > m || kh > 0) ? 1u : 0u;
+                if (m == 0) {
+                  const uint64_t bd = wd128 + (uint64_t)s * (STAGE_BYTES >> 4);
+                  mma_bf16_ss(dp, adp, bd, ID_MAIN, acc0);
 #pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                  const int k = kk * 32 + sub * 16;
-                  const uint32_t acc = (lp > m || kk > 0 || sub > 0) ? 1u : 0u;
-                  const uint64_t adp = smem_desc(ap + kmajor_off(0, k, 128), 128, 128 * 16);
-                  const uint64_t bdr = smem_desc(wb + kmajor_off(0, sub * 16, 32), 128, 32 * 16);
-                  if (m == 0) {
-                    mma_bf16_ss(dp, adp, bdr, ID_MAIN, acc);
+                  for (int sub = 1; sub < 8; ++sub) mma_bf16_ss(dp, adp + 16 * sub, bd + 16 * sub, ID_MAIN, 1u);
+                } else {
+                  const uint64_t br = wd64 + (uint64_t)s * (STAGE_BYTES >> 4), bi = br + (16384 >> 4);
+                  if (in_tmem) {
+                    // lane half 0 holds [v+ | v-], lane half 1 holds [v- | v+]
+                    const uint32_t a0 = tbase + TM_UNIT + 32 * kh, a1 = a0 + (16u << 16);
+#pragma unroll
+                    for (int sub = 0; sub < 4; ++sub) {
+                      const uint32_t acc = sub > 0 ? 1u : acc0;
+                      mma_bf16_ts(dp, a0 + 8 * sub, br + 16 * sub, ID_MAIN, acc);
+                      mma_bf16_ts(dp, a0 + 64 + 8 * sub, bi + 16 * sub, ID_NEGB, 1u);
+                      mma_bf16_ts(dmn, a1 + 8 * sub, br + 16 * sub, ID_MAIN, acc);
+                      mma_bf16_ts(dmn, a1 + 64 + 8 * sub, bi + 16 * sub, ID_MAIN, 1u);
+                    }
                   } else {
-                    const uint64_t adm = smem_desc(am + kmajor_off(0, k, 128), 128, 128 * 16);
-                    const uint64_t bdi = smem_desc(wb + 8192 + kmajor_off(0, sub * 16, 32), 128, 32 * 16);
-                    mma_bf16_ss(dp, adp, bdr, ID_MAIN, acc);
-                    mma_bf16_ss(dp, adm, bdi, ID_NEGB, 1);
-                    mma_bf16_ss(dmn, adm, bdr, ID_MAIN, acc);
-                    mma_bf16_ss(dmn, adp, bdi, ID_MAIN, 1);
+                    const uint64_t ap = adp + 64 * kh, am = adm + 64 * kh;
+#pragma unroll
+                    for (int sub = 0; sub < 4; ++sub) {
+                      const uint32_t acc = sub > 0 ? 1u : acc0;
+                      mma_bf16_ss(dp, ap + 16 * sub, br + 16 * sub, ID_MAIN, acc);
+                      mma_bf16_ss(dp, am + 16 * sub, bi + 16 * sub, ID_NEGB, 1u);
+                      mma_bf16_ss(dmn, am + 16 * sub, br + 16 * sub, ID_MAIN, acc);
+                      mma_bf16_ss(dmn, ap + 16 * sub, bi + 16 * sub, ID_MAIN, 1u);
+                    }
                   }
                 }
                 mma_commit(&w_empty[s]);
@@ -493,8 +623,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               if (bad) break;
               if (last_pass) {
                 mma_commit(&unit_empty[sp]);
-                ++fills[sp];
-                if (m > 0) { mma_commit(&unit_empty[sp + 1]); ++fills[sp + 1]; }
+                fillpar ^= 1u << sp;
+                if (m > 0) { mma_commit(&unit_empty[sp + 1]); fillpar ^= 1u << (sp + 1); }
               }
             }
             if (bad) break;
@@ -526,21 +656,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       uint32_t st = 0;
       bool ok = ti.start();
       while (ok && !W.aborted()) {
-        size_t off = 0;
-        int idx = 0;
-        for (int m = 0; m <= L; ++m) {
-          const uint32_t bytes = (m == 0) ? 8192u : 16384u;
-          const int nst = (L - m + 1) * (L - m + 1) * 4;
-          for (int i = 0; i < nst; ++i, ++idx, ++st, off += bytes) {
-            if ((int)(st % 2) != me) continue;
-            const uint32_t s = st % NSTAGE;
-            if (!W.wait(&w_empty[s], ((st / NSTAGE) & 1) ^ 1)) break;
-            mbar_arrive_expect_tx(&w_full[s], bytes);
-            bulk_g2s(wst + s * STAGE_BYTES, a.wpack + off, bytes, &w_full[s]);
-          }
-          if (W.aborted()) break;
+        for (int i = 0; i < SPT; ++i, ++st) {
+          if ((int)(st % 2) != me) continue;
+          const uint32_t s = st % NSTAGE;
+          if (!W.wait(&w_empty[s], ((st / NSTAGE) & 1) ^ 1, 20)) break;
+          mbar_arrive_expect_tx(&w_full[s], STAGE_BYTES);
+          bulk_g2s(wst + s * STAGE_BYTES, a.wpack + (size_t)i * STAGE_BYTES, STAGE_BYTES, &w_full[s]);
         }
-        (void)SPT;
+        if (W.aborted()) break;
         ok = ti.next();
       }
       // drain: wait for this loader's last copy so no bulk write lands after exit
@@ -564,26 +687,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       float z[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) z[i] = 0.f;
-      for (int c = 0; c < Cf::OUT_COLS; c += 16) tmem_st_32x32b_x16(tbase + lane_base + 256 + c, z);
+      for (int c = 0; c < Cf::OUT_COLS; c += 16) tmem_st_32x32b_x16(tbase + lane_base + TM_OUT + c, z);
       tmem_st_wait();
       tc_fence_before();
     }
     named_bar(1, 128);
-    uint32_t pc = 0, nA[2] = {0, 0};
+    uint32_t pc = 0, nA0 = 0, nA1 = 0;   // R hand-overs per sign
     int t = 0;
     bool dead = false;
     bool ok = ti.start();
     while (ok && !dead) {
-      dead = bar_or(1, 128, !W.wait(geo_full, t & 1));
+      dead = bar_or(1, 128, et == 0 && !W.wait(geo_full, t & 1, 100));
       if (dead) break;
       const int ne = (int)(ti.e1 - ti.e0);
+      #pragma unroll 1
       for (int m = 0; m <= L && !dead; ++m) {
+        #pragma unroll 1
         for (int l = m; l <= L && !dead; ++l) {
           const uint32_t b = pc & 1;
-          bool f = !W.wait(&y_full[b], (pc >> 1) & 1);
-          // A2 / R buffers free: the latest R-GEMM of each sign has completed
-          if (!f && nA[0] > 0) f = !W.wait(&rg_done[0], (nA[0] - 1) & 1);
-          if (!f && nA[1] > 0) f = !W.wait(&rg_done[1], (nA[1] - 1) & 1);
+          bool f = false;
+          // y ready, and the A2 / R buffers free: the latest R-GEMM of each
+          // sign has completed (one thread polls, the barrier hands it over)
+          if (et == 0) {
+            f = !W.wait(&y_full[b], (pc >> 1) & 1, 40);
+            if (!f && nA0 > 0) f = !W.wait(&rg_done[0], (nA0 - 1) & 1, 40);
+            if (!f && nA1 > 0) f = !W.wait(&rg_done[1], (nA1 - 1) & 1, 40);
+          }
           dead = bar_or(1, 128, f);
           if (dead) break;
           tc_fence_after();
@@ -594,20 +723,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const int p_ml = m * (L + 1) - m * (m - 1) / 2 + (l - m);
           const float ge = (e < ne) ? gs[e * P + p_ml] : 0.f;
           uint8_t *a2 = A2 + sg * A2_BYTES;
-          for (int i = 0; i < 8; ++i) {
-            float v[16];
-            tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i, v);
+#pragma unroll 1
+          for (int i = 0; i < 8; i += 2) {
+            float v[2][16];
+            tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i, v[0]);
+            tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i + 16, v[1]);
             tmem_ld_wait();
             if (act) {
-              __align__(16) __nv_bfloat16 o[16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int c = 16 * i + j;
-                const float sc = (e < ne) ? al[e * HMAX + (c >> hshift)] * ge : 0.f;
-                o[j] = __float2bfloat16_rn(v[j] * sc);
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int c0 = 16 * (i + h2);
+                // channels [c0, c0 + 8) and [c0 + 8, c0 + 16) lie in one head each
+                const float s_lo = (e < ne) ? al[e * ALS + (c0 >> hshift)] * ge : 0.f;
+                const float s_hi = (e < ne) ? al[e * ALS + ((c0 + 8) >> hshift)] * ge : 0.f;
+                __align__(16) __nv_bfloat16 o[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(v[h2][j] * (j < 8 ? s_lo : s_hi));
+                *reinterpret_cast<uint4 *>(a2 + mnmajor_off(c0, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
+                *reinterpret_cast<uint4 *>(a2 + mnmajor_off(c0 + 8, e, 64)) = *reinterpret_cast<uint4 *>(&o[8]);
               }
-              *reinterpret_cast<uint4 *>(a2 + mnmajor_off(16 * i, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
-              *reinterpret_cast<uint4 *>(a2 + mnmajor_off(16 * i + 8, e, 64)) = *reinterpret_cast<uint4 *>(&o[8]);
             }
           }
           fence_async_smem();
@@ -618,18 +752,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const int ng = (m == 0) ? 1 : 2;
           const int w2 = 2 * l + 1;
           const int nrow = Cf::NL(l);
+          #pragma unroll 1
           for (int s2 = 0; s2 < ng; ++s2) {
             uint8_t *Rs = Rb + (size_t)s2 * Cf::NLMAX * TE * 2;
             // rows (slot, m'), columns edges; entry D^l[sm][m'] for the edge's slot
+            const int ro = Cf::RO(l);
             for (int item = et; item < nrow * 8; item += 128) {
               const int row = item >> 3, e8 = (item & 7) * 8;
-              const int slot = row / w2, mp = row % w2 - l;
+              const int rr = row - ro;
+              const int slot = rr / w2, mp = rr - slot * w2 - l;
               __align__(16) __nv_bfloat16 o[8];
 #pragma unroll
               for (int t8 = 0; t8 < 8; ++t8) {
                 const int ee = e8 + t8;
                 float val = 0.f;
-                if (row < S * w2 && ee < ne && (nodeof[ee] % S) == slot) {
+                if (rr >= 0 && rr < S * w2 && ee < ne && (nodeof[ee] % S) == slot) {
                   const __half *d = dy + ee * Cf::NDYP;
                   const int amp = mp < 0 ? -mp : mp;
                   if (s2 == 0) {
@@ -647,7 +784,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             fence_async_smem();
             named_bar(1, 128);
             if (et == 0) mbar_arrive(&a2r_full[s2]);
-            ++nA[s2];
+            if (s2 == 0) ++nA0; else ++nA1;
           }
           ++pc;
         }
@@ -655,7 +792,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       if (dead) break;
       if (lane == 0) mbar_arrive(geo_empty);   // geometry of this tile no longer needed
       // ---- tile end: read out the nodes that finished here
-      dead = bar_or(1, 128, !W.wait(tile_done, t & 1));
+      dead = bar_or(1, 128, et == 0 && !W.wait(tile_done, t & 1, 40));
       if (dead) break;
       tc_fence_after();
       {
@@ -675,7 +812,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           for (int l = 0; l <= L; ++l) {
 #pragma unroll
             for (int mp = 0; mp < 2 * l + 1; ++mp) {
-              const uint32_t col = 256 + Cf::OCB(l) + slot * (2 * l + 1) + mp;
+              const uint32_t col = TM_OUT + Cf::OB(l) + Cf::RO(l) + slot * (2 * l + 1) + mp;
               asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
                            : "=r"(r[l * l + mp])
                            : "r"(tbase + lane_base + col));
@@ -686,7 +823,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           for (int l = 0; l <= L; ++l) {
 #pragma unroll
             for (int mp = 0; mp < 2 * l + 1; ++mp) {
-              const uint32_t col = 256 + Cf::OCB(l) + slot * (2 * l + 1) + mp;
+              const uint32_t col = TM_OUT + Cf::OB(l) + Cf::RO(l) + slot * (2 * l + 1) + mp;
               float *dst = orow + (size_t)(l * l + mp) * CH;
               const float val = __uint_as_float(r[l * l + mp]);
               if (shared_node) atomicAdd(dst, val);
@@ -708,153 +845,154 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     // ======================= producers =======================
     const int pt = tid - 256;        // 0..255
     const int pw = pt >> 5;          // 0..7
-    uint32_t pfill[NUNIT];
-    for (int s = 0; s < NUNIT; ++s) pfill[s] = 0;
+    uint32_t pfillpar = 0;   // bit sp: parity of unit sp's fill count
     int t = 0;
     bool dead = false;
     bool ok = ti.start();
     while (ok && !dead) {
       {
         bool f = false;
-        if (pt == 0) f = !W.wait(geo_empty, (t & 1) ^ 1);
+        if (pt == 0) f = !W.wait(geo_empty, (t & 1) ^ 1, 100);
         dead = bar_or(2, 256, f || W.aborted());
         if (dead) break;
       }
       const int64_t e0 = ti.e0;
       const int ne = (int)(ti.e1 - e0);
-      // ---- per-edge basics (thread per edge)
-      if (pt < TE) {
-        const int e = pt;
-        if (e < ne) {
+      // ---- per-edge basics: four threads per edge (consecutive lanes); the
+      // first computes the frame, all four share the radial MLP (hidden units
+      // 4q..4q+3 each, outputs reduced with shuffles)
+      {
+        const int e = pt >> 2, q4 = pt & 3;
+        const bool live = e < ne;
+        float r = 0.f;
+        if (live) {
           const int64_t E = e0 + e;
           int i = ti.n0;
           while ((int64_t)a.row_ptr[i + 1] <= E) ++i;
           const int j = a.col_idx[E];
-          jj[e] = j;
-          nodeof[e] = i;
           float dx, dyv, dz;
           pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dyv, dz);
-          const float r = sqrtf(dx * dx + dyv * dyv + dz * dz);
-          float ux = 0.f, uy = 0.f, uz = 1.f;
-          if (r > 0.f) { ux = dx / r; uy = dyv / r; uz = dz / r; }
-          const float rho = sqrtf(ux * ux + uy * uy);
-          float cp = 1.f, sp = 0.f;
-          if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
-          float cm = 1.f, sm = 0.f;
-          for (int mm = 1; mm <= L; ++mm) {
-            const float c2 = cm * cp - sm * sp, s2 = sm * cp + cm * sp;
-            cm = c2; sm = s2;
-            csb[e * L + mm - 1] = cm;
-            snb[e * L + mm - 1] = sm;
+          r = sqrtf(dx * dx + dyv * dyv + dz * dz);
+          if (q4 == 0) {
+            jj[e] = j;
+            nodeof[e] = i;
+            float ux = 0.f, uy = 0.f, uz = 1.f;
+            if (r > 0.f) { ux = dx / r; uy = dyv / r; uz = dz / r; }
+            const float rho = sqrtf(ux * ux + uy * uy);
+            float cp = 1.f, sp = 0.f;
+            if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
+            float cm = 1.f, sm = 0.f;
+            for (int mm = 1; mm <= L; ++mm) {
+              const float c2 = cm * cp - sm * sp, s2 = sm * cp + cm * sp;
+              cm = c2; sm = s2;
+              csb[e * L + mm - 1] = cm;
+              snb[e * L + mm - 1] = sm;
+            }
+            geo[e * 4 + 0] = uz;
+            geo[e * 4 + 1] = rho;
+            geo[e * 4 + 2] = 0.5f * (cospif(r / a.g.rc) + 1.f);
           }
-          geo[e * 4 + 0] = uz;
-          geo[e * 4 + 1] = rho;
-          geo[e * 4 + 2] = 0.5f * (cospif(r / a.g.rc) + 1.f);
-          // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5), 16 SiLU, P outputs
-          float phi[8];
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const float dd = r - (float)kk * (a.g.rc / 7.f);
-            phi[kk] = expf(-dd * dd * 2.f);
-          }
-          float hid[16];
-#pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            float z = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) z = fmaf(a.W1[h * 8 + kk], phi[kk], z);
-            hid[h] = z / (1.f + expf(-z));
-          }
-          for (int p = 0; p < P; ++p) {
-            float gv = 0.f;
-#pragma unroll
-            for (int h = 0; h < 16; ++h) gv = fmaf(a.W2[p * 16 + h], hid[h], gv);
-            gs[e * P + p] = gv;
-          }
-        } else {
+        } else if (q4 == 0) {
           jj[e] = -1;
           nodeof[e] = -1;
           for (int mm = 0; mm < L; ++mm) { csb[e * L + mm] = 1.f; snb[e * L + mm] = 0.f; }
           geo[e * 4 + 0] = 1.f; geo[e * 4 + 1] = 0.f; geo[e * 4 + 2] = 0.f;
-          for (int p = 0; p < P; ++p) gs[e * P + p] = 0.f;
         }
-      }
-      named_bar(2, 256);
-      // ---- Wigner blocks of Ry(-theta): lane = edge, warp = group of entries
-      // (no divergence); entries of opposite parity are zero for a y-rotation.
-      // Scratch: entry-major [entry][edge] floats in the last units (free now).
-      {
-        const int u0 = NUNIT >= 3 ? NUNIT - 3 : 0;
-        float *scr = reinterpret_cast<float *>(units + (size_t)u0 * UNIT_BYTES);
-        if (pt < TE) {
-          const int e = pt;
-          const float ct = geo[e * 4 + 0], stt = geo[e * 4 + 1];
-          // Ry(-theta) = [[ct, 0, -st], [0, 1, 0], [st, 0, ct]] in (x, y, z); D^1 in (y, z, x)
-          const float R[9] = {ct, 0.f, -stt, 0.f, 1.f, 0.f, stt, 0.f, ct};
-          float D1[9];
-          wig_l1_from_rotation(R, D1);
-          scr[0 * TE + e] = 1.f;
+        // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5), 16 SiLU, P outputs
+        float phi[8];
 #pragma unroll
-          for (int k = 0; k < 9; ++k) scr[(1 + k) * TE + e] = D1[k];
+        for (int kk = 0; kk < 8; ++kk) {
+          const float dd = r - (float)kk * (a.g.rc / 7.f);
+          phi[kk] = expf(-dd * dd * 2.f);
         }
-        named_bar(2, 256);
-#pragma unroll 1
-        for (int l = 2; l <= L; ++l) {
-          const int w = 2 * l + 1;
-          const float *D1 = scr + 1 * TE;
-          const float *Dp = scr + wig_offset(l - 1) * TE;
-          for (int x = pw; x < w * w; x += 8) {
-            const int m = x / w - l, mp = x % w - l;
-            const bool zero = (m < 0) != (mp < 0);
-            for (int e = lane; e < TE; e += 32) {
-              const float val = zero ? 0.f : wig_entry_s(l, m, mp, D1 + e, Dp + e, TE);
-              scr[(wig_offset(l) + x) * TE + e] = val;
-            }
-          }
-          named_bar(2, 256);
+        float hid[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float z = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) z = fmaf(__ldg(a.W1 + (4 * q4 + h) * 8 + kk), phi[kk], z);
+          hid[h] = z / (1.f + expf(-z));
         }
-        // parity blocks -> fp16, thread per (edge, entry)
-        for (int item = pt; item < TE * (Cf::NDYE + Cf::NDYO); item += 256) {
-          const int e = item % TE, x = item / TE;
-          int l = 0, off = 0, val_idx;
-          if (x < Cf::NDYE) {
-            while (off + (l + 1) * (l + 1) <= x) { off += (l + 1) * (l + 1); ++l; }
-            const int r = (x - off) / (l + 1), c = (x - off) % (l + 1);
-            val_idx = wig_offset(l) + (r + l) * (2 * l + 1) + (c + l);
-          } else {
-            const int y = x - Cf::NDYE;
-            l = 1;
-            while (off + l * l <= y) { off += l * l; ++l; }
-            const int r = (y - off) / l + 1, c = (y - off) % l + 1;
-            val_idx = wig_offset(l) + (l - r) * (2 * l + 1) + (l - c);
-          }
-          dy[e * Cf::NDYP + x] = __float2half_rn(scr[val_idx * TE + e]);
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+          float gv = 0.f;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) gv = fmaf(__ldg(a.W2 + p * 16 + 4 * q4 + h), hid[h], gv);
+          gv += __shfl_xor_sync(0xffffffffu, gv, 1);
+          gv += __shfl_xor_sync(0xffffffffu, gv, 2);
+          if ((p & 3) == q4) gs[e * P + p] = live ? gv : 0.f;
         }
       }
       named_bar(2, 256);
-      // ---- logits -> alpha: item = (edge, 8-channel block); loads of one
-      // degree are issued together; partial sums per block go through smem
+      // ---- Wigner blocks of Ry(-theta), parity blocks straight to fp16:
+      // warp = entry (coefficients broadcast from constant memory), lane = edge
+      for (int x = pw; x < Cf::NDYE + Cf::NDYO; x += 8) {
+        int l = 0, off = 0, m, mp;
+        if (x < Cf::NDYE) {
+          while (off + (l + 1) * (l + 1) <= x) { off += (l + 1) * (l + 1); ++l; }
+          m = (x - off) / (l + 1);
+          mp = (x - off) % (l + 1);
+        } else {
+          const int y = x - Cf::NDYE;
+          l = 1;
+          while (off + l * l <= y) { off += l * l; ++l; }
+          m = -((y - off) / l + 1);
+          mp = -((y - off) % l + 1);
+        }
+        const float *cf = c_dypoly + DYP_STRIDE * (wig_offset(l) + (m + l) * (2 * l + 1) + (mp + l));
+        float c[L + 1];
+#pragma unroll
+        for (int jd = 0; jd <= L; ++jd) c[jd] = cf[1 + jd];   // zero above the entry's degree
+        const bool eps = cf[0] != 0.f;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int e = lane + 32 * h2;
+          const float ct = geo[e * 4 + 0], stt = geo[e * 4 + 1];
+          float p = c[L];
+#pragma unroll
+          for (int jd = L - 1; jd >= 0; --jd) p = fmaf(p, ct, c[jd]);
+          dy[e * Cf::NDYP + x] = __float2half_rn(eps ? p * stt : p);
+        }
+      }
+      named_bar(2, 256);
+      // ---- logits -> alpha: item = (edge, 8-channel block).  The q rows of
+      // the tile's (<= S) destination nodes are staged in shared memory (the
+      // unit area is free while a tile's geometry is built); the gathered k
+      // rows are loaded in two batches of degrees.  The blocks of one head are
+      // summed with shuffles (16 consecutive lanes = one edge's 16 blocks).
+      __nv_bfloat16 *sq = reinterpret_cast<__nv_bfloat16 *>(units);   // [S][Q][CH]
       {
-        float *part = reinterpret_cast<float *>(units + (size_t)(NUNIT >= 3 ? NUNIT - 3 : 0) * UNIT_BYTES);  // [TE][16]
+        constexpr int NQV = S * Q * CH / 8;   // uint4 count
+        constexpr int PER = (NQV + 255) / 256;
+        uint4 tmp[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int idx = pt + 256 * k;
+          const int node = ti.n0 + idx / (Q * CH / 8);
+          if (idx < NQV && node < a.N)
+            tmp[k] = *reinterpret_cast<const uint4 *>(a.q + (size_t)ti.n0 * Q * CH + (size_t)idx * 8);
+        }
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int idx = pt + 256 * k;
+          const int node = ti.n0 + idx / (Q * CH / 8);
+          if (idx < NQV && node < a.N) reinterpret_cast<uint4 *>(sq)[idx] = tmp[k];
+        }
+      }
+      named_bar(2, 256);
+      {
         for (int item = pt; item < TE * 16; item += 256) {
           const int e = item >> 4, c0 = (item & 15) * 8;
           float acc = 0.f;
           if (e < ne) {
             const int i = nodeof[e], j = jj[e];
             const __half *d = dy + e * Cf::NDYP;
-            const __nv_bfloat16 *qr = a.q + (size_t)i * Q * CH + c0;
+            const __nv_bfloat16 *qr = sq + (size_t)(i - ti.n0) * Q * CH + c0;
             const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c0;
             float accv[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) accv[x] = 0.f;
-#pragma unroll
-            for (int l = 0; l <= L; ++l) {
-              uint4 qv[2 * L + 1], kv[2 * L + 1];
-#pragma unroll
-              for (int t = 0; t < 2 * l + 1; ++t) {
-                qv[t] = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + t) * CH);
-                kv[t] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + t) * CH);
-              }
+            auto degree = [&](int l, const uint4 *kv) {
               float qh[8], kh[8];
 #pragma unroll
               for (int x = 0; x < 8; ++x) { qh[x] = 0.f; kh[x] = 0.f; }
@@ -863,7 +1001,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 const int mp = t - l, amp = mp < 0 ? -mp : mp;
                 const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
                 const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[e * L + amp - 1] : de * snb[e * L + amp - 1]);
-                const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv[t]);
+                const uint4 qv = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + t) * CH);
+                const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
                 const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv[t]);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
@@ -873,95 +1012,190 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               }
 #pragma unroll
               for (int x = 0; x < 8; ++x) accv[x] = fmaf(qh[x], kh[x], accv[x]);
+            };
+            constexpr int LB = (L + 2) / 2;          // degrees [0, LB) then [LB, L]
+            {
+              uint4 kv[LB * LB];
+#pragma unroll
+              for (int t = 0; t < LB * LB; ++t) kv[t] = *reinterpret_cast<const uint4 *>(kr + (size_t)t * CH);
+#pragma unroll
+              for (int l = 0; l < LB; ++l) degree(l, kv + l * l);
+            }
+            {
+              uint4 kv[Q - LB * LB];
+#pragma unroll
+              for (int t = 0; t < Q - LB * LB; ++t) kv[t] = *reinterpret_cast<const uint4 *>(kr + (size_t)(LB * LB + t) * CH);
+#pragma unroll
+              for (int l = LB; l <= L; ++l) degree(l, kv + (l * l - LB * LB));
             }
 #pragma unroll
             for (int x = 0; x < 8; ++x) acc += accv[x];
           }
-          part[e * 16 + (item & 15)] = acc;
-        }
-        named_bar(2, 256);
-        // heads: Ch / 8 channel blocks per head
-        for (int item = pt; item < TE * HMAX; item += 256) {
-          const int e = item / HMAX, h = item % HMAX;
-          if (h >= H) continue;
-          if (e >= ne) { al[e * HMAX + h] = 0.f; continue; }
-          const int nb = Ch / 8;
-          float sv = 0.f;
-          for (int x = 0; x < nb; ++x) sv += part[e * 16 + h * nb + x];
-          const int i = nodeof[e];
-          const float2 stt = a.stats[(size_t)i * H + h];
-          const float u = geo[e * 4 + 2];
-          al[e * HMAX + h] = (stt.y > 0.f) ? u * expf(sv * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
+          const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
+          for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          const int blk = item & 15;
+          if ((blk & (nb - 1)) == 0) {
+            const int h = blk / nb;
+            float alpha = 0.f;
+            if (e < ne) {
+              const float2 stt = a.stats[(size_t)nodeof[e] * H + h];
+              const float u = geo[e * 4 + 2];
+              alpha = (stt.y > 0.f) ? u * expf(acc * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
+            }
+            al[e * ALS + h] = alpha;
+          }
         }
       }
       named_bar(2, 256);
       if (pt == 0) mbar_arrive(geo_full);
       // ---- rotate in, block by block
+      #pragma unroll 1
       for (int m = 0; m <= L && !dead; ++m) {
+        #pragma unroll 1
         for (int lp = m; lp <= L; ++lp) {
           const int sp = (m == 0) ? lp : 2 * (lp - m);
           {
             bool f = false;
             if (pt == 0) {
-              f = !W.wait(&unit_empty[sp], (pfill[sp] & 1) ^ 1);
-              if (!f && m > 0) f = !W.wait(&unit_empty[sp + 1], (pfill[sp + 1] & 1) ^ 1);
+              f = !W.wait(&unit_empty[sp], ((pfillpar >> sp) & 1) ^ 1, 40);
+              if (!f && m > 0) f = !W.wait(&unit_empty[sp + 1], ((pfillpar >> (sp + 1)) & 1) ^ 1, 40);
             }
             dead = bar_or(2, 256, f || W.aborted());
             if (dead) break;
           }
-          uint8_t *up = units + (size_t)sp * UNIT_BYTES;
-          uint8_t *um = up + UNIT_BYTES;
-          for (int item = pt; item < TE * 16; item += 256) {
-            const int e = item >> 4, cb = (item & 15) * 8;
-            __align__(16) __nv_bfloat16 op[8], om[8];
-            if (e < ne) {
-              const int j = jj[e];
-              const __half *d = dy + e * Cf::NDYP;
-              const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(lp * lp + lp) * CH + cb;
-              uint4 vz, vp[L > 0 ? L : 1], vn[L > 0 ? L : 1];
-              vz = *reinterpret_cast<const uint4 *>(vr);
+          // v~(+m), v~(-m) of edge e for two 8-channel blocks of degree l'
+          // (all gathered rows of both blocks are loaded before any use)
+          // (degree l' as a compile-time constant: register use follows the degree)
+          auto rot2 = [&](auto LPc, int e, int cbA, int cbB, __nv_bfloat16 (&op)[2][8], __nv_bfloat16 (&om)[2][8]) {
+            constexpr int LP = decltype(LPc)::value;
+            if (e >= ne) {
+#pragma unroll
+              for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) { op[q2][x] = __float2bfloat16_rn(0.f); om[q2][x] = __float2bfloat16_rn(0.f); }
+              return;
+            }
+            const int j = jj[e];
+            const __half *d = dy + e * Cf::NDYP;
+            const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(LP * LP + LP) * CH;
+            const int cbs[2] = {cbA, cbB};
+            uint4 vz[2], vp[2][L > 0 ? L : 1], vn[2][L > 0 ? L : 1];
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+              vz[q2] = *reinterpret_cast<const uint4 *>(vr + cbs[q2]);
 #pragma unroll
               for (int kq = 1; kq <= L; ++kq) {
-                if (kq <= lp) {
-                  vp[kq - 1] = *reinterpret_cast<const uint4 *>(vr + (size_t)kq * CH);
-                  vn[kq - 1] = *reinterpret_cast<const uint4 *>(vr - (size_t)kq * CH);
+                if (kq <= LP) {
+                  vp[q2][kq - 1] = *reinterpret_cast<const uint4 *>(vr + (size_t)kq * CH + cbs[q2]);
+                  vn[q2][kq - 1] = *reinterpret_cast<const uint4 *>(vr - (size_t)kq * CH + cbs[q2]);
                 }
               }
-              float accp[8], accm[8];
-              {
-                // k = 0 term (cos-type rows only)
-                const __nv_bfloat16 *b0 = reinterpret_cast<const __nv_bfloat16 *>(&vz);
-                const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + 0]);
+            }
+            float accp[2][8], accm[2][8];
+            {
+              // k = 0 term (cos-type rows only)
+              const float de = __half2float(d[dye_off<L>(LP) + m * (LP + 1) + 0]);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) { accp[x] = de * __bfloat162float(b0[x]); accm[x] = 0.f; }
+              for (int q2 = 0; q2 < 2; ++q2) {
+                const __nv_bfloat16 *b0 = reinterpret_cast<const __nv_bfloat16 *>(&vz[q2]);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) { accp[q2][x] = de * __bfloat162float(b0[x]); accm[q2][x] = 0.f; }
               }
+            }
 #pragma unroll
-              for (int kq = 1; kq <= L; ++kq) {
-                if (kq <= lp) {
-                  const __nv_bfloat16 *bp = reinterpret_cast<const __nv_bfloat16 *>(&vp[kq - 1]);
-                  const __nv_bfloat16 *bn = reinterpret_cast<const __nv_bfloat16 *>(&vn[kq - 1]);
-                  const float ck = csb[e * L + kq - 1], sk = snb[e * L + kq - 1];
-                  const float de = __half2float(d[dye_off<L>(lp) + m * (lp + 1) + kq]);
-                  const float dd = (m > 0) ? __half2float(d[dyo_off<L>(lp) + (m - 1) * lp + (kq - 1)]) : 0.f;
-                  // u+ = c v+ + s v-,  u- = -s v+ + c v-
-                  const float a_pp = de * ck, a_pm = de * sk;      // into v~(+m)
-                  const float a_mp = -dd * sk, a_mm = dd * ck;     // into v~(-m)
+            for (int kq = 1; kq <= L; ++kq) {
+              if (kq <= LP) {
+                const float ck = csb[e * L + kq - 1], sk = snb[e * L + kq - 1];
+                const float de = __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]);
+                const float dd = (m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
+                // u+ = c v+ + s v-,  u- = -s v+ + c v-
+                const float a_pp = de * ck, a_pm = de * sk;      // into v~(+m)
+                const float a_mp = -dd * sk, a_mm = dd * ck;     // into v~(-m)
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                  const __nv_bfloat16 *bp = reinterpret_cast<const __nv_bfloat16 *>(&vp[q2][kq - 1]);
+                  const __nv_bfloat16 *bn = reinterpret_cast<const __nv_bfloat16 *>(&vn[q2][kq - 1]);
 #pragma unroll
                   for (int x = 0; x < 8; ++x) {
                     const float vpx = __bfloat162float(bp[x]), vmx = __bfloat162float(bn[x]);
-                    accp[x] = fmaf(a_pp, vpx, fmaf(a_pm, vmx, accp[x]));
-                    accm[x] = fmaf(a_mp, vpx, fmaf(a_mm, vmx, accm[x]));
+                    accp[q2][x] = fmaf(a_pp, vpx, fmaf(a_pm, vmx, accp[q2][x]));
+                    accm[q2][x] = fmaf(a_mp, vpx, fmaf(a_mm, vmx, accm[q2][x]));
                   }
                 }
               }
-#pragma unroll
-              for (int x = 0; x < 8; ++x) { op[x] = __float2bfloat16_rn(accp[x]); om[x] = __float2bfloat16_rn(accm[x]); }
-            } else {
-#pragma unroll
-              for (int x = 0; x < 8; ++x) { op[x] = __float2bfloat16_rn(0.f); om[x] = __float2bfloat16_rn(0.f); }
             }
-            *reinterpret_cast<uint4 *>(up + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(op);
-            if (m > 0) *reinterpret_cast<uint4 *>(um + kmajor_off(e, cb, 128)) = *reinterpret_cast<uint4 *>(om);
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+              for (int x = 0; x < 8; ++x) {
+                op[q2][x] = __float2bfloat16_rn(accp[q2][x]);
+                om[q2][x] = __float2bfloat16_rn(accm[q2][x]);
+              }
+          };
+          if (Cf::TMU && sp >= Cf::NSU) {
+            // unit pair in TMEM as the M = 64 A operand: row e at lane
+            // 32 (e / 16) + e % 16 (+16 in the upper half); lane half 0 holds
+            // [v+ | v-], half 1 holds [v- | v+] (64 columns each, channel
+            // pairs packed low / high).  Warp 8 + pw writes subpartition pw % 4,
+            // channels [64 (pw / 4), +64).
+            const int q = pw & 3, chb = (pw >> 2) * 64;
+            const int e = 16 * q + (lane & 15), half = lane >> 4;
+#pragma unroll 1
+            for (int x = 0; x < 64; x += 32) {
+              uint32_t wpl[16], wmi[16];
+#pragma unroll
+              for (int c8 = 0; c8 < 4; c8 += 2) {
+                __align__(16) __nv_bfloat16 op[2][8], om[2][8];
+                rot2(std::integral_constant<int, L>{}, e, chb + x + 8 * c8, chb + x + 8 * c8 + 8, op, om);
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    wpl[4 * (c8 + q2) + i] = *reinterpret_cast<const uint32_t *>(&op[q2][2 * i]);
+                    wmi[4 * (c8 + q2) + i] = *reinterpret_cast<const uint32_t *>(&om[q2][2 * i]);
+                  }
+              }
+              const uint32_t ta = tbase + ((uint32_t)(32 * q) << 16) + TM_UNIT + (uint32_t)(chb + x) / 2;
+              uint32_t lo[16], hi[16];   // warp-collective stores: select per lane
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                lo[i] = half ? wmi[i] : wpl[i];
+                hi[i] = half ? wpl[i] : wmi[i];
+              }
+              tmem_st_32x32b_x16u(ta, lo);
+              tmem_st_32x32b_x16u(ta + 64, hi);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+          } else {
+            uint8_t *up = units + (size_t)sp * UNIT_BYTES;
+            uint8_t *um = up + UNIT_BYTES;
+            // a warp covers 8 edges x 4 channel blocks: 64 contiguous bytes per
+            // gathered row, and 8 edges x 16 B per core-matrix row block in
+            // shared memory (no bank conflicts beyond the 4 wavefronts of 512 B)
+            // thread: one edge, channel blocks lane/8 + {0, 4, 8, 12}
+            const int e = pw * 8 + (lane & 7);
+            auto fill = [&](auto LPc) {
+#pragma unroll 1
+              for (int k2 = 0; k2 < 4; k2 += 2) {
+                const int cbA = (4 * k2 + (lane >> 3)) * 8, cbB = cbA + 32;
+                __align__(16) __nv_bfloat16 op[2][8], om[2][8];
+                rot2(LPc, e, cbA, cbB, op, om);
+                *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbA, 128)) = *reinterpret_cast<uint4 *>(op[0]);
+                *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbB, 128)) = *reinterpret_cast<uint4 *>(op[1]);
+                if (m > 0) {
+                  *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbA, 128)) = *reinterpret_cast<uint4 *>(om[0]);
+                  *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbB, 128)) = *reinterpret_cast<uint4 *>(om[1]);
+                }
+              }
+            };
+            switch (lp) {
+              case 0: fill(std::integral_constant<int, 0>{}); break;
+              case 1: if constexpr (L >= 1) fill(std::integral_constant<int, (L >= 1 ? 1 : 0)>{}); break;
+              case 2: if constexpr (L >= 2) fill(std::integral_constant<int, (L >= 2 ? 2 : 0)>{}); break;
+              case 3: if constexpr (L >= 3) fill(std::integral_constant<int, (L >= 3 ? 3 : 0)>{}); break;
+              default: if constexpr (L >= 4) fill(std::integral_constant<int, (L >= 4 ? 4 : 0)>{}); break;
+            }
           }
           fence_async_smem();
           named_bar(2, 256);
@@ -969,8 +1203,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             mbar_arrive(&unit_full[sp]);
             if (m > 0) mbar_arrive(&unit_full[sp + 1]);
           }
-          ++pfill[sp];
-          if (m > 0) ++pfill[sp + 1];
+          pfillpar ^= 1u << sp;
+          if (m > 0) pfillpar ^= 1u << (sp + 1);
         }
       }
       if (dead) break;
@@ -1017,14 +1251,14 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   const size_t Q = (size_t)(L + 1) * (L + 1);
   E2F_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)N * Q * CH * sizeof(float), s));
   if (E == 0) return E2F_OK;
+  {
+    const e2f_status ps = ensure_dy_poly();
+    if (ps != E2F_OK) return ps;
+  }
   // pack weights
   int nst = 0;
-  size_t wbytes = 0;
-  for (int m = 0; m <= L; ++m) {
-    const int n = (L - m + 1) * (L - m + 1) * 4;
-    nst += n;
-    wbytes += (size_t)n * (m == 0 ? 8192 : 16384);
-  }
+  for (int m = 0; m <= L; ++m) nst += (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
+  const size_t wbytes = (size_t)nst * STAGE_BYTES;
   Scratch wp, st;
   E2F_CUDA_TRY(wp.alloc(wbytes, s));
   E2F_CUDA_TRY(st.alloc((size_t)N * w->H * sizeof(float2), s));

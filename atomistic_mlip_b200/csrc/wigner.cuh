@@ -28,8 +28,11 @@ namespace e2f {
 E2F_HD int wig_offset(int l) { return l * (4 * l * l - 1) / 3; }
 E2F_HD int wig_size(int L) { return wig_offset(L + 1); }
 
+E2F_HD float wig_sqrt(float x) { return sqrtf(x); }
+E2F_HD double wig_sqrt(double x) { return sqrt(x); }
+
 // D^1 from a row-major rotation R (index order (y, z, x) = (1, 2, 0)).
-E2F_HD void wig_l1_from_rotation(const float R[9], float D1[9]) {
+template <typename T> E2F_HD void wig_l1_from_rotation(const T R[9], T D1[9]) {
   const int p[3] = {1, 2, 0};
   for (int a = 0; a < 3; ++a)
     for (int b = 0; b < 3; ++b) D1[a * 3 + b] = R[p[a] * 3 + p[b]];
@@ -37,50 +40,50 @@ E2F_HD void wig_l1_from_rotation(const float R[9], float D1[9]) {
 
 // Helper P^i_{a,b} of the recursion: i in {-1,0,1}, a in -(l-1)..(l-1),
 // b in -l..l.  D1 is 3x3 (index +1), Dp is the (2l-1)^2 block of l-1.
-E2F_HD float wig_P(int i, int a, int b, int l, const float *D1, const float *Dp) {
+template <typename T> E2F_HD T wig_P(int i, int a, int b, int l, const T *D1, const T *Dp) {
   const int w = 2 * l - 1;            // width of the l-1 block
   const int ra = a + (l - 1);         // row in the l-1 block
-  const float ri1 = D1[(i + 1) * 3 + 2];   // R1(i, +1)
-  const float rim = D1[(i + 1) * 3 + 0];   // R1(i, -1)
-  const float ri0 = D1[(i + 1) * 3 + 1];   // R1(i,  0)
+  const T ri1 = D1[(i + 1) * 3 + 2];   // R1(i, +1)
+  const T rim = D1[(i + 1) * 3 + 0];   // R1(i, -1)
+  const T ri0 = D1[(i + 1) * 3 + 1];   // R1(i,  0)
   if (b == l) return ri1 * Dp[ra * w + (2 * l - 2)] - rim * Dp[ra * w + 0];
   if (b == -l) return ri1 * Dp[ra * w + 0] + rim * Dp[ra * w + (2 * l - 2)];
   return ri0 * Dp[ra * w + (b + l - 1)];
 }
 
 // One entry D^l[m][m'] (l >= 2) from D^1 and D^(l-1).
-E2F_HD float wig_entry(int l, int m, int mp, const float *D1, const float *Dp) {
+template <typename T> E2F_HD T wig_entry(int l, int m, int mp, const T *D1, const T *Dp) {
   const int am = m < 0 ? -m : m;
-  const float den = (mp == l || mp == -l) ? (float)(2 * l * (2 * l - 1))
-                                          : (float)((l + mp) * (l - mp));
-  float acc = 0.f;
+  const T den = (mp == l || mp == -l) ? (T)(2 * l * (2 * l - 1)) : (T)((l + mp) * (l - mp));
+  const T sqrt2 = (T)1.41421356237309504880;
+  T acc = 0;
   // u term
-  const float uu = (float)((l + m) * (l - m));
-  if (uu > 0.f) acc += sqrtf(uu / den) * wig_P(0, m, mp, l, D1, Dp);
+  const T uu = (T)((l + m) * (l - m));
+  if (uu > 0) acc += wig_sqrt(uu / den) * wig_P<T>(0, m, mp, l, D1, Dp);
   // v term
   {
-    const float kd = (m == 0) ? 2.f : 1.f;
-    float v = 0.5f * sqrtf(kd * (float)((l + am - 1) * (l + am)) / den);
+    const T kd = (m == 0) ? (T)2 : (T)1;
+    T v = (T)0.5 * wig_sqrt(kd * (T)((l + am - 1) * (l + am)) / den);
     if (m == 0) v = -v;
-    float V;
+    T V;
     if (m == 0) {
-      V = wig_P(1, 1, mp, l, D1, Dp) + wig_P(-1, -1, mp, l, D1, Dp);
+      V = wig_P<T>(1, 1, mp, l, D1, Dp) + wig_P<T>(-1, -1, mp, l, D1, Dp);
     } else if (m > 0) {
-      V = wig_P(1, m - 1, mp, l, D1, Dp) * (m == 1 ? 1.41421356237309515f : 1.f);
-      if (m != 1) V -= wig_P(-1, -m + 1, mp, l, D1, Dp);
+      V = wig_P<T>(1, m - 1, mp, l, D1, Dp) * (m == 1 ? sqrt2 : (T)1);
+      if (m != 1) V -= wig_P<T>(-1, -m + 1, mp, l, D1, Dp);
     } else {
-      V = wig_P(-1, -m - 1, mp, l, D1, Dp) * (m == -1 ? 1.41421356237309515f : 1.f);
-      if (m != -1) V += wig_P(1, m + 1, mp, l, D1, Dp);
+      V = wig_P<T>(-1, -m - 1, mp, l, D1, Dp) * (m == -1 ? sqrt2 : (T)1);
+      if (m != -1) V += wig_P<T>(1, m + 1, mp, l, D1, Dp);
     }
     acc += v * V;
   }
   // w term (zero for m = 0 and for |m| >= l - 1)
   if (m != 0 && am + 1 <= l - 1) {
-    const float w = -0.5f * sqrtf((float)((l - am - 1) * (l - am)) / den);
-    float W;
-    if (m > 0) W = wig_P(1, m + 1, mp, l, D1, Dp) + wig_P(-1, -m - 1, mp, l, D1, Dp);
-    else       W = wig_P(1, m - 1, mp, l, D1, Dp) - wig_P(-1, -m + 1, mp, l, D1, Dp);
-    acc += w * W;
+    const T w = (T)-0.5 * wig_sqrt((T)((l - am - 1) * (l - am)) / den);
+    T Wt;
+    if (m > 0) Wt = wig_P<T>(1, m + 1, mp, l, D1, Dp) + wig_P<T>(-1, -m - 1, mp, l, D1, Dp);
+    else       Wt = wig_P<T>(1, m - 1, mp, l, D1, Dp) - wig_P<T>(-1, -m + 1, mp, l, D1, Dp);
+    acc += w * Wt;
   }
   return acc;
 }
@@ -131,16 +134,16 @@ E2F_HD float wig_entry_s(int l, int m, int mp, const float *D1, const float *Dp,
 }
 
 // All blocks l = 0..L of one rotation, sequentially (one thread).
-E2F_HD void wig_all_serial(const float R[9], int L, float *D) {
-  D[0] = 1.f;
+template <typename T> E2F_HD void wig_all_serial(const T R[9], int L, T *D) {
+  D[0] = 1;
   if (L < 1) return;
-  wig_l1_from_rotation(R, D + 1);
+  wig_l1_from_rotation<T>(R, D + 1);
   for (int l = 2; l <= L; ++l) {
-    const float *Dp = D + wig_offset(l - 1);
-    float *Dl = D + wig_offset(l);
+    const T *Dp = D + wig_offset(l - 1);
+    T *Dl = D + wig_offset(l);
     const int w = 2 * l + 1;
     for (int m = -l; m <= l; ++m)
-      for (int mp = -l; mp <= l; ++mp) Dl[(m + l) * w + (mp + l)] = wig_entry(l, m, mp, D + 1, Dp);
+      for (int mp = -l; mp <= l; ++mp) Dl[(m + l) * w + (mp + l)] = wig_entry<T>(l, m, mp, D + 1, Dp);
   }
 }
 

@@ -29,11 +29,13 @@ def test_wigner_blocks_match_oracle(cuda_ok):
         assert np.max(np.abs(got - ref)) < 2e-6, l
 
 
-@pytest.mark.parametrize("prec", ["fp32", "bf16"])
-def test_projection_matches_oracle(cuda_ok, prec):
+@pytest.mark.parametrize("prec,C,H", [("fp32", 64, 4), ("bf16", 64, 4), ("bf16", 128, 8)])
+def test_projection_matches_oracle(cuda_ok, prec, C, H):
+    """C = 128 bf16 takes the tensor-core kernel (3,000 nodes: every degree
+    ends in a ragged 128-row tile); the others the SIMT kernel."""
     import torch
     from atomistic_mlip_b200 import e2f
-    wl = wlmod.make_workload(2, precision=prec, C=64, H=4)
+    wl = wlmod.make_workload(2, precision=prec, C=C, H=H)
     _, x, w, _ = helpers.to_device(wl, prec)
     q, k, v = e2f.project_qkv(x, w)
     torch.cuda.synchronize()

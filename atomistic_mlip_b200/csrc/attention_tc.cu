@@ -46,8 +46,8 @@ using namespace tc;
 constexpr int CH = 128;            // channels on this path
 constexpr int TE = 64;             // edges per tile (MMA M)
 constexpr int S = 4;               // destination-node slots per tile
-constexpr int NSTAGE = 2;          // weight ring stages
-constexpr int STAGE_BYTES = 32768; // one weight stage: W0 128 x 128, or Wr|Wi 128 x 64 each
+constexpr int NSTAGE = 3;          // weight ring stages
+constexpr int STAGE_BYTES = 16384; // one weight stage: W0 128 x 64, or Wr|Wi 128 x 32 each
 constexpr int UNIT_BYTES = TE * CH * 2;
 constexpr int A2_BYTES = CH * TE * 2;
 constexpr int NTHREADS = 512;
@@ -89,20 +89,25 @@ template <int L> struct Cfg {
   static constexpr size_t OFF_W = OFF_UNIT + (size_t)NSU * UNIT_BYTES;
   static constexpr size_t OFF_A2 = OFF_W + (size_t)NSTAGE * STAGE_BYTES;
   static constexpr size_t OFF_R = OFF_A2 + 2 * (size_t)A2_BYTES;
-  static constexpr size_t OFF_AL = OFF_R + 2 * (size_t)NLMAX * TE * 2;
-  static constexpr size_t OFF_DY = OFF_AL + (size_t)TE * ALS * 4;
-  static constexpr size_t OFF_CS = OFF_DY + (size_t)TE * NDYP * 2;
-  static constexpr size_t OFF_G = OFF_CS + 2 * (size_t)TE * (L > 0 ? L : 1) * 4;
-  static constexpr size_t OFF_GEO = OFF_G + (size_t)TE * P * 4;     // float [TE][4]: ct, st, u, pad
-  static constexpr size_t OFF_J = OFF_GEO + (size_t)TE * 4 * 4;      // int [TE] j, node
-  static constexpr size_t OFF_TILE = OFF_J + 2 * (size_t)TE * 4;     // 8 ints
+  // per-tile geometry, two copies (tile parity): the producers build the
+  // next tile's while the epilogue still reads the current one's
+  static __host__ __device__ constexpr size_t r16(size_t x) { return (x + 15) & ~(size_t)15; }
+  static constexpr size_t G_AL = 0;                                             // half [TE][ALS]
+  static constexpr size_t G_DY = r16(G_AL + (size_t)TE * ALS * 2);              // half [TE][NDYP]
+  static constexpr size_t G_CS = r16(G_DY + (size_t)TE * NDYP * 2);             // float cos [L][TE], sin [L][TE]
+  static constexpr size_t G_GS = r16(G_CS + 2 * (size_t)TE * (L > 0 ? L : 1) * 4);  // half [TE][P]
+  static constexpr size_t G_J = r16(G_GS + (size_t)TE * P * 2);                 // int j [TE], node [TE]
+  static constexpr size_t GEO_BYTES = r16(G_J + 2 * (size_t)TE * 4);
+  static constexpr size_t OFF_G2 = OFF_R + 2 * (size_t)NLMAX * TE * 2;
+  static constexpr size_t OFF_GEO = OFF_G2 + 2 * GEO_BYTES;          // float [TE][4]: ct, st, u, pad
+  static constexpr size_t OFF_TILE = OFF_GEO + (size_t)TE * 4 * 4;   // 8 ints
   static constexpr size_t OFF_BAR = (OFF_TILE + 32 + 7) & ~(size_t)7;
-  static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 5;
+  static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 7;
   static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(TM_OUT + OUT_COLS <= TM_UNIT, "TMEM budget");
   // weight stages per tile
-  static __host__ __device__ constexpr int stages_of_m(int m) { return (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2); }
+  static __host__ __device__ constexpr int stages_of_m(int m) { return (L - m + 1) * (L - m + 1) * (m == 0 ? 2 : 4); }
   static __host__ __device__ constexpr int stages_per_tile() {
     int s = 0;
     for (int m = 0; m <= L; ++m) s += stages_of_m(m);
@@ -210,10 +215,11 @@ template <int L> __device__ __forceinline__ int dyo_off(int l) {
 }
 
 // ---------------------------------------------------------------------------
-// weight packing: one 32 KB stage per (m, l, l', half), in the order the MMA
-// warp consumes them.  m = 0: W0 rows of degree l, columns of degree l'
-// (128 x 128, K-major core matrices, Kc = 128).  m >= 1: Wr then Wi rows of
-// degree l, columns of degree l', K half `kh` (128 x 64 each, Kc = 64).
+// weight packing: one 16 KB stage per (m, l, l', K chunk), in the order the
+// MMA warp consumes them.  m = 0: W0 rows of degree l, columns of degree l',
+// K chunk of 64 (128 x 64, K-major core matrices, Kc = 64).  m >= 1: Wr then
+// Wi rows of degree l, columns of degree l', K chunk of 32 (128 x 32 each,
+// Kc = 32).
 // ---------------------------------------------------------------------------
 struct PackArgs {
   const __nv_bfloat16 *W0;
@@ -229,28 +235,23 @@ __global__ void pack_w_kernel(PackArgs a) {
   int s = blockIdx.x;
   int m = 0;
   for (;; ++m) {
-    const int n = (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
+    const int n = (L - m + 1) * (L - m + 1) * (m == 0 ? 2 : 4);
     if (s < n) break;
     s -= n;
   }
-  const int nk = (m == 0) ? 1 : 2;
-  const int kh = s % nk;
+  const int nk = (m == 0) ? 2 : 4, kw = (m == 0) ? 64 : 32;
+  const int kc = s % nk;
   const int l = m + (s / nk) / (L - m + 1), lp = m + (s / nk) % (L - m + 1);
   uint8_t *stage = a.dst + (size_t)blockIdx.x * STAGE_BYTES;
   const int row = threadIdx.x;
   const int n = (L - m + 1) * CH;
   const size_t srow = (size_t)(l - m) * CH + row;
-  if (m == 0) {
-    const int scol = lp * CH;
-    for (int k = 0; k < 128; ++k)
-      *reinterpret_cast<__nv_bfloat16 *>(stage + kmajor_off(row, k, 128)) = a.W0[srow * n + scol + k];
-  } else {
-    const int scol = (lp - m) * CH + kh * 64;
-    for (int t = 0; t < 2; ++t) {
-      const __nv_bfloat16 *src = (t == 0) ? a.Wr[m] : a.Wi[m];
-      for (int k = 0; k < 64; ++k)
-        *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = src[srow * n + scol + k];
-    }
+  const int scol = (lp - m) * CH + kc * kw;
+  const int ntile = (m == 0) ? 1 : 2;
+  for (int t = 0; t < ntile; ++t) {
+    const __nv_bfloat16 *src = (m == 0) ? a.W0 : (t == 0 ? a.Wr[m] : a.Wi[m]);
+    for (int k = 0; k < kw; ++k)
+      *reinterpret_cast<__nv_bfloat16 *>(stage + t * 8192 + kmajor_off(row, k, kw)) = src[srow * n + scol + k];
   }
 }
 
@@ -474,9 +475,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   uint64_t *rg_done = a2r_full + 2;
   uint64_t *tile_done = rg_done + 2;
   uint64_t *slots_clean = tile_done + 1;
-  uint64_t *geo_full = slots_clean + 1;
-  uint64_t *geo_empty = geo_full + 1;
-  uint64_t *mma_drain = geo_empty + 1;
+  uint64_t *geo_full = slots_clean + 1;    // [2], per geometry copy
+  uint64_t *geo_empty = geo_full + 2;     // [2]
+  uint64_t *mma_drain = geo_empty + 2;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + Cf::NBAR);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -484,24 +485,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   uint8_t *wst = smem + Cf::OFF_W;
   uint8_t *A2 = smem + Cf::OFF_A2;
   uint8_t *Rb = smem + Cf::OFF_R;
-  float *al = reinterpret_cast<float *>(smem + Cf::OFF_AL);          // [TE][ALS]
-  __half *dy = reinterpret_cast<__half *>(smem + Cf::OFF_DY);        // [TE][NDYP]
-  float *csb = reinterpret_cast<float *>(smem + Cf::OFF_CS);         // cos [TE][L], sin [TE][L]
-  float *snb = csb + TE * (L > 0 ? L : 1);
-  float *gs = reinterpret_cast<float *>(smem + Cf::OFF_G);           // [TE][P]
   float *geo = reinterpret_cast<float *>(smem + Cf::OFF_GEO);        // [TE][4]
-  int *jj = reinterpret_cast<int *>(smem + Cf::OFF_J);               // [TE]
-  int *nodeof = jj + TE;                                             // [TE]
+  // geometry copy c
+  auto g_al = [&](int c) { return reinterpret_cast<__half *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_AL); };
+  auto g_dy = [&](int c) { return reinterpret_cast<__half *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_DY); };
+  auto g_cs = [&](int c) { return reinterpret_cast<float *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_CS); };
+  auto g_gs = [&](int c) { return reinterpret_cast<__half *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_GS); };
+  auto g_jj = [&](int c) { return reinterpret_cast<int *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_J); };
 
   if (tid == 0) {
-    for (int s = 0; s < NUNIT; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], 1); }
+    // unit_full: one arrival per producer warp (the warps fill units independently)
+    for (int s = 0; s < NUNIT; ++s) { mbar_init(&unit_full[s], 8); mbar_init(&unit_empty[s], 1); }
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&y_full[b], 1); mbar_init(&y_empty[b], 4);
       mbar_init(&a2r_full[b], 1); mbar_init(&rg_done[b], 1);
     }
     mbar_init(tile_done, 1); mbar_init(slots_clean, 4);
-    mbar_init(geo_full, 1); mbar_init(geo_empty, 4);
+    for (int c = 0; c < 2; ++c) { mbar_init(&geo_full[c], 1); mbar_init(&geo_empty[c], 4); }
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -531,8 +532,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       uint32_t rgpar = 0;          // bit sg: parity of the R-GEMMs issued for sign sg
       const uint32_t s_units = smem_addr(units), s_w = smem_addr(wst), s_a2 = smem_addr(A2), s_r = smem_addr(Rb);
       const uint64_t ud0 = smem_desc(s_units, 128, 128 * 16);   // unit 0, K-major, Kc = 128
-      const uint64_t wd128 = smem_desc(s_w, 128, 128 * 16);     // stage 0 as 128 x 128 (m = 0)
-      const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 2 x 128 x 64 (m >= 1)
+      const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 128 x 64 (m = 0)
+      const uint64_t wd32 = smem_desc(s_w, 128, 32 * 16);       // stage 0 as 2 x 128 x 32 (m >= 1)
       const uint64_t a2d = smem_desc(s_a2, 128, 64 * 16);       // A2, MN-major, K = 64 edges
       const uint64_t rd = smem_desc(s_r, 128, 64 * 16);         // R, K-major, K = 64 edges
       int t = 0;
@@ -580,25 +581,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               const bool in_tmem = Cf::TMU && sp >= Cf::NSU;
               // descriptors advance by (byte offset >> 4): 16 per 16-wide K step
               const uint64_t adp = ud0 + (uint64_t)sp * (UNIT_BYTES >> 4), adm = adp + (UNIT_BYTES >> 4);
-              const int nk = (m == 0) ? 1 : 2;
+              const int nk = (m == 0) ? 2 : 4;
               #pragma unroll 1
-              for (int kh = 0; kh < nk; ++kh) {
+              for (int kc = 0; kc < nk; ++kc) {
                 const uint32_t s = st % NSTAGE;
                 if (!W.wait(&w_full[s], (st / NSTAGE) & 1)) { bad = true; break; }
                 tc_fence_after();
-                const uint32_t acc0 = (lp > m || kh > 0) ? 1u : 0u;
+                const uint32_t acc0 = (lp > m || kc > 0) ? 1u : 0u;
                 if (m == 0) {
-                  const uint64_t bd = wd128 + (uint64_t)s * (STAGE_BYTES >> 4);
-                  mma_bf16_ss(dp, adp, bd, ID_MAIN, acc0);
+                  // K chunk of 64: 4 steps of 16
+                  const uint64_t bd = wd64 + (uint64_t)s * (STAGE_BYTES >> 4);
+                  const uint64_t ak = adp + 64 * kc;
+                  mma_bf16_ss(dp, ak, bd, ID_MAIN, acc0);
 #pragma unroll
-                  for (int sub = 1; sub < 8; ++sub) mma_bf16_ss(dp, adp + 16 * sub, bd + 16 * sub, ID_MAIN, 1u);
+                  for (int sub = 1; sub < 4; ++sub) mma_bf16_ss(dp, ak + 16 * sub, bd + 16 * sub, ID_MAIN, 1u);
                 } else {
-                  const uint64_t br = wd64 + (uint64_t)s * (STAGE_BYTES >> 4), bi = br + (16384 >> 4);
+                  // K chunk of 32: 2 steps of 16
+                  const uint64_t br = wd32 + (uint64_t)s * (STAGE_BYTES >> 4), bi = br + (8192 >> 4);
                   if (in_tmem) {
                     // lane half 0 holds [v+ | v-], lane half 1 holds [v- | v+]
-                    const uint32_t a0 = tbase + TM_UNIT + 32 * kh, a1 = a0 + (16u << 16);
+                    const uint32_t a0 = tbase + TM_UNIT + 16 * kc, a1 = a0 + (16u << 16);
 #pragma unroll
-                    for (int sub = 0; sub < 4; ++sub) {
+                    for (int sub = 0; sub < 2; ++sub) {
                       const uint32_t acc = sub > 0 ? 1u : acc0;
                       mma_bf16_ts(dp, a0 + 8 * sub, br + 16 * sub, ID_MAIN, acc);
                       mma_bf16_ts(dp, a0 + 64 + 8 * sub, bi + 16 * sub, ID_NEGB, 1u);
@@ -606,9 +610,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                       mma_bf16_ts(dmn, a1 + 64 + 8 * sub, bi + 16 * sub, ID_MAIN, 1u);
                     }
                   } else {
-                    const uint64_t ap = adp + 64 * kh, am = adm + 64 * kh;
+                    const uint64_t ap = adp + 32 * kc, am = adm + 32 * kc;
 #pragma unroll
-                    for (int sub = 0; sub < 4; ++sub) {
+                    for (int sub = 0; sub < 2; ++sub) {
                       const uint32_t acc = sub > 0 ? 1u : acc0;
                       mma_bf16_ss(dp, ap + 16 * sub, br + 16 * sub, ID_MAIN, acc);
                       mma_bf16_ss(dp, am + 16 * sub, bi + 16 * sub, ID_NEGB, 1u);
@@ -668,7 +672,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       }
       // drain: wait for this loader's last copy so no bulk write lands after exit
       if (st > 0) {
-        for (uint32_t back = 1; back <= 2 && back <= st; ++back) {
+        for (uint32_t back = 1; back <= (uint32_t)NSTAGE && back <= st; ++back) {
           const uint32_t s_last = st - back;
           if ((int)(s_last % 2) != me) continue;
           const uint32_t s = s_last % NSTAGE;
@@ -697,8 +701,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     bool dead = false;
     bool ok = ti.start();
     while (ok && !dead) {
-      dead = bar_or(1, 128, et == 0 && !W.wait(geo_full, t & 1, 100));
+      // this tile's geometry copy (tile parity), filled by the producers
+      const int gc = t & 1;
+      dead = bar_or(1, 128, et == 0 && !W.wait(&geo_full[gc], (t >> 1) & 1, 100));
       if (dead) break;
+      const __half *al = g_al(gc), *gs = g_gs(gc), *dy = g_dy(gc);
+      const float *csb = g_cs(gc), *snb = csb + TE * (L > 0 ? L : 1);
+      const int *nodeof = g_jj(gc) + TE;
       const int ne = (int)(ti.e1 - ti.e0);
       #pragma unroll 1
       for (int m = 0; m <= L && !dead; ++m) {
@@ -721,7 +730,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const int e = 16 * ew + (lane & 15);
           const bool act = (m > 0 || sg == 0);
           const int p_ml = m * (L + 1) - m * (m - 1) / 2 + (l - m);
-          const float ge = (e < ne) ? gs[e * P + p_ml] : 0.f;
+          const float ge = (e < ne) ? __half2float(gs[e * P + p_ml]) : 0.f;
           uint8_t *a2 = A2 + sg * A2_BYTES;
 #pragma unroll 1
           for (int i = 0; i < 8; i += 2) {
@@ -734,8 +743,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               for (int h2 = 0; h2 < 2; ++h2) {
                 const int c0 = 16 * (i + h2);
                 // channels [c0, c0 + 8) and [c0 + 8, c0 + 16) lie in one head each
-                const float s_lo = (e < ne) ? al[e * ALS + (c0 >> hshift)] * ge : 0.f;
-                const float s_hi = (e < ne) ? al[e * ALS + ((c0 + 8) >> hshift)] * ge : 0.f;
+                const float s_lo = (e < ne) ? __half2float(al[e * ALS + (c0 >> hshift)]) * ge : 0.f;
+                const float s_hi = (e < ne) ? __half2float(al[e * ALS + ((c0 + 8) >> hshift)]) * ge : 0.f;
                 __align__(16) __nv_bfloat16 o[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(v[h2][j] * (j < 8 ? s_lo : s_hi));
@@ -748,49 +757,54 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           tc_fence_before();
           named_bar(1, 128);
           if (lane == 0) mbar_arrive(&y_empty[b]);
-          // ---- R for each sign, then hand over to the MMA warp
+          // ---- R for each sign, then hand over to the MMA warp.  R_s has
+          // rows (slot, m') (from row RO(l)), columns edges; the only nonzero
+          // entry of an edge's column is D^l[+-m][m'] in its own slot's rows.
+          // Zero both R buffers, then one thread per (edge, sign) writes its
+          // 2l + 1 entries.
           const int ng = (m == 0) ? 1 : 2;
           const int w2 = 2 * l + 1;
           const int nrow = Cf::NL(l);
-          #pragma unroll 1
-          for (int s2 = 0; s2 < ng; ++s2) {
-            uint8_t *Rs = Rb + (size_t)s2 * Cf::NLMAX * TE * 2;
-            // rows (slot, m'), columns edges; entry D^l[sm][m'] for the edge's slot
-            const int ro = Cf::RO(l);
-            for (int item = et; item < nrow * 8; item += 128) {
-              const int row = item >> 3, e8 = (item & 7) * 8;
-              const int rr = row - ro;
-              const int slot = rr / w2, mp = rr - slot * w2 - l;
-              __align__(16) __nv_bfloat16 o[8];
-#pragma unroll
-              for (int t8 = 0; t8 < 8; ++t8) {
-                const int ee = e8 + t8;
-                float val = 0.f;
-                if (rr >= 0 && rr < S * w2 && ee < ne && (nodeof[ee] % S) == slot) {
-                  const __half *d = dy + ee * Cf::NDYP;
-                  const int amp = mp < 0 ? -mp : mp;
-                  if (s2 == 0) {
-                    const float de = __half2float(d[dye_off<L>(l) + m * (l + 1) + amp]);
-                    val = (mp == 0) ? de : (mp > 0 ? de * csb[ee * L + amp - 1] : de * snb[ee * L + amp - 1]);
-                  } else if (mp != 0) {
-                    const float dd = __half2float(d[dyo_off<L>(l) + (m - 1) * l + (amp - 1)]);
-                    val = (mp > 0) ? -dd * snb[ee * L + amp - 1] : dd * csb[ee * L + amp - 1];
-                  }
-                }
-                o[t8] = __float2bfloat16_rn(val);
-              }
-              *reinterpret_cast<uint4 *>(Rs + kmajor_off(row, e8, 64)) = *reinterpret_cast<uint4 *>(o);
-            }
-            fence_async_smem();
-            named_bar(1, 128);
-            if (et == 0) mbar_arrive(&a2r_full[s2]);
-            if (s2 == 0) ++nA0; else ++nA1;
+          for (int idx = et; idx < ng * nrow * 8; idx += 128) {
+            const int s2 = idx / (nrow * 8), rem = idx - s2 * nrow * 8;
+            *reinterpret_cast<uint4 *>(Rb + (size_t)s2 * Cf::NLMAX * TE * 2 + kmajor_off(rem >> 3, (rem & 7) * 8, 64)) =
+                make_uint4(0u, 0u, 0u, 0u);
           }
+          named_bar(1, 128);
+          {
+            const int e = et & (TE - 1), s2 = et >> 6;
+            if (s2 < ng && e < ne) {
+              uint8_t *Rs = Rb + (size_t)s2 * Cf::NLMAX * TE * 2;
+              const __half *d = dy + e * Cf::NDYP;
+              const int row0 = Cf::RO(l) + (nodeof[e] % S) * w2;
+#pragma unroll 1
+              for (int t = 0; t < w2; ++t) {
+                const int mp = t - l, amp = mp < 0 ? -mp : mp;
+                float val = 0.f;
+                if (s2 == 0) {
+                  const float de = __half2float(d[dye_off<L>(l) + m * (l + 1) + amp]);
+                  val = (mp == 0) ? de : (mp > 0 ? de * csb[(amp - 1) * TE + e] : de * snb[(amp - 1) * TE + e]);
+                } else if (mp != 0) {
+                  const float dd = __half2float(d[dyo_off<L>(l) + (m - 1) * l + (amp - 1)]);
+                  val = (mp > 0) ? -dd * snb[(amp - 1) * TE + e] : dd * csb[(amp - 1) * TE + e];
+                }
+                *reinterpret_cast<__nv_bfloat16 *>(Rs + kmajor_off(row0 + t, e, 64)) = __float2bfloat16_rn(val);
+              }
+            }
+          }
+          fence_async_smem();
+          named_bar(1, 128);
+          if (et == 0) {
+            mbar_arrive(&a2r_full[0]);
+            if (ng > 1) mbar_arrive(&a2r_full[1]);
+          }
+          ++nA0;
+          if (ng > 1) ++nA1;
           ++pc;
         }
       }
       if (dead) break;
-      if (lane == 0) mbar_arrive(geo_empty);   // geometry of this tile no longer needed
+      if (lane == 0) mbar_arrive(&geo_empty[gc]);   // this geometry copy is free again
       // ---- tile end: read out the nodes that finished here
       dead = bar_or(1, 128, et == 0 && !W.wait(tile_done, t & 1, 40));
       if (dead) break;
@@ -827,7 +841,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               float *dst = orow + (size_t)(l * l + mp) * CH;
               const float val = __uint_as_float(r[l * l + mp]);
               if (shared_node) atomicAdd(dst, val);
-              else *dst = val;
+              else __stcs(dst, val);   // written once: evict-first, keep L2 for the gathers
               asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col), "r"(0u)
                            : "memory");
             }
@@ -843,89 +857,87 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     }
   } else if (warp >= 8) {
     // ======================= producers =======================
+    // Per tile t (geometry copy t & 1): the rotated units, degree m by degree
+    // m.  While the MMA warp works through the passes of degree m, the
+    // producers (which wait for units to be released) build the geometry of
+    // tile t + 1 into the other copy, a step at a time: basics, Wigner blocks,
+    // logits in two halves.
     const int pt = tid - 256;        // 0..255
     const int pw = pt >> 5;          // 0..7
     uint32_t pfillpar = 0;   // bit sp: parity of unit sp's fill count
-    int t = 0;
-    bool dead = false;
-    bool ok = ti.start();
-    while (ok && !dead) {
-      {
-        bool f = false;
-        if (pt == 0) f = !W.wait(geo_empty, (t & 1) ^ 1, 100);
-        dead = bar_or(2, 256, f || W.aborted());
-        if (dead) break;
-      }
-      const int64_t e0 = ti.e0;
-      const int ne = (int)(ti.e1 - e0);
-      // ---- per-edge basics: four threads per edge (consecutive lanes); the
-      // first computes the frame, all four share the radial MLP (hidden units
-      // 4q..4q+3 each, outputs reduced with shuffles)
-      {
-        const int e = pt >> 2, q4 = pt & 3;
-        const bool live = e < ne;
-        float r = 0.f;
-        if (live) {
-          const int64_t E = e0 + e;
-          int i = ti.n0;
-          while ((int64_t)a.row_ptr[i + 1] <= E) ++i;
-          const int j = a.col_idx[E];
-          float dx, dyv, dz;
-          pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dyv, dz);
-          r = sqrtf(dx * dx + dyv * dyv + dz * dz);
-          if (q4 == 0) {
-            jj[e] = j;
-            nodeof[e] = i;
-            float ux = 0.f, uy = 0.f, uz = 1.f;
-            if (r > 0.f) { ux = dx / r; uy = dyv / r; uz = dz / r; }
-            const float rho = sqrtf(ux * ux + uy * uy);
-            float cp = 1.f, sp = 0.f;
-            if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
-            float cm = 1.f, sm = 0.f;
-            for (int mm = 1; mm <= L; ++mm) {
-              const float c2 = cm * cp - sm * sp, s2 = sm * cp + cm * sp;
-              cm = c2; sm = s2;
-              csb[e * L + mm - 1] = cm;
-              snb[e * L + mm - 1] = sm;
-            }
-            geo[e * 4 + 0] = uz;
-            geo[e * 4 + 1] = rho;
-            geo[e * 4 + 2] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+    // ---- per-edge basics: four threads per edge (consecutive lanes); the
+    // first computes the frame, all four share the radial MLP (hidden units
+    // 4q..4q+3 each, outputs reduced with shuffles)
+    auto basics = [&](const TileIter &g, int c) {
+      const int ne = (int)(g.e1 - g.e0);
+      int *jj = g_jj(c), *nodeof = jj + TE;
+      float *csb = g_cs(c), *snb = csb + TE * (L > 0 ? L : 1);
+      __half *gs = g_gs(c);
+      const int e = pt >> 2, q4 = pt & 3;
+      const bool live = e < ne;
+      float r = 0.f;
+      if (live) {
+        const int64_t E = g.e0 + e;
+        int i = g.n0;
+        while ((int64_t)a.row_ptr[i + 1] <= E) ++i;
+        const int j = a.col_idx[E];
+        float dx, dyv, dz;
+        pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dyv, dz);
+        r = sqrtf(dx * dx + dyv * dyv + dz * dz);
+        if (q4 == 0) {
+          jj[e] = j;
+          nodeof[e] = i;
+          float ux = 0.f, uy = 0.f, uz = 1.f;
+          if (r > 0.f) { ux = dx / r; uy = dyv / r; uz = dz / r; }
+          const float rho = sqrtf(ux * ux + uy * uy);
+          float cp = 1.f, sp = 0.f;
+          if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
+          float cm = 1.f, sm = 0.f;
+          for (int mm = 1; mm <= L; ++mm) {
+            const float c2 = cm * cp - sm * sp, s2 = sm * cp + cm * sp;
+            cm = c2; sm = s2;
+            csb[(mm - 1) * TE + e] = cm;
+            snb[(mm - 1) * TE + e] = sm;
           }
-        } else if (q4 == 0) {
-          jj[e] = -1;
-          nodeof[e] = -1;
-          for (int mm = 0; mm < L; ++mm) { csb[e * L + mm] = 1.f; snb[e * L + mm] = 0.f; }
-          geo[e * 4 + 0] = 1.f; geo[e * 4 + 1] = 0.f; geo[e * 4 + 2] = 0.f;
+          geo[e * 4 + 0] = uz;
+          geo[e * 4 + 1] = rho;
+          geo[e * 4 + 2] = 0.5f * (cospif(r / a.g.rc) + 1.f);
         }
-        // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5), 16 SiLU, P outputs
-        float phi[8];
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const float dd = r - (float)kk * (a.g.rc / 7.f);
-          phi[kk] = expf(-dd * dd * 2.f);
-        }
-        float hid[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          float z = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) z = fmaf(__ldg(a.W1 + (4 * q4 + h) * 8 + kk), phi[kk], z);
-          hid[h] = z / (1.f + expf(-z));
-        }
-#pragma unroll
-        for (int p = 0; p < P; ++p) {
-          float gv = 0.f;
-#pragma unroll
-          for (int h = 0; h < 4; ++h) gv = fmaf(__ldg(a.W2 + p * 16 + 4 * q4 + h), hid[h], gv);
-          gv += __shfl_xor_sync(0xffffffffu, gv, 1);
-          gv += __shfl_xor_sync(0xffffffffu, gv, 2);
-          if ((p & 3) == q4) gs[e * P + p] = live ? gv : 0.f;
-        }
+      } else if (q4 == 0) {
+        jj[e] = -1;
+        nodeof[e] = -1;
+        for (int mm = 0; mm < L; ++mm) { csb[mm * TE + e] = 1.f; snb[mm * TE + e] = 0.f; }
+        geo[e * 4 + 0] = 1.f; geo[e * 4 + 1] = 0.f; geo[e * 4 + 2] = 0.f;
       }
-      named_bar(2, 256);
-      // ---- Wigner blocks of Ry(-theta), parity blocks straight to fp16:
-      // warp = entry (coefficients broadcast from constant memory), lane = edge
+      // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5), 16 SiLU, P outputs
+      float phi[8];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const float dd = r - (float)kk * (a.g.rc / 7.f);
+        phi[kk] = expf(-dd * dd * 2.f);
+      }
+      float hid[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float z = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) z = fmaf(__ldg(a.W1 + (4 * q4 + h) * 8 + kk), phi[kk], z);
+        hid[h] = z / (1.f + expf(-z));
+      }
+#pragma unroll
+      for (int p = 0; p < P; ++p) {
+        float gv = 0.f;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) gv = fmaf(__ldg(a.W2 + p * 16 + 4 * q4 + h), hid[h], gv);
+        gv += __shfl_xor_sync(0xffffffffu, gv, 1);
+        gv += __shfl_xor_sync(0xffffffffu, gv, 2);
+        if ((p & 3) == q4) gs[e * P + p] = __float2half_rn(live ? gv : 0.f);
+      }
+    };
+    // ---- Wigner blocks of Ry(-theta), parity blocks straight to fp16:
+    // warp = entry (coefficients broadcast from constant memory), lane = edge
+    auto wigner = [&](int c) {
+      __half *dy = g_dy(c);
       for (int x = pw; x < Cf::NDYE + Cf::NDYO; x += 8) {
         int l = 0, off = 0, m, mp;
         if (x < Cf::NDYE) {
@@ -940,114 +952,119 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           mp = -((y - off) % l + 1);
         }
         const float *cf = c_dypoly + DYP_STRIDE * (wig_offset(l) + (m + l) * (2 * l + 1) + (mp + l));
-        float c[L + 1];
+        float cc[L + 1];
 #pragma unroll
-        for (int jd = 0; jd <= L; ++jd) c[jd] = cf[1 + jd];   // zero above the entry's degree
+        for (int jd = 0; jd <= L; ++jd) cc[jd] = cf[1 + jd];   // zero above the entry's degree
         const bool eps = cf[0] != 0.f;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int e = lane + 32 * h2;
           const float ct = geo[e * 4 + 0], stt = geo[e * 4 + 1];
-          float p = c[L];
+          float p = cc[L];
 #pragma unroll
-          for (int jd = L - 1; jd >= 0; --jd) p = fmaf(p, ct, c[jd]);
+          for (int jd = L - 1; jd >= 0; --jd) p = fmaf(p, ct, cc[jd]);
           dy[e * Cf::NDYP + x] = __float2half_rn(eps ? p * stt : p);
         }
       }
-      named_bar(2, 256);
-      // ---- logits -> alpha: item = (edge, 8-channel block).  The q rows of
-      // the tile's (<= S) destination nodes are staged in shared memory (the
-      // unit area is free while a tile's geometry is built); the gathered k
-      // rows are loaded in two batches of degrees.  The blocks of one head are
-      // summed with shuffles (16 consecutive lanes = one edge's 16 blocks).
-      __nv_bfloat16 *sq = reinterpret_cast<__nv_bfloat16 *>(units);   // [S][Q][CH]
-      {
-        constexpr int NQV = S * Q * CH / 8;   // uint4 count
-        constexpr int PER = (NQV + 255) / 256;
-        uint4 tmp[PER];
+    };
+    // ---- logits -> alpha, items (edge, 8-channel block) of one half of the
+    // tile: q and k rows loaded a degree at a time; the blocks of one head
+    // are summed with shuffles (16 consecutive lanes = one edge's 16 blocks)
+    auto logits = [&](const TileIter &g, int c, int half) {
+      const int ne = (int)(g.e1 - g.e0);
+      const int *jj = g_jj(c), *nodeof = jj + TE;
+      const float *csb = g_cs(c), *snb = csb + TE * (L > 0 ? L : 1);
+      const __half *dy = g_dy(c);
+      __half *al = g_al(c);
+      for (int item = pt + half * (TE * 8); item < (half + 1) * (TE * 8); item += 256) {
+        const int e = item >> 4, c0 = (item & 15) * 8;
+        float acc = 0.f;
+        if (e < ne) {
+          const int i = nodeof[e], j = jj[e];
+          const __half *d = dy + e * Cf::NDYP;
+          const __nv_bfloat16 *qr = a.q + (size_t)i * Q * CH + c0;
+          const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c0;
+          float2 accv[4];
 #pragma unroll
-        for (int k = 0; k < PER; ++k) {
-          const int idx = pt + 256 * k;
-          const int node = ti.n0 + idx / (Q * CH / 8);
-          if (idx < NQV && node < a.N)
-            tmp[k] = *reinterpret_cast<const uint4 *>(a.q + (size_t)ti.n0 * Q * CH + (size_t)idx * 8);
-        }
+          for (int x = 0; x < 4; ++x) accv[x] = make_float2(0.f, 0.f);
+          auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
 #pragma unroll
-        for (int k = 0; k < PER; ++k) {
-          const int idx = pt + 256 * k;
-          const int node = ti.n0 + idx / (Q * CH / 8);
-          if (idx < NQV && node < a.N) reinterpret_cast<uint4 *>(sq)[idx] = tmp[k];
-        }
-      }
-      named_bar(2, 256);
-      {
-        for (int item = pt; item < TE * 16; item += 256) {
-          const int e = item >> 4, c0 = (item & 15) * 8;
-          float acc = 0.f;
-          if (e < ne) {
-            const int i = nodeof[e], j = jj[e];
-            const __half *d = dy + e * Cf::NDYP;
-            const __nv_bfloat16 *qr = sq + (size_t)(i - ti.n0) * Q * CH + c0;
-            const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c0;
-            float accv[8];
+          for (int l = 0; l <= L; ++l) {
+            uint4 qv[2 * L + 1], kv[2 * L + 1];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) accv[x] = 0.f;
-            auto degree = [&](int l, const uint4 *kv) {
-              float qh[8], kh[8];
+            for (int tt = 0; tt < 2 * l + 1; ++tt) {
+              qv[tt] = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + tt) * CH);
+              kv[tt] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + tt) * CH);
+            }
+            float2 qh[4], kh[4];
 #pragma unroll
-              for (int x = 0; x < 8; ++x) { qh[x] = 0.f; kh[x] = 0.f; }
+            for (int x = 0; x < 4; ++x) { qh[x] = make_float2(0.f, 0.f); kh[x] = make_float2(0.f, 0.f); }
 #pragma unroll
-              for (int t = 0; t < 2 * l + 1; ++t) {
-                const int mp = t - l, amp = mp < 0 ? -mp : mp;
-                const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
-                const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[e * L + amp - 1] : de * snb[e * L + amp - 1]);
-                const uint4 qv = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + t) * CH);
-                const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
-                const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv[t]);
+            for (int tt = 0; tt < 2 * l + 1; ++tt) {
+              const int mp = tt - l, amp = mp < 0 ? -mp : mp;
+              const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
+              const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[(amp - 1) * TE + e] : de * snb[(amp - 1) * TE + e]);
+              const float2 c2 = make_float2(coef, coef);
+              const uint32_t *qw = reinterpret_cast<const uint32_t *>(&qv[tt]);
+              const uint32_t *kw = reinterpret_cast<const uint32_t *>(&kv[tt]);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                  qh[x] = fmaf(coef, __bfloat162float(qb[x]), qh[x]);
-                  kh[x] = fmaf(coef, __bfloat162float(kb[x]), kh[x]);
-                }
+              for (int x = 0; x < 4; ++x) {
+                qh[x] = __ffma2_rn(c2, pair(qw[x]), qh[x]);
+                kh[x] = __ffma2_rn(c2, pair(kw[x]), kh[x]);
               }
-#pragma unroll
-              for (int x = 0; x < 8; ++x) accv[x] = fmaf(qh[x], kh[x], accv[x]);
-            };
-            constexpr int LB = (L + 2) / 2;          // degrees [0, LB) then [LB, L]
-            {
-              uint4 kv[LB * LB];
-#pragma unroll
-              for (int t = 0; t < LB * LB; ++t) kv[t] = *reinterpret_cast<const uint4 *>(kr + (size_t)t * CH);
-#pragma unroll
-              for (int l = 0; l < LB; ++l) degree(l, kv + l * l);
-            }
-            {
-              uint4 kv[Q - LB * LB];
-#pragma unroll
-              for (int t = 0; t < Q - LB * LB; ++t) kv[t] = *reinterpret_cast<const uint4 *>(kr + (size_t)(LB * LB + t) * CH);
-#pragma unroll
-              for (int l = LB; l <= L; ++l) degree(l, kv + (l * l - LB * LB));
             }
 #pragma unroll
-            for (int x = 0; x < 8; ++x) acc += accv[x];
+            for (int x = 0; x < 4; ++x) accv[x] = __ffma2_rn(qh[x], kh[x], accv[x]);
           }
-          const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
-          for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          const int blk = item & 15;
-          if ((blk & (nb - 1)) == 0) {
-            const int h = blk / nb;
-            float alpha = 0.f;
-            if (e < ne) {
-              const float2 stt = a.stats[(size_t)nodeof[e] * H + h];
-              const float u = geo[e * 4 + 2];
-              alpha = (stt.y > 0.f) ? u * expf(acc * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
-            }
-            al[e * ALS + h] = alpha;
+#pragma unroll
+          for (int x = 0; x < 4; ++x) acc += accv[x].x + accv[x].y;
+        }
+        const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
+        for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        const int blk = item & 15;
+        if ((blk & (nb - 1)) == 0) {
+          const int h = blk / nb;
+          float alpha = 0.f;
+          if (e < ne) {
+            const float2 stt = a.stats[(size_t)nodeof[e] * H + h];
+            const float u = geo[e * 4 + 2];
+            alpha = (stt.y > 0.f) ? u * expf(acc * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
           }
+          al[e * ALS + h] = __float2half_rn(alpha);
         }
       }
+    };
+    // geometry step k (0 basics, 1 Wigner, 2 / 3 logits halves) of tile g
+    // into copy c; step 0 first waits until the epilogue has released the copy
+    auto geo_step = [&](int k, const TileIter &g, int c, int tg) -> bool {
+      if (k == 0) {
+        bool f = false;
+        if (pt == 0) f = !W.wait(&geo_empty[c], ((tg >> 1) & 1) ^ 1, 100);
+        if (bar_or(2, 256, f || W.aborted())) return false;
+        basics(g, c);
+      } else if (k == 1) {
+        wigner(c);
+      } else {
+        logits(g, c, k - 2);
+      }
       named_bar(2, 256);
-      if (pt == 0) mbar_arrive(geo_full);
+      if (k == 3 && pt == 0) mbar_arrive(&geo_full[c]);
+      return true;
+    };
+    int t = 0;
+    bool dead = false;
+    bool ok = ti.start();
+    if (ok) {
+      for (int k = 0; k < 4 && !dead; ++k) dead = !geo_step(k, ti, 0, 0);
+    }
+    while (ok && !dead) {
+      const int gc = t & 1;
+      TileIter tn = ti;
+      const bool has_next = tn.next();
+      const int ne = (int)(ti.e1 - ti.e0);
+      const int *jj = g_jj(gc);
+      const float *csb = g_cs(gc), *snb = csb + TE * (L > 0 ? L : 1);
+      const __half *dy = g_dy(gc);
       // ---- rotate in, block by block
       #pragma unroll 1
       for (int m = 0; m <= L && !dead; ++m) {
@@ -1055,82 +1072,92 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         for (int lp = m; lp <= L; ++lp) {
           const int sp = (m == 0) ? lp : 2 * (lp - m);
           {
+            // each producer warp waits for the unit on its own: the warps run
+            // through the units independently (a warp that finished its part
+            // of one unit starts loading for the next)
             bool f = false;
-            if (pt == 0) {
+            if (lane == 0) {
               f = !W.wait(&unit_empty[sp], ((pfillpar >> sp) & 1) ^ 1, 40);
               if (!f && m > 0) f = !W.wait(&unit_empty[sp + 1], ((pfillpar >> (sp + 1)) & 1) ^ 1, 40);
             }
-            dead = bar_or(2, 256, f || W.aborted());
+            dead = __shfl_sync(0xffffffffu, (int)(f || W.aborted()), 0) != 0;
             if (dead) break;
           }
-          // v~(+m), v~(-m) of edge e for two 8-channel blocks of degree l'
-          // (all gathered rows of both blocks are loaded before any use)
-          // (degree l' as a compile-time constant: register use follows the degree)
-          auto rot2 = [&](auto LPc, int e, int cbA, int cbB, __nv_bfloat16 (&op)[2][8], __nv_bfloat16 (&om)[2][8]) {
+          // v~(+m), v~(-m) of edge e for four 8-channel blocks of degree l'
+          // (compile-time constant: register use follows the degree).  The
+          // gathered rows of block b + 1 are loaded while block b is computed;
+          // pairs of channels go through packed fp32 FMAs.  emit(b, wp, wm)
+          // receives block b as packed bf16 pairs (wp: +m, wm: -m).
+          auto rot4 = [&](auto LPc, int e, const int (&cbs)[4], auto &&emit) {
             constexpr int LP = decltype(LPc)::value;
+            constexpr int NR = 2 * LP + 1;
             if (e >= ne) {
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-              for (int q2 = 0; q2 < 2; ++q2)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) { op[q2][x] = __float2bfloat16_rn(0.f); om[q2][x] = __float2bfloat16_rn(0.f); }
+              for (int bb = 0; bb < 4; ++bb) emit(bb, z, z);
               return;
             }
             const int j = jj[e];
             const __half *d = dy + e * Cf::NDYP;
-            const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(LP * LP + LP) * CH;
-            const int cbs[2] = {cbA, cbB};
-            uint4 vz[2], vp[2][L > 0 ? L : 1], vn[2][L > 0 ? L : 1];
+            const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(LP * LP) * CH;
+            // per-edge coefficients: u+ = c v+ + s v-, u- = -s v+ + c v-, scaled
+            // by the y-rotation entries of row +m (even block) / -m (odd block)
+            const float c0 = __half2float(d[dye_off<L>(LP) + m * (LP + 1)]);
+            float app[LP > 0 ? LP : 1], apm[LP > 0 ? LP : 1], amp[LP > 0 ? LP : 1], amm[LP > 0 ? LP : 1];
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              vz[q2] = *reinterpret_cast<const uint4 *>(vr + cbs[q2]);
+            for (int kq = 1; kq <= LP; ++kq) {
+              const float ck = csb[(kq - 1) * TE + e], sk = snb[(kq - 1) * TE + e];
+              const float de = __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]);
+              const float dd = (m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
+              app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
+              amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
+            }
+            uint4 buf[2][NR];
 #pragma unroll
-              for (int kq = 1; kq <= L; ++kq) {
-                if (kq <= LP) {
-                  vp[q2][kq - 1] = *reinterpret_cast<const uint4 *>(vr + (size_t)kq * CH + cbs[q2]);
-                  vn[q2][kq - 1] = *reinterpret_cast<const uint4 *>(vr - (size_t)kq * CH + cbs[q2]);
+            for (int t = 0; t < NR; ++t) buf[0][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[0]);
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+              if (bb < 3) {
+#pragma unroll
+                for (int t = 0; t < NR; ++t)
+                  buf[(bb + 1) & 1][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[bb < 3 ? bb + 1 : bb]);
+              }
+              const uint4 *rb = buf[bb & 1];
+              auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+              float2 ap[4], am[4];
+              {
+                const uint32_t *w0 = reinterpret_cast<const uint32_t *>(&rb[LP]);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const float2 v0 = pair(w0[x]);
+                  ap[x] = make_float2(c0 * v0.x, c0 * v0.y);
+                  am[x] = make_float2(0.f, 0.f);
                 }
               }
-            }
-            float accp[2][8], accm[2][8];
-            {
-              // k = 0 term (cos-type rows only)
-              const float de = __half2float(d[dye_off<L>(LP) + m * (LP + 1) + 0]);
 #pragma unroll
-              for (int q2 = 0; q2 < 2; ++q2) {
-                const __nv_bfloat16 *b0 = reinterpret_cast<const __nv_bfloat16 *>(&vz[q2]);
+              for (int kq = 1; kq <= LP; ++kq) {
+                const uint32_t *wpv = reinterpret_cast<const uint32_t *>(&rb[LP + kq]);
+                const uint32_t *wnv = reinterpret_cast<const uint32_t *>(&rb[LP - kq]);
+                const float2 cpp = make_float2(app[kq - 1], app[kq - 1]), cpm = make_float2(apm[kq - 1], apm[kq - 1]);
+                const float2 cmp = make_float2(amp[kq - 1], amp[kq - 1]), cmm = make_float2(amm[kq - 1], amm[kq - 1]);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) { accp[q2][x] = de * __bfloat162float(b0[x]); accm[q2][x] = 0.f; }
-              }
-            }
-#pragma unroll
-            for (int kq = 1; kq <= L; ++kq) {
-              if (kq <= LP) {
-                const float ck = csb[e * L + kq - 1], sk = snb[e * L + kq - 1];
-                const float de = __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]);
-                const float dd = (m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
-                // u+ = c v+ + s v-,  u- = -s v+ + c v-
-                const float a_pp = de * ck, a_pm = de * sk;      // into v~(+m)
-                const float a_mp = -dd * sk, a_mm = dd * ck;     // into v~(-m)
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                  const __nv_bfloat16 *bp = reinterpret_cast<const __nv_bfloat16 *>(&vp[q2][kq - 1]);
-                  const __nv_bfloat16 *bn = reinterpret_cast<const __nv_bfloat16 *>(&vn[q2][kq - 1]);
-#pragma unroll
-                  for (int x = 0; x < 8; ++x) {
-                    const float vpx = __bfloat162float(bp[x]), vmx = __bfloat162float(bn[x]);
-                    accp[q2][x] = fmaf(a_pp, vpx, fmaf(a_pm, vmx, accp[q2][x]));
-                    accm[q2][x] = fmaf(a_mp, vpx, fmaf(a_mm, vmx, accm[q2][x]));
-                  }
+                for (int x = 0; x < 4; ++x) {
+                  const float2 vp2 = pair(wpv[x]), vn2 = pair(wnv[x]);
+                  ap[x] = __ffma2_rn(cpp, vp2, __ffma2_rn(cpm, vn2, ap[x]));
+                  am[x] = __ffma2_rn(cmp, vp2, __ffma2_rn(cmm, vn2, am[x]));
                 }
               }
-            }
+              uint4 wp, wm;
+              uint32_t *pp = reinterpret_cast<uint32_t *>(&wp), *pm = reinterpret_cast<uint32_t *>(&wm);
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2)
-#pragma unroll
-              for (int x = 0; x < 8; ++x) {
-                op[q2][x] = __float2bfloat16_rn(accp[q2][x]);
-                om[q2][x] = __float2bfloat16_rn(accm[q2][x]);
+              for (int x = 0; x < 4; ++x) {
+                const __nv_bfloat162 hp = __floats2bfloat162_rn(ap[x].x, ap[x].y);
+                const __nv_bfloat162 hm = __floats2bfloat162_rn(am[x].x, am[x].y);
+                pp[x] = *reinterpret_cast<const uint32_t *>(&hp);
+                pm[x] = *reinterpret_cast<const uint32_t *>(&hm);
               }
+              emit(bb, wp, wm);
+            }
           };
           if (Cf::TMU && sp >= Cf::NSU) {
             // unit pair in TMEM as the M = 64 A operand: row e at lane
@@ -1140,31 +1167,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             // channels [64 (pw / 4), +64).
             const int q = pw & 3, chb = (pw >> 2) * 64;
             const int e = 16 * q + (lane & 15), half = lane >> 4;
-#pragma unroll 1
-            for (int x = 0; x < 64; x += 32) {
-              uint32_t wpl[16], wmi[16];
+            // lane half h computes channels [chb + 32h, +32) of both signs;
+            // the two halves swap what the other one stores
+            uint32_t wpl[16], wmi[16];
+            {
+              const int cb0 = chb + 32 * half;
+              const int cbs[4] = {cb0, cb0 + 8, cb0 + 16, cb0 + 24};
+              rot4(std::integral_constant<int, L>{}, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
+                const uint32_t *pp = reinterpret_cast<const uint32_t *>(&wp), *pm = reinterpret_cast<const uint32_t *>(&wm);
 #pragma unroll
-              for (int c8 = 0; c8 < 4; c8 += 2) {
-                __align__(16) __nv_bfloat16 op[2][8], om[2][8];
-                rot2(std::integral_constant<int, L>{}, e, chb + x + 8 * c8, chb + x + 8 * c8 + 8, op, om);
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2)
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    wpl[4 * (c8 + q2) + i] = *reinterpret_cast<const uint32_t *>(&op[q2][2 * i]);
-                    wmi[4 * (c8 + q2) + i] = *reinterpret_cast<const uint32_t *>(&om[q2][2 * i]);
-                  }
-              }
-              const uint32_t ta = tbase + ((uint32_t)(32 * q) << 16) + TM_UNIT + (uint32_t)(chb + x) / 2;
-              uint32_t lo[16], hi[16];   // warp-collective stores: select per lane
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                lo[i] = half ? wmi[i] : wpl[i];
-                hi[i] = half ? wpl[i] : wmi[i];
-              }
-              tmem_st_32x32b_x16u(ta, lo);
-              tmem_st_32x32b_x16u(ta + 64, hi);
+                for (int i = 0; i < 4; ++i) { wpl[4 * bb + i] = pp[i]; wmi[4 * bb + i] = pm[i]; }
+              });
             }
+            uint32_t opl[16], omi[16];   // the partner half's block
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              opl[i] = __shfl_xor_sync(0xffffffffu, wpl[i], 16);
+              omi[i] = __shfl_xor_sync(0xffffffffu, wmi[i], 16);
+            }
+            const uint32_t ta = tbase + ((uint32_t)(32 * q) << 16) + TM_UNIT + (uint32_t)chb / 2;
+            uint32_t st0[16], st1[16], st2[16], st3[16];   // warp-collective stores: select per lane
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              st0[i] = half ? omi[i] : wpl[i];   // cols [ta, +16):      v+ (half 0) / v- (half 1), block A
+              st1[i] = half ? opl[i] : wmi[i];   // cols [ta + 64, +16): v- / v+, block A
+              st2[i] = half ? wmi[i] : opl[i];   // cols [ta + 16, +16): v+ / v-, block B
+              st3[i] = half ? wpl[i] : omi[i];   // cols [ta + 80, +16): v- / v+, block B
+            }
+            tmem_st_32x32b_x16u(ta, st0);
+            tmem_st_32x32b_x16u(ta + 64, st1);
+            tmem_st_32x32b_x16u(ta + 16, st2);
+            tmem_st_32x32b_x16u(ta + 80, st3);
             tmem_st_wait();
             tc_fence_before();
           } else {
@@ -1176,18 +1209,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             // thread: one edge, channel blocks lane/8 + {0, 4, 8, 12}
             const int e = pw * 8 + (lane & 7);
             auto fill = [&](auto LPc) {
-#pragma unroll 1
-              for (int k2 = 0; k2 < 4; k2 += 2) {
-                const int cbA = (4 * k2 + (lane >> 3)) * 8, cbB = cbA + 32;
-                __align__(16) __nv_bfloat16 op[2][8], om[2][8];
-                rot2(LPc, e, cbA, cbB, op, om);
-                *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbA, 128)) = *reinterpret_cast<uint4 *>(op[0]);
-                *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbB, 128)) = *reinterpret_cast<uint4 *>(op[1]);
-                if (m > 0) {
-                  *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbA, 128)) = *reinterpret_cast<uint4 *>(om[0]);
-                  *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbB, 128)) = *reinterpret_cast<uint4 *>(om[1]);
-                }
-              }
+              const int cb0 = (lane >> 3) * 8;
+              const int cbs[4] = {cb0, cb0 + 32, cb0 + 64, cb0 + 96};
+              rot4(LPc, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
+                *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbs[bb], 128)) = wp;
+                if (m > 0) *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbs[bb], 128)) = wm;
+              });
             };
             switch (lp) {
               case 0: fill(std::integral_constant<int, 0>{}); break;
@@ -1198,18 +1225,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             }
           }
           fence_async_smem();
-          named_bar(2, 256);
-          if (pt == 0) {
+          __syncwarp();
+          if (lane == 0) {
             mbar_arrive(&unit_full[sp]);
             if (m > 0) mbar_arrive(&unit_full[sp + 1]);
           }
           pfillpar ^= 1u << sp;
           if (m > 0) pfillpar ^= 1u << (sp + 1);
         }
+        // every producer warp reaches this point (done, or broken out on an
+        // abort), so the geometry barriers never wait for a missing warp
+        dead = bar_or(2, 256, dead || W.aborted());
+        if (dead) break;
+        // while the passes of degree m run: geometry steps of the next tile
+        if (has_next) {
+          for (int k = 0; k < 4 && !dead; ++k)
+            if ((k < L ? k : L) == m) dead = !geo_step(k, tn, gc ^ 1, t + 1);
+        }
       }
       if (dead) break;
       ++t;
-      ok = ti.next();
+      ti = tn;
+      ok = has_next;
     }
   }
   // warp 3 idles
@@ -1257,7 +1294,7 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   }
   // pack weights
   int nst = 0;
-  for (int m = 0; m <= L; ++m) nst += (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
+  for (int m = 0; m <= L; ++m) nst += (L - m + 1) * (L - m + 1) * (m == 0 ? 2 : 4);
   const size_t wbytes = (size_t)nst * STAGE_BYTES;
   Scratch wp, st;
   E2F_CUDA_TRY(wp.alloc(wbytes, s));

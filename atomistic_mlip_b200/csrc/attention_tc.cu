@@ -390,67 +390,92 @@ __device__ __forceinline__ void norm_sh_row0(float ux, float uy, float uz, float
 }
 
 template <int L>
-__global__ void __launch_bounds__(128) node_stats_kernel(TcArgs a) {
+__global__ void __launch_bounds__(256) node_stats_kernel(TcArgs a) {
+  // one block per destination node at a time; items (edge, 8-channel block)
+  // with the node's q row staged in shared memory, k rows gathered a degree
+  // at a time, head sums by shuffles, then an online (max, sum) per head
   constexpr int Q = (L + 1) * (L + 1);
-  __shared__ float y0s[32][Q];
-  __shared__ float us[32];
-  __shared__ float sv[32][HMAX];
+  constexpr int EC = 64;   // edges per chunk
+  __shared__ __align__(16) uint4 sq[Q * CH / 8];
+  __shared__ float y0s[EC][Q];
+  __shared__ float us[EC];
+  __shared__ float sv[EC][HMAX + 1];
   __shared__ float stat_m[HMAX], stat_l[HMAX];
-  const int c = threadIdx.x;
-  const int H = a.H, Ch = CH / H;
+  const int t = threadIdx.x;
+  const int H = a.H, Ch = CH / H, nb = Ch >> 3;
+  auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
   for (int i = blockIdx.x; i < a.N; i += gridDim.x) {
     const int r0 = a.row_ptr[i], r1 = a.row_ptr[i + 1];
-    float qreg[Q];
-#pragma unroll
-    for (int t = 0; t < Q; ++t) qreg[t] = __bfloat162float(a.q[((size_t)i * Q + t) * CH + c]);
-    if (c < HMAX) { stat_m[c] = -INFINITY; stat_l[c] = 0.f; }
+    __syncthreads();
+    for (int x = t; x < Q * CH / 8; x += 256) sq[x] = reinterpret_cast<const uint4 *>(a.q + (size_t)i * Q * CH)[x];
+    if (t < HMAX) { stat_m[t] = -INFINITY; stat_l[t] = 0.f; }
     const float3 pi = load_pos(a.pos, i);
-    for (int e0 = r0; e0 < r1; e0 += 32) {
-      const int nb = min(32, r1 - e0);
+    for (int c0 = r0; c0 < r1; c0 += EC) {
+      const int ne = min(EC, r1 - c0);
       __syncthreads();
-      if (c < nb) {
-        const int j = a.col_idx[e0 + c];
+      if (t < ne) {
+        const int j = a.col_idx[c0 + t];
         float dx, dy, dz;
         pair_disp(a.g, pi, load_pos(a.pos, j), dx, dy, dz);
         const float r = sqrtf(dx * dx + dy * dy + dz * dz);
         float ux = 0.f, uy = 0.f, uz = 1.f;
         if (r > 0.f) { ux = dx / r; uy = dy / r; uz = dz / r; }
-        norm_sh_row0<L>(ux, uy, uz, y0s[c]);
-        us[c] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+        norm_sh_row0<L>(ux, uy, uz, y0s[t]);
+        us[t] = 0.5f * (cospif(r / a.g.rc) + 1.f);
       }
       __syncthreads();
-      for (int e = 0; e < nb; ++e) {
-        const int j = a.col_idx[e0 + e];
-        const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c;
-        float s = 0.f;
+      for (int item = t; item < EC * 16; item += 256) {
+        const int e = item >> 4, blk = item & 15;
+        float acc = 0.f;
+        if (e < ne) {
+          const int j = a.col_idx[c0 + e];
+          const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + blk * 8;
+          float2 accv[4];
 #pragma unroll
-        for (int l = 0; l <= L; ++l) {
-          float qh = 0.f, kh = 0.f;
+          for (int x = 0; x < 4; ++x) accv[x] = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int mp = 0; mp < 2 * l + 1; ++mp) {
-            const float yv = y0s[e][l * l + mp];
-            qh = fmaf(yv, qreg[l * l + mp], qh);
-            kh = fmaf(yv, __bfloat162float(kr[(size_t)(l * l + mp) * CH]), kh);
+          for (int l = 0; l <= L; ++l) {
+            uint4 kv[2 * L + 1];
+#pragma unroll
+            for (int tt = 0; tt < 2 * l + 1; ++tt) kv[tt] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + tt) * CH);
+            float2 qh[4], kh[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) { qh[x] = make_float2(0.f, 0.f); kh[x] = make_float2(0.f, 0.f); }
+#pragma unroll
+            for (int tt = 0; tt < 2 * l + 1; ++tt) {
+              const float yv = y0s[e][l * l + tt];
+              const float2 y2 = make_float2(yv, yv);
+              const uint4 qv = sq[(l * l + tt) * (CH / 8) + blk];
+              const uint32_t *qw = reinterpret_cast<const uint32_t *>(&qv);
+              const uint32_t *kw = reinterpret_cast<const uint32_t *>(&kv[tt]);
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                qh[x] = __ffma2_rn(y2, pair(qw[x]), qh[x]);
+                kh[x] = __ffma2_rn(y2, pair(kw[x]), kh[x]);
+              }
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) accv[x] = __ffma2_rn(qh[x], kh[x], accv[x]);
           }
-          s = fmaf(qh, kh, s);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) acc += accv[x].x + accv[x].y;
         }
-        for (int o = 1; o < Ch; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (c % Ch == 0) sv[e][c / Ch] = s * a.inv_sqrt_d;
+        for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (e < ne && (blk & (nb - 1)) == 0) sv[e][blk / nb] = acc * a.inv_sqrt_d;
       }
       __syncthreads();
-      if (c < H) {
-        float mx = stat_m[c];
-        for (int e = 0; e < nb; ++e) mx = fmaxf(mx, sv[e][c]);
-        const float scale = (stat_m[c] == -INFINITY) ? 0.f : expf(stat_m[c] - mx);
+      if (t < H) {
+        float mx = stat_m[t];
+        for (int e = 0; e < ne; ++e) mx = fmaxf(mx, sv[e][t]);
+        const float scale = (stat_m[t] == -INFINITY) ? 0.f : expf(stat_m[t] - mx);
         float sum = 0.f;
-        for (int e = 0; e < nb; ++e) sum += us[e] * expf(sv[e][c] - mx);
-        stat_l[c] = stat_l[c] * scale + sum;
-        stat_m[c] = mx;
+        for (int e = 0; e < ne; ++e) sum += us[e] * expf(sv[e][t] - mx);
+        stat_l[t] = stat_l[t] * scale + sum;
+        stat_m[t] = mx;
       }
     }
     __syncthreads();
-    if (c < H) a.stats[(size_t)i * H + c] = make_float2(stat_m[c] == -INFINITY ? 0.f : stat_m[c], stat_l[c]);
-    __syncthreads();
+    if (t < H) a.stats[(size_t)i * H + t] = make_float2(stat_m[t] == -INFINITY ? 0.f : stat_m[t], stat_l[t]);
   }
 }
 
@@ -1265,8 +1290,8 @@ static e2f_status launch_tc(const TcArgs &args, int grid, cudaStream_t s) {
 
 template <int L>
 static e2f_status launch_stats(const TcArgs &args, cudaStream_t s) {
-  const int grid = (int)std::min<int64_t>(args.N, 148 * 16);
-  E2F_LAUNCH(node_stats_kernel<L>, grid, 128, 0, s, args);
+  const int grid = (int)std::min<int64_t>(args.N, 148 * 8);
+  E2F_LAUNCH(node_stats_kernel<L>, grid, 256, 0, s, args);
   return E2F_OK;
 }
 

@@ -46,8 +46,8 @@ using namespace tc;
 constexpr int CH = 128;            // channels on this path
 constexpr int TE = 64;             // edges per tile (MMA M)
 constexpr int S = 4;               // destination-node slots per tile
-constexpr int NSTAGE = 3;          // weight ring stages
-constexpr int STAGE_BYTES = 16384; // one weight stage: W0 128 x 64, or Wr|Wi 128 x 32 each
+constexpr int NSTAGE = 2;          // weight ring stages
+constexpr int STAGE_BYTES = 32768; // one weight stage: W0 128 x 128, or Wr|Wi 128 x 64 each
 constexpr int UNIT_BYTES = TE * CH * 2;
 constexpr int A2_BYTES = CH * TE * 2;
 constexpr int NTHREADS = 512;
@@ -88,7 +88,7 @@ template <int L> struct Cfg {
   static constexpr size_t OFF_UNIT = 0;
   static constexpr size_t OFF_W = OFF_UNIT + (size_t)NSU * UNIT_BYTES;
   static constexpr size_t OFF_A2 = OFF_W + (size_t)NSTAGE * STAGE_BYTES;
-  static constexpr size_t OFF_R = OFF_A2 + 2 * (size_t)A2_BYTES;
+  static constexpr size_t OFF_R = OFF_A2 + (size_t)A2_BYTES;   // one A2 buffer: the signs take turns
   // per-tile geometry, two copies (tile parity): the producers build the
   // next tile's while the epilogue still reads the current one's
   static __host__ __device__ constexpr size_t r16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -107,7 +107,7 @@ template <int L> struct Cfg {
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(TM_OUT + OUT_COLS <= TM_UNIT, "TMEM budget");
   // weight stages per tile
-  static __host__ __device__ constexpr int stages_of_m(int m) { return (L - m + 1) * (L - m + 1) * (m == 0 ? 2 : 4); }
+  static __host__ __device__ constexpr int stages_of_m(int m) { return (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2); }
   static __host__ __device__ constexpr int stages_per_tile() {
     int s = 0;
     for (int m = 0; m <= L; ++m) s += stages_of_m(m);
@@ -215,11 +215,10 @@ template <int L> __device__ __forceinline__ int dyo_off(int l) {
 }
 
 // ---------------------------------------------------------------------------
-// weight packing: one 16 KB stage per (m, l, l', K chunk), in the order the
-// MMA warp consumes them.  m = 0: W0 rows of degree l, columns of degree l',
-// K chunk of 64 (128 x 64, K-major core matrices, Kc = 64).  m >= 1: Wr then
-// Wi rows of degree l, columns of degree l', K chunk of 32 (128 x 32 each,
-// Kc = 32).
+// weight packing: one 32 KB stage per (m, l, l', half), in the order the MMA
+// warp consumes them.  m = 0: W0 rows of degree l, columns of degree l'
+// (128 x 128, K-major core matrices, Kc = 128).  m >= 1: Wr then Wi rows of
+// degree l, columns of degree l', K half `kh` (128 x 64 each, Kc = 64).
 // ---------------------------------------------------------------------------
 struct PackArgs {
   const __nv_bfloat16 *W0;
@@ -235,23 +234,28 @@ __global__ void pack_w_kernel(PackArgs a) {
   int s = blockIdx.x;
   int m = 0;
   for (;; ++m) {
-    const int n = (L - m + 1) * (L - m + 1) * (m == 0 ? 2 : 4);
+    const int n = (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
     if (s < n) break;
     s -= n;
   }
-  const int nk = (m == 0) ? 2 : 4, kw = (m == 0) ? 64 : 32;
-  const int kc = s % nk;
+  const int nk = (m == 0) ? 1 : 2;
+  const int kh = s % nk;
   const int l = m + (s / nk) / (L - m + 1), lp = m + (s / nk) % (L - m + 1);
   uint8_t *stage = a.dst + (size_t)blockIdx.x * STAGE_BYTES;
   const int row = threadIdx.x;
   const int n = (L - m + 1) * CH;
   const size_t srow = (size_t)(l - m) * CH + row;
-  const int scol = (lp - m) * CH + kc * kw;
-  const int ntile = (m == 0) ? 1 : 2;
-  for (int t = 0; t < ntile; ++t) {
-    const __nv_bfloat16 *src = (m == 0) ? a.W0 : (t == 0 ? a.Wr[m] : a.Wi[m]);
-    for (int k = 0; k < kw; ++k)
-      *reinterpret_cast<__nv_bfloat16 *>(stage + t * 8192 + kmajor_off(row, k, kw)) = src[srow * n + scol + k];
+  if (m == 0) {
+    const int scol = lp * CH;
+    for (int k = 0; k < 128; ++k)
+      *reinterpret_cast<__nv_bfloat16 *>(stage + kmajor_off(row, k, 128)) = a.W0[srow * n + scol + k];
+  } else {
+    const int scol = (lp - m) * CH + kh * 64;
+    for (int t = 0; t < 2; ++t) {
+      const __nv_bfloat16 *src = (t == 0) ? a.Wr[m] : a.Wi[m];
+      for (int k = 0; k < 64; ++k)
+        *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = src[srow * n + scol + k];
+    }
   }
 }
 
@@ -557,77 +561,93 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       uint32_t rgpar = 0;          // bit sg: parity of the R-GEMMs issued for sign sg
       const uint32_t s_units = smem_addr(units), s_w = smem_addr(wst), s_a2 = smem_addr(A2), s_r = smem_addr(Rb);
       const uint64_t ud0 = smem_desc(s_units, 128, 128 * 16);   // unit 0, K-major, Kc = 128
-      const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 128 x 64 (m = 0)
-      const uint64_t wd32 = smem_desc(s_w, 128, 32 * 16);       // stage 0 as 2 x 128 x 32 (m >= 1)
+      const uint64_t wd128 = smem_desc(s_w, 128, 128 * 16);     // stage 0 as 128 x 128 (m = 0)
+      const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 2 x 128 x 64 (m >= 1)
       const uint64_t a2d = smem_desc(s_a2, 128, 64 * 16);       // A2, MN-major, K = 64 edges
       const uint64_t rd = smem_desc(s_r, 128, 64 * 16);         // R, K-major, K = 64 edges
       int t = 0;
       bool ok = ti.start();
-      auto rgemm = [&](int m, int l, bool first_in_tile) -> bool {
-        const int ng = (m == 0) ? 1 : 2;
-        #pragma unroll 1
-        for (int sg = 0; sg < ng; ++sg) {
-          if (!W.wait(&a2r_full[sg], (rgpar >> sg) & 1)) return false;
-          if (first_in_tile && sg == 0 && t > 0)
-            if (!W.wait(slots_clean, (t - 1) & 1)) return false;
-          tc_fence_after();
-          const uint32_t id = idesc_bf16(128, Cf::NL(l), 1, 0);
-          const uint32_t d = tbase + TM_OUT + Cf::OB(l);
-          const uint64_t ad = a2d + (uint64_t)sg * (A2_BYTES >> 4);
-          const uint64_t bd = rd + (uint64_t)sg * ((Cf::NLMAX * TE * 2) >> 4);
+      // Back-rotation GEMMs are issued as soon as the epilogue hands A2 / R
+      // over, polled between weight stages and inside every wait of this
+      // thread (the epilogue's second sign waits for the first one's GEMM).
+      // Queue head: pass (hm, hl) of tile ht, next sign hs; npend passes whose
+      // y has been committed and whose GEMMs are not all issued.
+      int hm = 0, hl = 0, hs = 0, ht = 0, npend = 0;
+      auto poll_rg = [&]() -> bool {   // false: gave up (abort)
+        if (npend == 0) return true;
+        if (!mbar_try_wait(&a2r_full[hs], (rgpar >> hs) & 1)) return true;
+        if (hm == 0 && hl == 0 && hs == 0 && ht > 0)   // first GEMM of a tile: Out columns cleared
+          if (!W.wait(slots_clean, (ht - 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, Cf::NL(hl), 1, 0);
+        const uint32_t d = tbase + TM_OUT + Cf::OB(hl);
+        const uint64_t bd = rd + (uint64_t)hs * ((Cf::NLMAX * TE * 2) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, ad + 16 * kk, bd + 16 * kk, id, 1u);
-          mma_commit(&rg_done[sg]);
-          rgpar ^= 1u << sg;
+        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, a2d + 16 * kk, bd + 16 * kk, id, 1u);
+        mma_commit(&rg_done[hs]);
+        rgpar ^= 1u << hs;
+        if (++hs == (hm == 0 ? 1 : 2)) {
+          hs = 0;
+          --npend;
+          if (hl < L) ++hl;
+          else if (hm < L) { ++hm; hl = hm; }
+          else { hm = 0; hl = 0; ++ht; }
         }
         return true;
       };
+      auto mw = [&](uint64_t *bar, uint32_t parity) -> bool {
+        for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+          if (mbar_try_wait(bar, parity)) return true;
+          if (!poll_rg()) return false;
+          if ((it & 255) == 255 && W.aborted()) return false;
+        }
+        *abort_flag = 1;
+        atomicExch(a.err, E2F_ERR_TIMEOUT);
+        return false;
+      };
       while (ok && !W.aborted()) {
-        int pm = -1, pl = -1;
-        bool first_rg = true;
+        bool bad = false;
         #pragma unroll 1
-        for (int m = 0; m <= L && !W.aborted(); ++m) {
+        for (int m = 0; m <= L && !bad; ++m) {
           #pragma unroll 1
-          for (int l = m; l <= L; ++l) {
+          for (int l = m; l <= L && !bad; ++l) {
             const uint32_t b = pc & 1;
-            if (!W.wait(&y_empty[b], ((pc >> 1) & 1) ^ 1)) break;
+            if (!mw(&y_empty[b], ((pc >> 1) & 1) ^ 1)) { bad = true; break; }
             tc_fence_after();
             const bool first_pass = (l == m), last_pass = (l == L);
             const uint32_t dp = tbase + 128 * b, dmn = tbase + (16u << 16) + 128 * b;
-            bool bad = false;
             #pragma unroll 1
             for (int lp = m; lp <= L && !bad; ++lp) {
               const int sp = (m == 0) ? lp : 2 * (lp - m);
               if (first_pass) {
-                if (!W.wait(&unit_full[sp], (fillpar >> sp) & 1)) { bad = true; break; }
-                if (m > 0 && !W.wait(&unit_full[sp + 1], (fillpar >> (sp + 1)) & 1)) { bad = true; break; }
+                if (!mw(&unit_full[sp], (fillpar >> sp) & 1)) { bad = true; break; }
+                if (m > 0 && !mw(&unit_full[sp + 1], (fillpar >> (sp + 1)) & 1)) { bad = true; break; }
                 tc_fence_after();
               }
               const bool in_tmem = Cf::TMU && sp >= Cf::NSU;
               // descriptors advance by (byte offset >> 4): 16 per 16-wide K step
               const uint64_t adp = ud0 + (uint64_t)sp * (UNIT_BYTES >> 4), adm = adp + (UNIT_BYTES >> 4);
-              const int nk = (m == 0) ? 2 : 4;
+              const int nk = (m == 0) ? 1 : 2;
               #pragma unroll 1
-              for (int kc = 0; kc < nk; ++kc) {
+              for (int kh = 0; kh < nk; ++kh) {
                 const uint32_t s = st % NSTAGE;
-                if (!W.wait(&w_full[s], (st / NSTAGE) & 1)) { bad = true; break; }
+                if (!mw(&w_full[s], (st / NSTAGE) & 1)) { bad = true; break; }
                 tc_fence_after();
-                const uint32_t acc0 = (lp > m || kc > 0) ? 1u : 0u;
+                const uint32_t acc0 = (lp > m || kh > 0) ? 1u : 0u;
                 if (m == 0) {
-                  // K chunk of 64: 4 steps of 16
-                  const uint64_t bd = wd64 + (uint64_t)s * (STAGE_BYTES >> 4);
-                  const uint64_t ak = adp + 64 * kc;
-                  mma_bf16_ss(dp, ak, bd, ID_MAIN, acc0);
+                  // the whole 128 x 128 block: 8 steps of 16
+                  const uint64_t bd = wd128 + (uint64_t)s * (STAGE_BYTES >> 4);
+                  mma_bf16_ss(dp, adp, bd, ID_MAIN, acc0);
 #pragma unroll
-                  for (int sub = 1; sub < 4; ++sub) mma_bf16_ss(dp, ak + 16 * sub, bd + 16 * sub, ID_MAIN, 1u);
+                  for (int sub = 1; sub < 8; ++sub) mma_bf16_ss(dp, adp + 16 * sub, bd + 16 * sub, ID_MAIN, 1u);
                 } else {
-                  // K chunk of 32: 2 steps of 16
-                  const uint64_t br = wd32 + (uint64_t)s * (STAGE_BYTES >> 4), bi = br + (8192 >> 4);
+                  // K half of 64: 4 steps of 16
+                  const uint64_t br = wd64 + (uint64_t)s * (STAGE_BYTES >> 4), bi = br + (16384 >> 4);
                   if (in_tmem) {
                     // lane half 0 holds [v+ | v-], lane half 1 holds [v- | v+]
-                    const uint32_t a0 = tbase + TM_UNIT + 16 * kc, a1 = a0 + (16u << 16);
+                    const uint32_t a0 = tbase + TM_UNIT + 32 * kh, a1 = a0 + (16u << 16);
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
+                    for (int sub = 0; sub < 4; ++sub) {
                       const uint32_t acc = sub > 0 ? 1u : acc0;
                       mma_bf16_ts(dp, a0 + 8 * sub, br + 16 * sub, ID_MAIN, acc);
                       mma_bf16_ts(dp, a0 + 64 + 8 * sub, bi + 16 * sub, ID_NEGB, 1u);
@@ -635,9 +655,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                       mma_bf16_ts(dmn, a1 + 64 + 8 * sub, bi + 16 * sub, ID_MAIN, 1u);
                     }
                   } else {
-                    const uint64_t ap = adp + 32 * kc, am = adm + 32 * kc;
+                    const uint64_t ap = adp + 64 * kh, am = adm + 64 * kh;
 #pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
+                    for (int sub = 0; sub < 4; ++sub) {
                       const uint32_t acc = sub > 0 ? 1u : acc0;
                       mma_bf16_ss(dp, ap + 16 * sub, br + 16 * sub, ID_MAIN, acc);
                       mma_bf16_ss(dp, am + 16 * sub, bi + 16 * sub, ID_NEGB, 1u);
@@ -648,6 +668,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 }
                 mma_commit(&w_empty[s]);
                 ++st;
+                if (!poll_rg()) { bad = true; break; }
               }
               if (bad) break;
               if (last_pass) {
@@ -659,15 +680,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             if (bad) break;
             mma_commit(&y_full[b]);
             ++pc;
-            if (pm >= 0) {
-              if (!rgemm(pm, pl, first_rg)) break;
-              first_rg = false;
-            }
-            pm = m; pl = l;
+            ++npend;
           }
         }
-        if (W.aborted()) break;
-        if (!rgemm(pm, pl, first_rg)) break;
+        if (bad || W.aborted()) break;
+        // the tile's last back-rotation GEMMs, then hand the tile over
+        for (uint32_t it = 0; npend > 0 && it < WAIT_LIMIT; ++it) {
+          if (!poll_rg()) { bad = true; break; }
+          if ((it & 255) == 255 && W.aborted()) { bad = true; break; }
+        }
+        if (bad || npend > 0) {
+          if (npend > 0 && !bad) { *abort_flag = 1; atomicExch(a.err, E2F_ERR_TIMEOUT); }
+          break;
+        }
         mma_commit(tile_done);
         ++t;
         ok = ti.next();
@@ -750,43 +775,40 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           dead = bar_or(1, 128, f);
           if (dead) break;
           tc_fence_after();
-          // ---- y -> A2 (scaled by alpha g, bf16, MN-major [c][e])
+          // ---- y -> A2 (scaled by alpha g, bf16, MN-major [c][e]), one sign
+          // at a time through the single A2 buffer
           const int sg = lane >> 4;                // 0: y+ rows, 1: y- rows
           const int e = 16 * ew + (lane & 15);
-          const bool act = (m > 0 || sg == 0);
           const int p_ml = m * (L + 1) - m * (m - 1) / 2 + (l - m);
           const float ge = (e < ne) ? __half2float(gs[e * P + p_ml]) : 0.f;
-          uint8_t *a2 = A2 + sg * A2_BYTES;
+          auto to_a2 = [&](int which) {
 #pragma unroll 1
-          for (int i = 0; i < 8; i += 2) {
-            float v[2][16];
-            tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i, v[0]);
-            tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i + 16, v[1]);
-            tmem_ld_wait();
-            if (act) {
+            for (int i = 0; i < 8; i += 2) {
+              float v[2][16];
+              tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i, v[0]);
+              tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i + 16, v[1]);
+              tmem_ld_wait();
+              if (sg == which) {
 #pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
-                const int c0 = 16 * (i + h2);
-                // channels [c0, c0 + 8) and [c0 + 8, c0 + 16) lie in one head each
-                const float s_lo = (e < ne) ? __half2float(al[e * ALS + (c0 >> hshift)]) * ge : 0.f;
-                const float s_hi = (e < ne) ? __half2float(al[e * ALS + ((c0 + 8) >> hshift)]) * ge : 0.f;
-                __align__(16) __nv_bfloat16 o[16];
+                for (int h2 = 0; h2 < 2; ++h2) {
+                  const int c0 = 16 * (i + h2);
+                  // channels [c0, c0 + 8) and [c0 + 8, c0 + 16) lie in one head each
+                  const float s_lo = (e < ne) ? __half2float(al[e * ALS + (c0 >> hshift)]) * ge : 0.f;
+                  const float s_hi = (e < ne) ? __half2float(al[e * ALS + ((c0 + 8) >> hshift)]) * ge : 0.f;
+                  __align__(16) __nv_bfloat16 o[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(v[h2][j] * (j < 8 ? s_lo : s_hi));
-                *reinterpret_cast<uint4 *>(a2 + mnmajor_off(c0, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
-                *reinterpret_cast<uint4 *>(a2 + mnmajor_off(c0 + 8, e, 64)) = *reinterpret_cast<uint4 *>(&o[8]);
+                  for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(v[h2][j] * (j < 8 ? s_lo : s_hi));
+                  *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
+                  *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0 + 8, e, 64)) = *reinterpret_cast<uint4 *>(&o[8]);
+                }
               }
             }
-          }
-          fence_async_smem();
-          tc_fence_before();
-          named_bar(1, 128);
-          if (lane == 0) mbar_arrive(&y_empty[b]);
-          // ---- R for each sign, then hand over to the MMA warp.  R_s has
-          // rows (slot, m') (from row RO(l)), columns edges; the only nonzero
-          // entry of an edge's column is D^l[+-m][m'] in its own slot's rows.
-          // Zero both R buffers, then one thread per (edge, sign) writes its
-          // 2l + 1 entries.
+          };
+          to_a2(0);
+          // ---- R for each sign.  R_s has rows (slot, m') (from row RO(l)),
+          // columns edges; the only nonzero entry of an edge's column is
+          // D^l[+-m][m'] in its own slot's rows.  Zero both R buffers, then one
+          // thread per (edge, sign) writes its 2l + 1 entries.
           const int ng = (m == 0) ? 1 : 2;
           const int w2 = 2 * l + 1;
           const int nrow = Cf::NL(l);
@@ -803,8 +825,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               const __half *d = dy + e * Cf::NDYP;
               const int row0 = Cf::RO(l) + (nodeof[e] % S) * w2;
 #pragma unroll 1
-              for (int t = 0; t < w2; ++t) {
-                const int mp = t - l, amp = mp < 0 ? -mp : mp;
+              for (int tq = 0; tq < w2; ++tq) {
+                const int mp = tq - l, amp = mp < 0 ? -mp : mp;
                 float val = 0.f;
                 if (s2 == 0) {
                   const float de = __half2float(d[dye_off<L>(l) + m * (l + 1) + amp]);
@@ -813,18 +835,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                   const float dd = __half2float(d[dyo_off<L>(l) + (m - 1) * l + (amp - 1)]);
                   val = (mp > 0) ? -dd * snb[(amp - 1) * TE + e] : dd * csb[(amp - 1) * TE + e];
                 }
-                *reinterpret_cast<__nv_bfloat16 *>(Rs + kmajor_off(row0 + t, e, 64)) = __float2bfloat16_rn(val);
+                *reinterpret_cast<__nv_bfloat16 *>(Rs + kmajor_off(row0 + tq, e, 64)) = __float2bfloat16_rn(val);
               }
             }
           }
           fence_async_smem();
           named_bar(1, 128);
-          if (et == 0) {
-            mbar_arrive(&a2r_full[0]);
-            if (ng > 1) mbar_arrive(&a2r_full[1]);
-          }
+          if (et == 0) mbar_arrive(&a2r_full[0]);
           ++nA0;
-          if (ng > 1) ++nA1;
+          if (ng > 1) {
+            // the second sign waits for the first sign's GEMM to release A2
+            bool f2 = false;
+            if (et == 0) f2 = !W.wait(&rg_done[0], (nA0 - 1) & 1, 20);
+            dead = bar_or(1, 128, f2);
+            if (dead) break;
+            to_a2(1);
+            fence_async_smem();
+            named_bar(1, 128);
+            if (et == 0) mbar_arrive(&a2r_full[1]);
+            ++nA1;
+          }
+          tc_fence_before();
+          named_bar(1, 128);
+          if (lane == 0) mbar_arrive(&y_empty[b]);   // y of this pass fully read
           ++pc;
         }
       }
@@ -1319,7 +1352,7 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   }
   // pack weights
   int nst = 0;
-  for (int m = 0; m <= L; ++m) nst += (L - m + 1) * (L - m + 1) * (m == 0 ? 2 : 4);
+  for (int m = 0; m <= L; ++m) nst += (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
   const size_t wbytes = (size_t)nst * STAGE_BYTES;
   Scratch wp, st;
   E2F_CUDA_TRY(wp.alloc(wbytes, s));

@@ -397,16 +397,123 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# per-row measurements (one JSON line per hot-path row and workload)
+# ----------------------------------------------------------------------------
+def run_rows(args):
+    """Each row of the hot path against its own roofline, on every workload:
+    the neighbour build (HBM: algorithmic bytes 12N + 4(N+1) + 4E, the
+    positions read, row_ptr and col_idx written) and the fused attention
+    (tensor: F(L, C) FLOP per edge), plus peak device memory against N on the
+    water-box sweep.  Times are CUDA events on the working stream, median of
+    `--steps` calls after `--warmup`; the neighbour build's time includes its
+    two host read-backs (bounding box, edge count)."""
+    import torch
+    from atomistic_mlip_b200 import e2f
+    from atomistic_mlip_b200 import workloads as w
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --rows needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    e2f.lib()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, reps):
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def one(cfg, n_target=None, attention=True, reps=None):
+        steps = args.steps if reps is None else reps
+        warm = args.warmup if reps is None else 1
+        wl = w.make_workload(cfg, n_target=n_target)
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        e2f.scratch_high_water(reset=True)
+        pos = torch.from_numpy(wl.pos).to(dev)
+        x = torch.from_numpy(wl.x).to(dev, torch.bfloat16 if wl.precision == "bf16" else torch.float32)
+        dw = e2f.DeviceWeights.from_workload(wl, dev)
+        box = None if wl.box is None else [float(b) for b in wl.box]
+        nl = e2f.build_neighbors(pos, box, wl.r_c)
+        cap = nl.n_edges
+        row_ptr = torch.empty(wl.N + 1, dtype=torch.int32, device=dev)
+        col_idx = torch.empty(max(1, cap), dtype=torch.int32, device=dev)
+
+        def nb():
+            e2f.build_neighbors(pos, box, wl.r_c, row_ptr=row_ptr, col_idx=col_idx)
+        for _ in range(warm):
+            nb()
+        t_nb = timed(nb, steps)
+        E = nl.n_edges
+        nb_bytes = 12 * wl.N + 4 * (wl.N + 1) + 4 * E
+        out = {"row": "A1-A3 neighbour build", "workload": wl.cfg_name if hasattr(wl, "cfg_name") else f"cfg{cfg}",
+               "N": wl.N, "E": E, "ms": t_nb,
+               "roofline": {"bound": "hbm", "algorithmic_bytes": nb_bytes,
+                            "achieved": nb_bytes / (t_nb * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
+                            "unit": "GB/s", "frac": nb_bytes / (t_nb * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                            "peak_source": f"hbm_gbs, {peak_src}"}}
+        print(json.dumps(out), flush=True)
+        if not attention:
+            return
+        o = torch.empty((wl.N, (wl.L + 1) ** 2, wl.C), dtype=torch.float32, device=dev)
+
+        def att():
+            e2f.attention_forward(x, pos, nl, dw, out=o)
+        for _ in range(warm):
+            att()
+        e2f.profile_enable(True)
+        t_call = timed(att, steps)
+        e2f.profile_enable(False)
+        n_k, k_ms = e2f.profile_read()
+        k_ms = k_ms / max(n_k, 1)
+        F = so2_flops_per_edge(wl.L, wl.C)
+        peak = float(peaks["bf16_tflops"])
+        out = {"row": "A4-A11 attention forward (projections + fused kernel)", "workload": f"cfg{cfg}",
+               "N": wl.N, "E": E, "L": wl.L, "C": wl.C, "H": wl.H, "precision": wl.precision,
+               "call_ms": t_call, "fused_kernel_ms": k_ms,
+               "edges_per_s": E / (t_call * 1e-3), "node_updates_per_s": wl.N / (t_call * 1e-3),
+               "roofline": {"bound": "tensor", "flops_per_edge": F, "achieved": F * E / (k_ms * 1e-3) / 1e12,
+                            "peak": peak, "unit": "TFLOP/s", "frac": F * E / (k_ms * 1e-3) / 1e12 / peak,
+                            "peak_source": f"bf16_tflops burst, {peak_src}",
+                            "path": "tcgen05" if (wl.precision == "bf16" and wl.C == 128 and 1 <= wl.L <= 4) else "SIMT"},
+               "peak_device_bytes": {"torch": int(torch.cuda.max_memory_allocated(dev)),
+                                     "library_scratch": int(e2f.scratch_high_water())}}
+        print(json.dumps(out), flush=True)
+        del o
+
+    if args.rows_what == "neighbors":
+        one(4, attention=False)
+        return
+    for cfg in (1, 2, 4):
+        one(cfg)
+    for n in (10002, 30000):   # memory sweep of the water box (cfg4 is the 100k point)
+        one(4, n_target=n)
+    one(3, reps=1)   # L = 6 runs on the SIMT kernel: one timed call
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rows", action="store_true", help="per-row measurements on every workload (one GPU)")
+    ap.add_argument("--rows-what", choices=["all", "neighbors"], default="all",
+                    help="with --rows: every row, or the neighbour build of the 100k-atom water box only")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.rows:
+        run_rows(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

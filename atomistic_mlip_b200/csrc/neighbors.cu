@@ -5,8 +5,9 @@
 // Steps (all on `stream`):
 //   bbox (open dims only; one host read)  -> grid of cells of edge >= r_c
 //   cell_assign: cell of each atom + per-cell counts (+ domain check)
-//   scan -> cell_start;  cell_scatter -> atoms grouped by cell
-//   count: warp per atom over the 27-cell stencil, exact fp32 predicate
+//   scan -> cell_start;  cell_scatter -> positions grouped by cell
+//   count: warp per atom (in cell order) over the 27-cell stencil, exact
+//          fp32 predicate
 //   scan -> row_ptr, E read back (one host read), capacity check
 //   fill: warp per atom, same stencil; the row is collected in shared
 //         memory and written in ascending j (rank placement), or, for rows
@@ -94,61 +95,95 @@ __global__ void cell_assign_kernel(const float *__restrict__ pos, int n, CellGri
   atomicAdd(&cell_count[cid], 1);
 }
 
-__global__ void cell_scatter_kernel(const int32_t *__restrict__ cell_of, int n,
+// Atoms grouped by cell: spos[k] = (x_i, y_i, z_i, bits of i) for the k-th
+// atom in cell order, so that a candidate is one 16-byte load.
+__global__ void cell_scatter_kernel(const float *__restrict__ pos, const int32_t *__restrict__ cell_of, int n,
                                     const int32_t *__restrict__ cell_start, int32_t *__restrict__ cursor,
-                                    int32_t *__restrict__ atom_by_cell) {
+                                    float4 *__restrict__ spos) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int c = cell_of[i];
-  const int slot = atomicAdd(&cursor[c], 1);
-  atom_by_cell[cell_start[c] + slot] = i;
+  const int k = cell_start[c] + atomicAdd(&cursor[c], 1);
+  const float3 p = load_pos(pos, i);
+  spos[k] = make_float4(p.x, p.y, p.z, __int_as_float(i));
 }
 
-// Visit the stencil cells of atom i; f(j) is called by each lane for its
-// candidates (all lanes of the warp iterate together, inactive lanes get -1).
+// Visit the stencil cells of atom i.  The (start, length) of the 27 stencil
+// cells are loaded at once (lane c holds cell c), then the cells are taken
+// four at a time: the atom indices of four cells, then their positions, are
+// loaded before any is used, so a warp waits for a few round trips instead
+// of three per cell.  f(j, pj) is called by every lane for each candidate
+// slot (inactive lanes get j = -1); candidates beyond 32 per cell (dense
+// cells) are visited in extra rounds.  Candidates come from the cell-sorted
+// positions (one 16-byte load: coordinates and the atom's index).
 template <typename F>
 __device__ __forceinline__ void for_stencil(int cid, const CellGrid &cg, const Geom &g,
-                                            const int32_t *__restrict__ cell_start,
-                                            const int32_t *__restrict__ atom_by_cell, int lane, F &&f) {
+                                            const float4 *__restrict__ spos,
+                                            const int32_t *__restrict__ cell_start, int lane, F &&f) {
   const int cx = cid % cg.nc[0];
   const int cy = (cid / cg.nc[0]) % cg.nc[1];
   const int cz = cid / (cg.nc[0] * cg.nc[1]);
-  const int rz = cg.stencil[2], ry = cg.stencil[1], rx = cg.stencil[0];
-  for (int dz = -rz; dz <= rz; ++dz) {
-    int z = cz + dz;
-    if (g.periodic[2]) z = (z + cg.nc[2]) % cg.nc[2];
-    else if (z < 0 || z >= cg.nc[2]) continue;
-    for (int dy = -ry; dy <= ry; ++dy) {
-      int y = cy + dy;
-      if (g.periodic[1]) y = (y + cg.nc[1]) % cg.nc[1];
-      else if (y < 0 || y >= cg.nc[1]) continue;
-      for (int dx = -rx; dx <= rx; ++dx) {
-        int x = cx + dx;
-        if (g.periodic[0]) x = (x + cg.nc[0]) % cg.nc[0];
-        else if (x < 0 || x >= cg.nc[0]) continue;
-        const int c = x + cg.nc[0] * (y + cg.nc[1] * z);
-        const int s = cell_start[c], e = cell_start[c + 1];
-        for (int t = s; t < e; t += 32) {
-          const int idx = t + lane;
-          f(idx < e ? atom_by_cell[idx] : -1);
-        }
+  int my_s = 0, my_n = 0;
+  if (lane < 27) {
+    const int d[3] = {lane % 3 - 1, (lane / 3) % 3 - 1, lane / 9 - 1};
+    const int c0[3] = {cx, cy, cz};
+    int cc[3];
+    bool ok = true;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      if (d[k] != 0 && cg.stencil[k] == 0) ok = false;
+      int v = c0[k] + d[k];
+      if (g.periodic[k]) v = (v + cg.nc[k]) % cg.nc[k];
+      else if (v < 0 || v >= cg.nc[k]) ok = false;
+      cc[k] = v;
+    }
+    if (ok) {
+      const int c = cc[0] + cg.nc[0] * (cc[1] + cg.nc[1] * cc[2]);
+      my_s = cell_start[c];
+      my_n = cell_start[c + 1] - my_s;
+    }
+  }
+  for (int q0 = 0; q0 < 27; q0 += 4) {
+    int st[4], nn[4], j[4];
+    float3 pj[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      st[q] = __shfl_sync(0xffffffffu, my_s, (q0 + q) & 31);
+      nn[q] = (q0 + q < 27) ? __shfl_sync(0xffffffffu, my_n, (q0 + q) & 31) : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = lane < nn[q] ? spos[st[q] + lane] : make_float4(0.f, 0.f, 0.f, __int_as_float(-1));
+      j[q] = __float_as_int(v.w);
+      pj[q] = make_float3(v.x, v.y, v.z);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) f(j[q], pj[q]);
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      for (int t = 32; t < nn[q]; t += 32) {   // cells with more than 32 atoms
+        const float4 v = t + lane < nn[q] ? spos[st[q] + t + lane] : make_float4(0.f, 0.f, 0.f, __int_as_float(-1));
+        f(__float_as_int(v.w), make_float3(v.x, v.y, v.z));
       }
     }
   }
 }
 
-__global__ void count_kernel(const float *__restrict__ pos, int n, CellGrid cg, Geom g,
-                             const int32_t *__restrict__ cell_of, const int32_t *__restrict__ cell_start,
-                             const int32_t *__restrict__ atom_by_cell, int32_t *__restrict__ deg) {
+__global__ void count_kernel(int n, CellGrid cg, Geom g, const int32_t *__restrict__ cell_of,
+                             const int32_t *__restrict__ cell_start, const float4 *__restrict__ spos,
+                             int32_t *__restrict__ deg) {
+  // warp per atom, atoms taken in cell order
   const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * NB_WARPS + (threadIdx.x >> 5);
-  if (i >= n) return;
-  const float3 pi = load_pos(pos, i);
+  const int k = blockIdx.x * NB_WARPS + (threadIdx.x >> 5);
+  if (k >= n) return;
+  const float4 me = spos[k];
+  const int i = __float_as_int(me.w);
+  const float3 pi = make_float3(me.x, me.y, me.z);
   int cnt = 0;
-  for_stencil(cell_of[i], cg, g, cell_start, atom_by_cell, lane, [&](int j) {
+  for_stencil(cell_of[i], cg, g, spos, cell_start, lane, [&](int j, float3 pj) {
     if (j >= 0 && j != i) {
       float dx, dy, dz;
-      pair_disp(g, pi, load_pos(pos, j), dx, dy, dz);
+      pair_disp(g, pi, pj, dx, dy, dz);
       if (pair_r2(dx, dy, dz) < g.rc2) ++cnt;
     }
   });
@@ -156,26 +191,27 @@ __global__ void count_kernel(const float *__restrict__ pos, int n, CellGrid cg, 
   if (lane == 0) deg[i] = cnt;
 }
 
-__global__ void fill_kernel(const float *__restrict__ pos, int n, CellGrid cg, Geom g,
-                            const int32_t *__restrict__ cell_of, const int32_t *__restrict__ cell_start,
-                            const int32_t *__restrict__ atom_by_cell, const int32_t *__restrict__ row_ptr,
-                            int32_t *__restrict__ col_idx) {
+__global__ void fill_kernel(int n, CellGrid cg, Geom g, const int32_t *__restrict__ cell_of,
+                            const int32_t *__restrict__ cell_start, const float4 *__restrict__ spos,
+                            const int32_t *__restrict__ row_ptr, int32_t *__restrict__ col_idx) {
   __shared__ int32_t buf[NB_WARPS][ROW_CAP];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int i = blockIdx.x * NB_WARPS + wid;
-  if (i >= n) return;
+  const int k = blockIdx.x * NB_WARPS + wid;
+  if (k >= n) return;
+  const float4 me = spos[k];
+  const int i = __float_as_int(me.w);
   const int r0 = row_ptr[i];
   const int deg = row_ptr[i + 1] - r0;
   const bool in_smem = deg <= ROW_CAP;
   int32_t *row = col_idx + r0;
   int32_t *b = buf[wid];
-  const float3 pi = load_pos(pos, i);
+  const float3 pi = make_float3(me.x, me.y, me.z);
   int w = 0;
-  for_stencil(cell_of[i], cg, g, cell_start, atom_by_cell, lane, [&](int j) {
+  for_stencil(cell_of[i], cg, g, spos, cell_start, lane, [&](int j, float3 pj) {
     bool pass = false;
     if (j >= 0 && j != i) {
       float dx, dy, dz;
-      pair_disp(g, pi, load_pos(pos, j), dx, dy, dz);
+      pair_disp(g, pi, pj, dx, dy, dz);
       pass = pair_r2(dx, dy, dz) < g.rc2;
     }
     const unsigned m = __ballot_sync(0xffffffffu, pass);
@@ -283,12 +319,12 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
       if (!g.periodic[k]) cs[k] *= 1.25;
   }
 
-  Scratch cell_of, cnt, cstart, cursor, abc, deg, flag, scan_tmp;
+  Scratch cell_of, cnt, cstart, cursor, deg, flag, scan_tmp, spos;
   E2F_CUDA_TRY(cell_of.alloc(sizeof(int32_t) * n, s));
   E2F_CUDA_TRY(cnt.alloc(sizeof(int32_t) * ncell, s));
   E2F_CUDA_TRY(cstart.alloc(sizeof(int32_t) * (ncell + 1), s));
   E2F_CUDA_TRY(cursor.alloc(sizeof(int32_t) * ncell, s));
-  E2F_CUDA_TRY(abc.alloc(sizeof(int32_t) * n, s));
+  E2F_CUDA_TRY(spos.alloc(sizeof(float4) * n, s));
   E2F_CUDA_TRY(deg.alloc(sizeof(int32_t) * n, s));
   E2F_CUDA_TRY(flag.alloc(sizeof(int32_t) * 4, s));
   E2F_CUDA_TRY(scan_tmp.alloc(std::max(scan_scratch_bytes(ncell), scan_scratch_bytes(n)), s));
@@ -301,11 +337,11 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
              cnt.as<int32_t>(), flag.as<int32_t>());
   e2f_status st = exclusive_scan(cnt.as<int32_t>(), ncell, cstart.as<int32_t>(), scan_tmp.p, s, nullptr);
   if (st != E2F_OK) return st;
-  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, cell_of.as<int32_t>(), n,
-             cstart.as<int32_t>(), cursor.as<int32_t>(), abc.as<int32_t>());
+  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, pos, cell_of.as<int32_t>(), n,
+             cstart.as<int32_t>(), cursor.as<int32_t>(), spos.as<float4>());
   const int nblk = (n + NB_WARPS - 1) / NB_WARPS;
-  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of.as<int32_t>(),
-             cstart.as<int32_t>(), abc.as<int32_t>(), deg.as<int32_t>());
+  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of.as<int32_t>(), cstart.as<int32_t>(),
+             spos.as<float4>(), deg.as<int32_t>());
   long long *total = nullptr;
   st = exclusive_scan(deg.as<int32_t>(), n, row_ptr, scan_tmp.p, s, &total);
   if (st != E2F_OK) return st;
@@ -321,8 +357,8 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
   if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
   if (E > capacity) return E2F_ERR_CAPACITY;
   if (E > 0) {
-    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of.as<int32_t>(),
-               cstart.as<int32_t>(), abc.as<int32_t>(), row_ptr, col_idx);
+    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of.as<int32_t>(), cstart.as<int32_t>(),
+               spos.as<float4>(), row_ptr, col_idx);
   }
   return E2F_OK;
 }
@@ -349,15 +385,16 @@ constexpr int64_t NOALLOC_MAX_CELLS = 1 << 17;   // 131,072 cells
 
 // layout of the array, in 4-byte words (offsets kept 64-word aligned)
 constexpr size_t NA_CELL_OF = 0;
-constexpr size_t NA_ABC = NA_CELL_OF + NOALLOC_MAX_ATOMS;
-constexpr size_t NA_DEG = NA_ABC + NOALLOC_MAX_ATOMS;
+constexpr size_t NA_DEG = NA_CELL_OF + NOALLOC_MAX_ATOMS;
 constexpr size_t NA_CNT = NA_DEG + NOALLOC_MAX_ATOMS;
 constexpr size_t NA_CSTART = NA_CNT + NOALLOC_MAX_CELLS;
 constexpr size_t NA_CURSOR = NA_CSTART + NOALLOC_MAX_CELLS + 64;
 constexpr size_t NA_FLAG = NA_CURSOR + NOALLOC_MAX_CELLS;
 constexpr size_t NA_BBOX = NA_FLAG + 64;
 constexpr size_t NA_SCAN = NA_BBOX + 2048;        // 6 * 256 + 6 floats fit
-constexpr size_t NA_WORDS = NA_SCAN + 256;        // scan sums: long longs
+constexpr size_t NA_SPOS = NA_SCAN + 256;         // scan sums: long longs; then float4 per atom
+constexpr size_t NA_WORDS = NA_SPOS + 4 * NOALLOC_MAX_ATOMS;
+static_assert(NA_SPOS % 4 == 0, "cell-sorted positions need 16-byte alignment");
 static_assert(NA_SCAN % 2 == 0, "scan sums need 8-byte alignment");
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[NA_WORDS];
@@ -462,8 +499,9 @@ static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, cons
       cg.stencil[k] = cg.nc[k] >= 3 ? 1 : 0;
     }
   }
-  int32_t *cell_of = ws + NA_CELL_OF, *abc = ws + NA_ABC, *deg = ws + NA_DEG;
+  int32_t *cell_of = ws + NA_CELL_OF, *deg = ws + NA_DEG;
   int32_t *cnt = ws + NA_CNT, *cstart = ws + NA_CSTART, *cursor = ws + NA_CURSOR, *flag = ws + NA_FLAG;
+  float4 *spos = reinterpret_cast<float4 *>(ws + NA_SPOS);
   void *scan_tmp = ws + NA_SCAN;
   E2F_CUDA_TRY(cudaMemsetAsync(cnt, 0, sizeof(int32_t) * ncell, s));
   E2F_CUDA_TRY(cudaMemsetAsync(cursor, 0, sizeof(int32_t) * ncell, s));
@@ -472,9 +510,9 @@ static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, cons
   E2F_LAUNCH(cell_assign_kernel, (n + tb - 1) / tb, tb, 0, s, pos, n, cg, g, cell_of, cnt, flag);
   st = exclusive_scan(cnt, ncell, cstart, scan_tmp, s, nullptr);
   if (st != E2F_OK) return st;
-  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, cell_of, n, cstart, cursor, abc);
+  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, pos, cell_of, n, cstart, cursor, spos);
   const int nblk = (n + NB_WARPS - 1) / NB_WARPS;
-  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of, cstart, abc, deg);
+  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of, cstart, spos, deg);
   long long *total = nullptr;
   st = exclusive_scan(deg, n, row_ptr, scan_tmp, s, &total);
   if (st != E2F_OK) return st;
@@ -488,7 +526,7 @@ static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, cons
   if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
   if (E > capacity) return E2F_ERR_CAPACITY;
   if (E > 0) {
-    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, pos, n, cg, g, cell_of, cstart, abc, row_ptr, col_idx);
+    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of, cstart, spos, row_ptr, col_idx);
   }
   return E2F_OK;
 }

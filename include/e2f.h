@@ -119,7 +119,7 @@ E2F_API e2f_status e2f_build_neighbors(const float *pos, int64_t N, const float 
  * meet an allocation (its failure mode, its implicit synchronisation) in
  * the middle of a step.
  *
- * All temporary arrays live in one fixed array of about 3.2 MB that is part
+ * All temporary arrays live in one fixed array of about 4.7 MB that is part
  * of the library's device image, so every GPU that loads the library holds
  * it until the process exits.  The caller still passes pos, row_ptr and
  * col_idx; arguments, result and status codes are those of

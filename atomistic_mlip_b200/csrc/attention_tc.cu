@@ -44,12 +44,10 @@ namespace tca {
 using namespace tc;
 
 constexpr int CH = 128;            // channels on this path
-constexpr int TE = 64;             // edges per tile (MMA M)
+constexpr int TE64 = 64;           // edges per tile for L <= 4 (MMA M)
 constexpr int S = 4;               // destination-node slots per tile
 constexpr int NSTAGE = 2;          // weight ring stages
 constexpr int STAGE_BYTES = 32768; // one weight stage: W0 128 x 128, or Wr|Wi 128 x 64 each
-constexpr int UNIT_BYTES = TE * CH * 2;
-constexpr int A2_BYTES = CH * TE * 2;
 constexpr int NTHREADS = 512;
 constexpr int HMAX = 16;
 constexpr int ALS = HMAX + 1;     // alpha row stride (odd: conflict-free per-edge rows)
@@ -61,12 +59,19 @@ constexpr uint32_t TM_OUT = 256;
 constexpr uint32_t TM_UNIT = 384;
 
 template <int L> struct Cfg {
+  // Tile edges: 64 up to L = 4; 32 for L = 5, 6, where the SO(2) units of
+  // one degree m would not fit otherwise.  With 32 edges the M = 64 MMA reads
+  // its rows 32..63 from the next unit (units are contiguous), whose rows of
+  // D are never used.
+  static constexpr int TE = L >= 5 ? 32 : TE64;
+  static constexpr int UNIT_BYTES = TE * CH * 2;
+  static constexpr int A2_BYTES = CH * TE * 2;
   static constexpr int Q = (L + 1) * (L + 1);
   static constexpr int P = (L + 1) * (L + 2) / 2;
   static constexpr int NUNIT = (L + 1 > 2 * L) ? L + 1 : 2 * L;
   // From L = 3 on, the unit pair of (m = 1, l' = L) lives in TMEM: those two
   // units are used by the m = 1 passes only, and shared memory is tight.
-  static constexpr bool TMU = (L >= 3);
+  static constexpr bool TMU = (L == 3 || L == 4);
   static constexpr int TMU_SP = 2 * L - 2;                 // first TMEM unit index
   static constexpr int NSU = TMU ? NUNIT - 2 : NUNIT;      // units in shared memory
   static constexpr int NDYE = (L + 1) * (L + 2) * (2 * L + 3) / 6;   // sum (l+1)^2
@@ -78,15 +83,20 @@ template <int L> struct Cfg {
   // the block only ever receives exact zeros (zero rows of R), so real
   // columns of another degree may sit there.
   static __host__ __device__ constexpr int NL(int l) { return ((S * (2 * l + 1) + 15) / 16) * 16; }
-  static __host__ __device__ constexpr int OB(int l) {
-    return l <= 1 ? 0 : (l == 2 ? (L >= 3 ? 32 : 16) : (l == 3 ? 16 : 64));
+  static __host__ __device__ constexpr int OCB(int l) {   // plain consecutive blocks
+    int s = 0;
+    for (int k = 0; k < l; ++k) s += NL(k);
+    return s;
   }
-  static __host__ __device__ constexpr int RO(int l) { return l == 0 ? 12 : (l == 2 && L >= 3 ? 12 : 0); }
-  static constexpr int OUT_COLS = L == 1 ? 16 : (L == 2 ? 48 : (L == 3 ? 64 : 112));
+  static __host__ __device__ constexpr int OB(int l) {
+    return L >= 5 ? OCB(l) : (l <= 1 ? 0 : (l == 2 ? (L >= 3 ? 32 : 16) : (l == 3 ? 16 : 64)));
+  }
+  static __host__ __device__ constexpr int RO(int l) { return L >= 5 ? 0 : (l == 0 ? 12 : (l == 2 && L >= 3 ? 12 : 0)); }
+  static constexpr int OUT_COLS = L >= 5 ? OCB(L + 1) : (L == 1 ? 16 : (L == 2 ? 48 : (L == 3 ? 64 : 112)));
   static constexpr int NLMAX = NL(L);
   // shared-memory carve-up (bytes)
   static constexpr size_t OFF_UNIT = 0;
-  static constexpr size_t OFF_W = OFF_UNIT + (size_t)NSU * UNIT_BYTES;
+  static constexpr size_t OFF_W = OFF_UNIT + (size_t)(NSU + (TE < 64 ? 1 : 0)) * UNIT_BYTES;
   static constexpr size_t OFF_A2 = OFF_W + (size_t)NSTAGE * STAGE_BYTES;
   static constexpr size_t OFF_R = OFF_A2 + (size_t)A2_BYTES;   // one A2 buffer: the signs take turns
   // per-tile geometry, two copies (tile parity): the producers build the
@@ -105,7 +115,7 @@ template <int L> struct Cfg {
   static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 7;
   static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(TM_OUT + OUT_COLS <= TM_UNIT, "TMEM budget");
+  static_assert(TM_OUT + OUT_COLS <= (TMU ? TM_UNIT : 512u), "TMEM budget");
   // weight stages per tile
   static __host__ __device__ constexpr int stages_of_m(int m) { return (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2); }
   static __host__ __device__ constexpr int stages_per_tile() {
@@ -175,12 +185,13 @@ struct Waiter {
 struct TileIter {
   const int32_t *rp;
   int N;
+  int te;   // edges per tile
   int64_t ebeg, eend;
   int64_t e0, e1;
   int n0;
   __device__ void bounds() {
     const int nlim = min(n0 + S, N);
-    int64_t e = e0 + TE;
+    int64_t e = e0 + te;
     if (eend < e) e = eend;
     if ((int64_t)rp[nlim] < e) e = rp[nlim];
     e1 = e;
@@ -490,6 +501,7 @@ template <int L>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   using Cf = Cfg<L>;
   constexpr int Q = Cf::Q, P = Cf::P, NUNIT = Cf::NUNIT;
+  constexpr int TE = Cf::TE, UNIT_BYTES = Cf::UNIT_BYTES, A2_BYTES = Cf::A2_BYTES;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -545,7 +557,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   Waiter W{abort_flag, a.err};
 
   TileIter ti;
-  ti.rp = a.row_ptr; ti.N = a.N;
+  ti.rp = a.row_ptr; ti.N = a.N; ti.te = Cf::TE;
   ti.ebeg = a.E * (int64_t)blockIdx.x / gridDim.x;
   ti.eend = a.E * (int64_t)(blockIdx.x + 1) / gridDim.x;
   const int H = a.H, Ch = CH / H;
@@ -563,8 +575,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       const uint64_t ud0 = smem_desc(s_units, 128, 128 * 16);   // unit 0, K-major, Kc = 128
       const uint64_t wd128 = smem_desc(s_w, 128, 128 * 16);     // stage 0 as 128 x 128 (m = 0)
       const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 2 x 128 x 64 (m >= 1)
-      const uint64_t a2d = smem_desc(s_a2, 128, 64 * 16);       // A2, MN-major, K = 64 edges
-      const uint64_t rd = smem_desc(s_r, 128, 64 * 16);         // R, K-major, K = 64 edges
+      const uint64_t a2d = smem_desc(s_a2, 128, TE * 16);       // A2, MN-major, K = TE edges
+      const uint64_t rd = smem_desc(s_r, 128, TE * 16);         // R, K-major, K = TE edges
       int t = 0;
       bool ok = ti.start();
       // Back-rotation GEMMs are issued as soon as the epilogue hands A2 / R
@@ -583,7 +595,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         const uint32_t d = tbase + TM_OUT + Cf::OB(hl);
         const uint64_t bd = rd + (uint64_t)hs * ((Cf::NLMAX * TE * 2) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, a2d + 16 * kk, bd + 16 * kk, id, 1u);
+        for (int kk = 0; kk < TE / 16; ++kk) mma_bf16_ss(d, a2d + 16 * kk, bd + 16 * kk, id, 1u);
         mma_commit(&rg_done[hs]);
         rgpar ^= 1u << hs;
         if (++hs == (hm == 0 ? 1 : 2)) {
@@ -798,8 +810,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                   __align__(16) __nv_bfloat16 o[16];
 #pragma unroll
                   for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(v[h2][j] * (j < 8 ? s_lo : s_hi));
-                  *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0, e, 64)) = *reinterpret_cast<uint4 *>(&o[0]);
-                  *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0 + 8, e, 64)) = *reinterpret_cast<uint4 *>(&o[8]);
+                  if (e < TE) {   // TMEM rows of edges >= TE (32-edge tiles) are not real
+                    *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0, e, TE)) = *reinterpret_cast<uint4 *>(&o[0]);
+                    *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0 + 8, e, TE)) = *reinterpret_cast<uint4 *>(&o[8]);
+                  }
                 }
               }
             }
@@ -812,14 +826,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const int ng = (m == 0) ? 1 : 2;
           const int w2 = 2 * l + 1;
           const int nrow = Cf::NL(l);
-          for (int idx = et; idx < ng * nrow * 8; idx += 128) {
-            const int s2 = idx / (nrow * 8), rem = idx - s2 * nrow * 8;
-            *reinterpret_cast<uint4 *>(Rb + (size_t)s2 * Cf::NLMAX * TE * 2 + kmajor_off(rem >> 3, (rem & 7) * 8, 64)) =
+          constexpr int RCH = TE / 8;   // 16-byte chunks per R row
+          for (int idx = et; idx < ng * nrow * RCH; idx += 128) {
+            const int s2 = idx / (nrow * RCH), rem = idx - s2 * nrow * RCH;
+            *reinterpret_cast<uint4 *>(Rb + (size_t)s2 * Cf::NLMAX * TE * 2 + kmajor_off(rem / RCH, (rem % RCH) * 8, TE)) =
                 make_uint4(0u, 0u, 0u, 0u);
           }
           named_bar(1, 128);
           {
-            const int e = et & (TE - 1), s2 = et >> 6;
+            const int e = et % TE, s2 = et / TE;
             if (s2 < ng && e < ne) {
               uint8_t *Rs = Rb + (size_t)s2 * Cf::NLMAX * TE * 2;
               const __half *d = dy + e * Cf::NDYP;
@@ -835,7 +850,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                   const float dd = __half2float(d[dyo_off<L>(l) + (m - 1) * l + (amp - 1)]);
                   val = (mp > 0) ? -dd * snb[(amp - 1) * TE + e] : dd * csb[(amp - 1) * TE + e];
                 }
-                *reinterpret_cast<__nv_bfloat16 *>(Rs + kmajor_off(row0 + tq, e, 64)) = __float2bfloat16_rn(val);
+                *reinterpret_cast<__nv_bfloat16 *>(Rs + kmajor_off(row0 + tq, e, TE)) = __float2bfloat16_rn(val);
               }
             }
           }
@@ -931,7 +946,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       int *jj = g_jj(c), *nodeof = jj + TE;
       float *csb = g_cs(c), *snb = csb + TE * (L > 0 ? L : 1);
       __half *gs = g_gs(c);
-      const int e = pt >> 2, q4 = pt & 3;
+      const int e = pt >> 2, q4 = pt & 3;   // (TE < 64: threads past 4 TE only help the shuffles)
       const bool live = e < ne;
       float r = 0.f;
       if (live) {
@@ -961,7 +976,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           geo[e * 4 + 1] = rho;
           geo[e * 4 + 2] = 0.5f * (cospif(r / a.g.rc) + 1.f);
         }
-      } else if (q4 == 0) {
+      } else if (q4 == 0 && e < TE) {
         jj[e] = -1;
         nodeof[e] = -1;
         for (int mm = 0; mm < L; ++mm) { csb[mm * TE + e] = 1.f; snb[mm * TE + e] = 0.f; }
@@ -989,7 +1004,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         for (int h = 0; h < 4; ++h) gv = fmaf(__ldg(a.W2 + p * 16 + 4 * q4 + h), hid[h], gv);
         gv += __shfl_xor_sync(0xffffffffu, gv, 1);
         gv += __shfl_xor_sync(0xffffffffu, gv, 2);
-        if ((p & 3) == q4) gs[e * P + p] = __float2half_rn(live ? gv : 0.f);
+        if ((p & 3) == q4 && e < TE) gs[e * P + p] = __float2half_rn(live ? gv : 0.f);
       }
     };
     // ---- Wigner blocks of Ry(-theta), parity blocks straight to fp16:
@@ -1015,7 +1030,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         for (int jd = 0; jd <= L; ++jd) cc[jd] = cf[1 + jd];   // zero above the entry's degree
         const bool eps = cf[0] != 0.f;
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
+        for (int h2 = 0; h2 < TE / 32; ++h2) {
           const int e = lane + 32 * h2;
           const float ct = geo[e * 4 + 0], stt = geo[e * 4 + 1];
           float p = cc[L];
@@ -1146,13 +1161,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           // gathered rows of block b + 1 are loaded while block b is computed;
           // pairs of channels go through packed fp32 FMAs.  emit(b, wp, wm)
           // receives block b as packed bf16 pairs (wp: +m, wm: -m).
-          auto rot4 = [&](auto LPc, int e, const int (&cbs)[4], auto &&emit) {
+          auto rot4 = [&](auto LPc, int e, const auto &cbs, auto &&emit) {
             constexpr int LP = decltype(LPc)::value;
             constexpr int NR = 2 * LP + 1;
+            constexpr int NB = (int)(sizeof(cbs) / sizeof(int));   // channel blocks of this thread
             if (e >= ne) {
               const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-              for (int bb = 0; bb < 4; ++bb) emit(bb, z, z);
+              for (int bb = 0; bb < NB; ++bb) emit(bb, z, z);
               return;
             }
             const int j = jj[e];
@@ -1174,11 +1190,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 #pragma unroll
             for (int t = 0; t < NR; ++t) buf[0][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[0]);
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-              if (bb < 3) {
+            for (int bb = 0; bb < NB; ++bb) {
+              if (bb < NB - 1) {
 #pragma unroll
                 for (int t = 0; t < NR; ++t)
-                  buf[(bb + 1) & 1][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[bb < 3 ? bb + 1 : bb]);
+                  buf[(bb + 1) & 1][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[bb < NB - 1 ? bb + 1 : bb]);
               }
               const uint4 *rb = buf[bb & 1];
               auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
@@ -1218,6 +1234,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             }
           };
           if (Cf::TMU && sp >= Cf::NSU) {
+            if constexpr (Cf::TMU) {
             // unit pair in TMEM as the M = 64 A operand: row e at lane
             // 32 (e / 16) + e % 16 (+16 in the upper half); lane half 0 holds
             // [v+ | v-], half 1 holds [v- | v+] (64 columns each, channel
@@ -1258,17 +1275,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             tmem_st_32x32b_x16u(ta + 80, st3);
             tmem_st_wait();
             tc_fence_before();
+            }
           } else {
             uint8_t *up = units + (size_t)sp * UNIT_BYTES;
             uint8_t *um = up + UNIT_BYTES;
-            // a warp covers 8 edges x 4 channel blocks: 64 contiguous bytes per
-            // gathered row, and 8 edges x 16 B per core-matrix row block in
-            // shared memory (no bank conflicts beyond the 4 wavefronts of 512 B)
-            // thread: one edge, channel blocks lane/8 + {0, 4, 8, 12}
-            const int e = pw * 8 + (lane & 7);
+            // a warp covers EPW = TE / 8 edges: 8 edges x 4 channel blocks
+            // (64-edge tiles) or 4 edges x 8 blocks (32-edge tiles); gathered
+            // rows are read in >= 64 contiguous bytes, and shared-memory stores
+            // fill whole 16-byte core-matrix rows.  Thread: one edge, NBT blocks
+            constexpr int EPW = TE / 8, NBT = EPW / 2;
+            const int e = pw * EPW + (lane % EPW);
             auto fill = [&](auto LPc) {
-              const int cb0 = (lane >> 3) * 8;
-              const int cbs[4] = {cb0, cb0 + 32, cb0 + 64, cb0 + 96};
+              const int cb0 = (lane / EPW) * 8;
+              int cbs[NBT];
+#pragma unroll
+              for (int k = 0; k < NBT; ++k) cbs[k] = cb0 + k * (128 / NBT);
               rot4(LPc, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
                 *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbs[bb], 128)) = wp;
                 if (m > 0) *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbs[bb], 128)) = wm;
@@ -1279,7 +1300,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               case 1: if constexpr (L >= 1) fill(std::integral_constant<int, (L >= 1 ? 1 : 0)>{}); break;
               case 2: if constexpr (L >= 2) fill(std::integral_constant<int, (L >= 2 ? 2 : 0)>{}); break;
               case 3: if constexpr (L >= 3) fill(std::integral_constant<int, (L >= 3 ? 3 : 0)>{}); break;
-              default: if constexpr (L >= 4) fill(std::integral_constant<int, (L >= 4 ? 4 : 0)>{}); break;
+              case 4: if constexpr (L >= 4) fill(std::integral_constant<int, (L >= 4 ? 4 : 0)>{}); break;
+              case 5: if constexpr (L >= 5) fill(std::integral_constant<int, (L >= 5 ? 5 : 0)>{}); break;
+              default: if constexpr (L >= 6) fill(std::integral_constant<int, (L >= 6 ? 6 : 0)>{}); break;
             }
           }
           fence_async_smem();
@@ -1332,7 +1355,7 @@ static e2f_status launch_stats(const TcArgs &args, cudaStream_t s) {
 
 e2f_status attention_tc_available(const e2f_weights *w) {
   if (w->dtype != E2F_BF16 || w->C != tca::CH) return E2F_ERR_UNSUPPORTED;
-  if (w->L_max < 1 || w->L_max > 4) return E2F_ERR_UNSUPPORTED;
+  if (w->L_max < 1 || w->L_max > 6) return E2F_ERR_UNSUPPORTED;
   // heads of 8..32 channels (the head reductions run inside one warp)
   if (w->H < 4 || w->H > tca::HMAX || tca::CH % w->H != 0) return E2F_ERR_UNSUPPORTED;
   return E2F_OK;
@@ -1398,19 +1421,24 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
     case 2: r = launch_stats<2>(a, s); break;
     case 3: r = launch_stats<3>(a, s); break;
     case 4: r = launch_stats<4>(a, s); break;
+    case 5: r = launch_stats<5>(a, s); break;
+    case 6: r = launch_stats<6>(a, s); break;
     default: return E2F_ERR_UNSUPPORTED;
   }
   if (r != E2F_OK) return r;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(nsm, (E + TE - 1) / TE));
+  const int te = L >= 5 ? Cfg<6>::TE : TE64;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(nsm, (E + te - 1) / te));
   if (ev0) E2F_CUDA_TRY(cudaEventRecord(ev0, s));
   switch (L) {
     case 1: r = launch_tc<1>(a, grid, s); break;
     case 2: r = launch_tc<2>(a, grid, s); break;
     case 3: r = launch_tc<3>(a, grid, s); break;
     case 4: r = launch_tc<4>(a, grid, s); break;
+    case 5: r = launch_tc<5>(a, grid, s); break;
+    case 6: r = launch_tc<6>(a, grid, s); break;
     default: return E2F_ERR_UNSUPPORTED;
   }
   if (ev1) E2F_CUDA_TRY(cudaEventRecord(ev1, s));

@@ -483,7 +483,7 @@ def run_rows(args):
                "roofline": {"bound": "tensor", "flops_per_edge": F, "achieved": F * E / (k_ms * 1e-3) / 1e12,
                             "peak": peak, "unit": "TFLOP/s", "frac": F * E / (k_ms * 1e-3) / 1e12 / peak,
                             "peak_source": f"bf16_tflops burst, {peak_src}",
-                            "path": "tcgen05" if (wl.precision == "bf16" and wl.C == 128 and 1 <= wl.L <= 4) else "SIMT"},
+                            "path": "tcgen05" if (wl.precision == "bf16" and wl.C == 128 and 1 <= wl.L <= 6) else "SIMT"},
                "peak_device_bytes": {"torch": int(torch.cuda.max_memory_allocated(dev)),
                                      "library_scratch": int(e2f.scratch_high_water())}}
         print(json.dumps(out), flush=True)
@@ -496,7 +496,7 @@ def run_rows(args):
         one(cfg)
     for n in (10002, 30000):   # memory sweep of the water box (cfg4 is the 100k point)
         one(4, n_target=n)
-    one(3, reps=1)   # L = 6 runs on the SIMT kernel: one timed call
+    one(3)
 
 
 def main(argv=None):

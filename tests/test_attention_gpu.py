@@ -79,10 +79,10 @@ def test_full_size_sampled_rows(cuda_ok, cfg, prec, n):
     _compare(wl, nodes=nodes)
 
 
-@pytest.mark.parametrize("L", [1, 2, 3, 4])
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 6])
 def test_tensor_core_path_small(cuda_ok, L):
     """bf16, C = 128, H = 8 takes the tcgen05 kernel: 24-atom cluster (7 edge
-    tiles, ragged last tile) for every supported degree."""
+    tiles of 64, or 14 of 32 for L >= 5; ragged last tile) for every degree."""
     wl0 = wlmod.make_workload(0)
     wl = wlmod.make_custom(wl0.pos, None, wl0.r_c, L=L, C=128, H=8, precision="bf16", seed=3 + L)
     _compare(wl)

@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       int hm = 0, hl = 0, hs = 0, ht = 0, npend = 0;
       auto poll_rg = [&]() -> bool {   // false: gave up (abort)
         if (npend == 0) return true;
-        if (!mbar_try_wait(&a2r_full[hs], (rgpar >> hs) & 1)) return true;
+        if (!mbar_test_wait(&a2r_full[hs], (rgpar >> hs) & 1)) return true;
         if (hm == 0 && hl == 0 && hs == 0 && ht > 0)   // first GEMM of a tile: Out columns cleared
           if (!W.wait(slots_clean, (ht - 1) & 1)) return false;
         tc_fence_after();
@@ -609,7 +609,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       };
       auto mw = [&](uint64_t *bar, uint32_t parity) -> bool {
         for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
-          if (mbar_try_wait(bar, parity)) return true;
+          if (mbar_test_wait(bar, parity)) return true;
           if (!poll_rg()) return false;
           if ((it & 255) == 255 && W.aborted()) return false;
         }
@@ -1156,47 +1156,79 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             dead = __shfl_sync(0xffffffffu, (int)(f || W.aborted()), 0) != 0;
             if (dead) break;
           }
-          // v~(+m), v~(-m) of edge e for four 8-channel blocks of degree l'
-          // (compile-time constant: register use follows the degree).  The
-          // gathered rows of block b + 1 are loaded while block b is computed;
-          // pairs of channels go through packed fp32 FMAs.  emit(b, wp, wm)
-          // receives block b as packed bf16 pairs (wp: +m, wm: -m).
-          auto rot4 = [&](auto LPc, int e, const auto &cbs, auto &&emit) {
+          // v~(+m), v~(-m) of degree l' (compile-time constant: register use
+          // follows the degree) for NB (edge, 8-channel block) items of this
+          // thread: block b belongs to edge ea (first half of the blocks, or
+          // all of them when NEc = 1) or eb (second half), and covers
+          // channels [cbs[b], +8).  Pairs of channels go through packed fp32
+          // FMAs.  emit(b, wp, wm) receives block b as packed bf16 pairs (wp:
+          // +m, wm: -m); edges past the tile's end come out zero.
+          auto rot4 = [&](auto LPc, auto NEc, const int ea, const int eb, const auto &cbs, auto &&emit) {
             constexpr int LP = decltype(LPc)::value;
             constexpr int NR = 2 * LP + 1;
-            constexpr int NB = (int)(sizeof(cbs) / sizeof(int));   // channel blocks of this thread
-            if (e >= ne) {
-              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            constexpr int NB = (int)(sizeof(cbs) / sizeof(int));   // blocks of this thread
+            constexpr int NE = decltype(NEc)::value;               // distinct edges: 1 or 2
+            constexpr int BPE = NB / NE;                           // blocks per edge
+            if constexpr (NE == 1) {
+              if (ea >= ne) {
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-              for (int bb = 0; bb < NB; ++bb) emit(bb, z, z);
-              return;
+                for (int bb = 0; bb < NB; ++bb) emit(bb, z, z);
+                return;
+              }
             }
-            const int j = jj[e];
-            const __half *d = dy + e * Cf::NDYP;
-            const __nv_bfloat16 *vr = a.v + (size_t)j * Q * CH + (size_t)(LP * LP) * CH;
+            // rows of edges past the tile's end: node 0's, scaled by zero
+            const __nv_bfloat16 *vra = a.v + (size_t)(ea < ne ? jj[ea] : 0) * Q * CH + (size_t)(LP * LP) * CH;
+            const __nv_bfloat16 *vrb = NE == 1 ? vra : a.v + (size_t)(eb < ne ? jj[eb] : 0) * Q * CH + (size_t)(LP * LP) * CH;
             // per-edge coefficients: u+ = c v+ + s v-, u- = -s v+ + c v-, scaled
             // by the y-rotation entries of row +m (even block) / -m (odd block)
-            const float c0 = __half2float(d[dye_off<L>(LP) + m * (LP + 1)]);
-            float app[LP > 0 ? LP : 1], apm[LP > 0 ? LP : 1], amp[LP > 0 ? LP : 1], amm[LP > 0 ? LP : 1];
+            float c0 = 0.f, app[LP > 0 ? LP : 1], apm[LP > 0 ? LP : 1], amp[LP > 0 ? LP : 1], amm[LP > 0 ? LP : 1];
+            {
+              const int e = ea;
+              const bool live = e < ne;
+              const __half *d = dy + (live ? e : 0) * Cf::NDYP;
+              c0 = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1)]) : 0.f;
 #pragma unroll
-            for (int kq = 1; kq <= LP; ++kq) {
-              const float ck = csb[(kq - 1) * TE + e], sk = snb[(kq - 1) * TE + e];
-              const float de = __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]);
-              const float dd = (m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
-              app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
-              amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
+              for (int kq = 1; kq <= LP; ++kq) {
+                const float ck = csb[(kq - 1) * TE + e], sk = snb[(kq - 1) * TE + e];
+                const float de = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]) : 0.f;
+                const float dd = (live && m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
+                app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
+                amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
+              }
             }
-            uint4 buf[2][NR];
+            // two blocks of gathered rows in flight: block b + 1 is loaded
+            // while block b is computed
+            constexpr int DEPTH = 2;
+            uint4 buf[DEPTH][NR];
 #pragma unroll
-            for (int t = 0; t < NR; ++t) buf[0][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[0]);
+            for (int bb = 0; bb < DEPTH - 1; ++bb)
+#pragma unroll
+              for (int t = 0; t < NR; ++t) buf[bb][t] = *reinterpret_cast<const uint4 *>((bb < BPE ? vra : vrb) + (size_t)t * CH + cbs[bb]);
 #pragma unroll
             for (int bb = 0; bb < NB; ++bb) {
-              if (bb < NB - 1) {
+              if (bb > 0 && bb % BPE == 0)   // next edge
+              {
+                const int e = eb;
+                const bool live = e < ne;
+                const __half *d = dy + (live ? e : 0) * Cf::NDYP;
+                c0 = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1)]) : 0.f;
+#pragma unroll
+                for (int kq = 1; kq <= LP; ++kq) {
+                  const float ck = csb[(kq - 1) * TE + e], sk = snb[(kq - 1) * TE + e];
+                  const float de = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]) : 0.f;
+                  const float dd = (live && m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
+                  app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
+                  amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
+                }
+              }
+              if (bb + DEPTH - 1 < NB) {
+                const int nb = bb + DEPTH - 1 < NB ? bb + DEPTH - 1 : 0;
 #pragma unroll
                 for (int t = 0; t < NR; ++t)
-                  buf[(bb + 1) & 1][t] = *reinterpret_cast<const uint4 *>(vr + (size_t)t * CH + cbs[bb < NB - 1 ? bb + 1 : bb]);
+                  buf[(bb + DEPTH - 1) % DEPTH][t] = *reinterpret_cast<const uint4 *>((nb < BPE ? vra : vrb) + (size_t)t * CH + cbs[nb]);
               }
-              const uint4 *rb = buf[bb & 1];
+              const uint4 *rb = buf[bb % DEPTH];
               auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
               float2 ap[4], am[4];
               {
@@ -1248,7 +1280,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             {
               const int cb0 = chb + 32 * half;
               const int cbs[4] = {cb0, cb0 + 8, cb0 + 16, cb0 + 24};
-              rot4(std::integral_constant<int, L>{}, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
+              rot4(std::integral_constant<int, L>{}, std::integral_constant<int, 1>{}, e, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
                 const uint32_t *pp = reinterpret_cast<const uint32_t *>(&wp), *pm = reinterpret_cast<const uint32_t *>(&wm);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) { wpl[4 * bb + i] = pp[i]; wmi[4 * bb + i] = pm[i]; }
@@ -1279,18 +1311,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           } else {
             uint8_t *up = units + (size_t)sp * UNIT_BYTES;
             uint8_t *um = up + UNIT_BYTES;
-            // a warp covers EPW = TE / 8 edges: 8 edges x 4 channel blocks
-            // (64-edge tiles) or 4 edges x 8 blocks (32-edge tiles); gathered
-            // rows are read in >= 64 contiguous bytes, and shared-memory stores
-            // fill whole 16-byte core-matrix rows.  Thread: one edge, NBT blocks
-            constexpr int EPW = TE / 8, NBT = EPW / 2;
-            const int e = pw * EPW + (lane % EPW);
+            // a warp covers EPW = TE / 8 edges, in groups of four: a gathered
+            // row is read as four edges x 128 contiguous bytes, and the stores
+            // fill whole 128-byte rows of the K-major unit.  Thread: edge
+            // 4 g + (lane & 3) of group g, channels [8 (lane >> 2), +8) and
+            // the same + 64.
+            constexpr int NG = TE / 32;
+            const int cb0 = (lane >> 2) * 8;
+            const int ea = pw * (TE / 8) + (lane & 3), eb = ea + 4;
             auto fill = [&](auto LPc) {
-              const int cb0 = (lane / EPW) * 8;
-              int cbs[NBT];
+              int cbs[2 * NG];
 #pragma unroll
-              for (int k = 0; k < NBT; ++k) cbs[k] = cb0 + k * (128 / NBT);
-              rot4(LPc, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
+              for (int k = 0; k < 2 * NG; ++k) cbs[k] = cb0 + 64 * (k & 1);
+              rot4(LPc, std::integral_constant<int, NG>{}, ea, eb, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
+                const int e = bb < 2 ? ea : eb;
                 *reinterpret_cast<uint4 *>(up + kmajor_off(e, cbs[bb], 128)) = wp;
                 if (m > 0) *reinterpret_cast<uint4 *>(um + kmajor_off(e, cbs[bb], 128)) = wm;
               });

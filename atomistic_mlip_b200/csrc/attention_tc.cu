@@ -112,7 +112,7 @@ template <int L> struct Cfg {
   static constexpr size_t OFF_GEO = OFF_G2 + 2 * GEO_BYTES;          // float [TE][4]: ct, st, u, pad
   static constexpr size_t OFF_TILE = OFF_GEO + (size_t)TE * 4 * 4;   // 8 ints
   static constexpr size_t OFF_BAR = (OFF_TILE + 32 + 7) & ~(size_t)7;
-  static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 7;
+  static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 8;
   static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(TM_OUT + OUT_COLS <= (TMU ? TM_UNIT : 512u), "TMEM budget");
@@ -501,7 +501,7 @@ template <int L>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   using Cf = Cfg<L>;
   constexpr int Q = Cf::Q, P = Cf::P, NUNIT = Cf::NUNIT;
-  constexpr int TE = Cf::TE, UNIT_BYTES = Cf::UNIT_BYTES, A2_BYTES = Cf::A2_BYTES;
+  constexpr int TE = Cf::TE, UNIT_BYTES = Cf::UNIT_BYTES;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -519,6 +519,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   uint64_t *geo_full = slots_clean + 1;    // [2], per geometry copy
   uint64_t *geo_empty = geo_full + 2;     // [2]
   uint64_t *mma_drain = geo_empty + 2;
+  uint64_t *rg_drain = mma_drain + 1;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + Cf::NBAR);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -544,7 +545,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     }
     mbar_init(tile_done, 1); mbar_init(slots_clean, 4);
     for (int c = 0; c < 2; ++c) { mbar_init(&geo_full[c], 1); mbar_init(&geo_empty[c], 4); }
-    mbar_init(mma_drain, 1);
+    mbar_init(mma_drain, 1); mbar_init(rg_drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -570,47 +571,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       constexpr uint32_t ID_NEGB = ID_MAIN | (1u << 14);
       uint32_t st = 0, pc = 0;
       uint32_t fillpar = 0;        // bit sp: parity of unit sp's fill count
-      uint32_t rgpar = 0;          // bit sg: parity of the R-GEMMs issued for sign sg
-      const uint32_t s_units = smem_addr(units), s_w = smem_addr(wst), s_a2 = smem_addr(A2), s_r = smem_addr(Rb);
+      const uint32_t s_units = smem_addr(units), s_w = smem_addr(wst);
       const uint64_t ud0 = smem_desc(s_units, 128, 128 * 16);   // unit 0, K-major, Kc = 128
       const uint64_t wd128 = smem_desc(s_w, 128, 128 * 16);     // stage 0 as 128 x 128 (m = 0)
       const uint64_t wd64 = smem_desc(s_w, 128, 64 * 16);       // stage 0 as 2 x 128 x 64 (m >= 1)
-      const uint64_t a2d = smem_desc(s_a2, 128, TE * 16);       // A2, MN-major, K = TE edges
-      const uint64_t rd = smem_desc(s_r, 128, TE * 16);         // R, K-major, K = TE edges
-      int t = 0;
       bool ok = ti.start();
-      // Back-rotation GEMMs are issued as soon as the epilogue hands A2 / R
-      // over, polled between weight stages and inside every wait of this
-      // thread (the epilogue's second sign waits for the first one's GEMM).
-      // Queue head: pass (hm, hl) of tile ht, next sign hs; npend passes whose
-      // y has been committed and whose GEMMs are not all issued.
-      int hm = 0, hl = 0, hs = 0, ht = 0, npend = 0;
-      auto poll_rg = [&]() -> bool {   // false: gave up (abort)
-        if (npend == 0) return true;
-        if (!mbar_test_wait(&a2r_full[hs], (rgpar >> hs) & 1)) return true;
-        if (hm == 0 && hl == 0 && hs == 0 && ht > 0)   // first GEMM of a tile: Out columns cleared
-          if (!W.wait(slots_clean, (ht - 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t id = idesc_bf16(128, Cf::NL(hl), 1, 0);
-        const uint32_t d = tbase + TM_OUT + Cf::OB(hl);
-        const uint64_t bd = rd + (uint64_t)hs * ((Cf::NLMAX * TE * 2) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < TE / 16; ++kk) mma_bf16_ss(d, a2d + 16 * kk, bd + 16 * kk, id, 1u);
-        mma_commit(&rg_done[hs]);
-        rgpar ^= 1u << hs;
-        if (++hs == (hm == 0 ? 1 : 2)) {
-          hs = 0;
-          --npend;
-          if (hl < L) ++hl;
-          else if (hm < L) { ++hm; hl = hm; }
-          else { hm = 0; hl = 0; ++ht; }
-        }
-        return true;
-      };
       auto mw = [&](uint64_t *bar, uint32_t parity) -> bool {
         for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
           if (mbar_test_wait(bar, parity)) return true;
-          if (!poll_rg()) return false;
           if ((it & 255) == 255 && W.aborted()) return false;
         }
         *abort_flag = 1;
@@ -644,7 +612,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               for (int kh = 0; kh < nk; ++kh) {
                 const uint32_t s = st % NSTAGE;
                 if (!mw(&w_full[s], (st / NSTAGE) & 1)) { bad = true; break; }
-                tc_fence_after();
                 const uint32_t acc0 = (lp > m || kh > 0) ? 1u : 0u;
                 if (m == 0) {
                   // the whole 128 x 128 block: 8 steps of 16
@@ -680,7 +647,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 }
                 mma_commit(&w_empty[s]);
                 ++st;
-                if (!poll_rg()) { bad = true; break; }
               }
               if (bad) break;
               if (last_pass) {
@@ -692,21 +658,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             if (bad) break;
             mma_commit(&y_full[b]);
             ++pc;
-            ++npend;
           }
         }
         if (bad || W.aborted()) break;
-        // the tile's last back-rotation GEMMs, then hand the tile over
-        for (uint32_t it = 0; npend > 0 && it < WAIT_LIMIT; ++it) {
-          if (!poll_rg()) { bad = true; break; }
-          if ((it & 255) == 255 && W.aborted()) { bad = true; break; }
-        }
-        if (bad || npend > 0) {
-          if (npend > 0 && !bad) { *abort_flag = 1; atomicExch(a.err, E2F_ERR_TIMEOUT); }
-          break;
-        }
-        mma_commit(tile_done);
-        ++t;
         ok = ti.next();
       }
       // every MMA this thread issued has completed before TMEM is released
@@ -725,7 +679,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         for (int i = 0; i < SPT; ++i, ++st) {
           if ((int)(st % 2) != me) continue;
           const uint32_t s = st % NSTAGE;
-          if (!W.wait(&w_empty[s], ((st / NSTAGE) & 1) ^ 1, 20)) break;
+          if (!W.wait(&w_empty[s], ((st / NSTAGE) & 1) ^ 1)) break;
           mbar_arrive_expect_tx(&w_full[s], STAGE_BYTES);
           bulk_g2s(wst + s * STAGE_BYTES, a.wpack + (size_t)i * STAGE_BYTES, STAGE_BYTES, &w_full[s]);
         }
@@ -742,6 +696,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             if (mbar_try_wait(&w_full[s], (s_last / NSTAGE) & 1)) break;
         }
       }
+    }
+  } else if (warp == 3) {
+    // ======================= back-rotation GEMM issuer =======================
+    // Out[c][slot m'] += sum_e A2[c][e] R[slot m'][e] for each pass and sign,
+    // issued as soon as the epilogue hands A2 / R over (a2r_full), so that
+    // the SO(2) MMA thread never stops to poll for them.
+    if (lane == 0) {
+      const uint64_t a2d = smem_desc(smem_addr(A2), 128, TE * 16);   // A2, MN-major, K = TE edges
+      const uint64_t rd = smem_desc(smem_addr(Rb), 128, TE * 16);    // R, K-major, K = TE edges
+      uint32_t rgpar = 0;   // bit sg: parity of the GEMMs issued for sign sg
+      int t = 0;
+      bool ok = ti.start();
+      while (ok && !W.aborted()) {
+        bool bad = false;
+        #pragma unroll 1
+        for (int m = 0; m <= L && !bad; ++m) {
+          #pragma unroll 1
+          for (int l = m; l <= L && !bad; ++l) {
+            const int ng = (m == 0) ? 1 : 2;
+            for (int hs = 0; hs < ng; ++hs) {
+              if (!W.wait(&a2r_full[hs], (rgpar >> hs) & 1)) { bad = true; break; }
+              if (m == 0 && l == 0 && hs == 0 && t > 0)   // first GEMM of a tile: Out columns cleared
+                if (!W.wait(slots_clean, (t - 1) & 1)) { bad = true; break; }
+              tc_fence_after();
+              const uint32_t id = idesc_bf16(128, Cf::NL(l), 1, 0);
+              const uint32_t d = tbase + TM_OUT + Cf::OB(l);
+              const uint64_t bd = rd + (uint64_t)hs * ((Cf::NLMAX * TE * 2) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < TE / 16; ++kk) mma_bf16_ss(d, a2d + 16 * kk, bd + 16 * kk, id, 1u);
+              mma_commit(&rg_done[hs]);
+              rgpar ^= 1u << hs;
+            }
+          }
+        }
+        if (bad || W.aborted()) break;
+        mma_commit(tile_done);   // the tile's Out sums are complete once these GEMMs are
+        ++t;
+        ok = ti.next();
+      }
+      // every GEMM this thread issued has completed before TMEM is released
+      mma_commit(rg_drain);
+      for (uint32_t it = 0; it < WAIT_LIMIT; ++it)
+        if (mbar_try_wait(rg_drain, 0)) break;
     }
   } else if (warp >= 4 && warp < 8) {
     // ======================= epilogue =======================
@@ -1364,7 +1361,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       ok = has_next;
     }
   }
-  // warp 3 idles
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tbase, 512);

@@ -65,94 +65,141 @@ project_simt_kernel(const T *__restrict__ x, int N, int L, int C, ProjArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core path (bf16, C = 128): one CTA per (128-row tile of one degree,
-// which of q / k / v).  Rows (node, m) of degree l are gathered from x into a
-// K-major core-matrix tile in shared memory; W[l] (out x in, already K-major)
-// is the B operand; one tcgen05.mma chain M = 128, N = 128, K = 128 into a
-// 128-column TMEM accumulator; the epilogue rounds to bf16 and scatters the
-// rows back to [N][Q][C].
+// Tensor-core path (bf16, C = 128): persistent CTAs (one per SM, 256
+// threads).  A tile is 128 rows (node, m) of one degree l, gathered from x
+// into a K-major core-matrix tile in shared memory.  q, k and v of the tile
+// come from three tcgen05.mma chains (M = 128, N = 128, K = 128) into three
+// 128-column TMEM accumulators, against Wq[l], Wk[l], Wv[l] (out x in, the
+// B operands), which stay in shared memory while the CTA's tiles are of
+// degree l.  x is read once for all three outputs, and the next tile's rows
+// are loaded into registers while the current tile's MMAs and epilogue run.
+// The epilogue rounds to bf16 and scatters the rows back to [N][Q][C].
 // ---------------------------------------------------------------------------
 namespace ptc {
-constexpr int CH = 128, TR = 128;
-constexpr size_t SMEM = 2 * (size_t)TR * CH * 2 + 16;
+constexpr int CH = 128, TR = 128, NT = 256;
+constexpr size_t TILE_BYTES = (size_t)TR * CH * 2;   // one 128 x 128 bf16 tile
+constexpr size_t SMEM = 4 * TILE_BYTES + 64;         // Wq, Wk, Wv, rows of x; barrier
 
-__global__ void __launch_bounds__(128) project_tc_kernel(const __nv_bfloat16 *__restrict__ x, int N, int L,
-                                                          ProjArgs a, int *err) {
+__global__ void __launch_bounds__(NT, 1) project_tc_kernel(const __nv_bfloat16 *__restrict__ x, int N, int L,
+                                                             ProjArgs a, long long ntiles, int *err) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *sA = smem, *sB = smem + TR * CH * 2;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + 2 * TR * CH * 2);
+  uint8_t *sW = smem, *sA = smem + 3 * TILE_BYTES;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + 4 * TILE_BYTES);
   __shared__ uint32_t tslot;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int Q = (L + 1) * (L + 1);
-  // decode (degree, tile) from the flat tile index
-  int l = 0;
-  long long tile = blockIdx.x;
-  for (;; ++l) {
-    const long long nt = ((long long)N * (2 * l + 1) + TR - 1) / TR;
-    if (tile < nt || l == L) break;
-    tile -= nt;
-  }
-  const int w = 2 * l + 1;
-  const long long rows = (long long)N * w;
-  const int which = blockIdx.y;
-  const __nv_bfloat16 *W = static_cast<const __nv_bfloat16 *>(a.W[which][l]);
-  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out[which]);
-  // gather: thread t owns row t of A and row t of B
-  const long long r = tile * TR + t;
-  const bool valid = r < rows;
-  long long off = 0;
-  if (valid) {
-    const long long node = r / w;
-    off = (node * Q + l * l + (r - node * w)) * CH;
-  }
-#pragma unroll
-  for (int c = 0; c < CH / 8; ++c) {
-    uint4 va = make_uint4(0, 0, 0, 0);
-    if (valid) va = *reinterpret_cast<const uint4 *>(x + off + 8 * c);
-    *reinterpret_cast<uint4 *>(sA + kmajor_off(t, 8 * c, CH)) = va;
-    *reinterpret_cast<uint4 *>(sB + kmajor_off(t, 8 * c, CH)) =
-        *reinterpret_cast<const uint4 *>(W + (size_t)t * CH + 8 * c);
-  }
+  const int row = t & (TR - 1), half = t >> 7;   // staging: tile row, 64-channel half
   if (t == 0) { mbar_init(bar, 1); mbar_fence_init(); }
-  fence_async_smem();
   __syncthreads();
-  if (warp == 0) { tmem_alloc(&tslot, 128); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(&tslot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  if (t == 0) {
-    constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
-    const uint32_t a0 = smem_addr(sA), b0 = smem_addr(sB);
+
+  // flat tile index -> degree l and first row r0 of the tile
+  auto decode = [&](long long g, int &l, long long &r0) {
+    l = 0;
+    for (;; ++l) {
+      const long long nt = ((long long)N * (2 * l + 1) + TR - 1) / TR;
+      if (g < nt || l == L) break;
+      g -= nt;
+    }
+    r0 = g * TR;
+  };
+  // element offset of row r (node, m) of degree l in x / q / k / v, or -1
+  auto row_off = [&](int l, long long r) -> long long {
+    const int w = 2 * l + 1;
+    if (r >= (long long)N * w) return -1;
+    const long long node = r / w;
+    return (node * Q + l * l + (r - node * w)) * CH;
+  };
+  uint4 pre[8];   // this thread's 64 channels of the next tile's row
+  auto fetch = [&](long long g) {
+    int l;
+    long long r0;
+    decode(g, l, r0);
+    const long long off = row_off(l, r0 + row);
 #pragma unroll
-    for (int kk = 0; kk < CH / 16; ++kk)
-      mma_bf16_ss(tb, smem_desc(a0 + kmajor_off(0, 16 * kk, CH), 128, CH * 16),
-                  smem_desc(b0 + kmajor_off(0, 16 * kk, CH), 128, CH * 16), id, kk > 0);
-    mma_commit(bar);
-  }
-  __syncwarp();
-  const bool ok = mbar_wait(bar, 0, 1u << 26);
-  if (!ok && lane == 0) atomicExch(err, E2F_ERR_TIMEOUT);
-  tc_fence_after();
-  if (ok) {
+    for (int c = 0; c < 8; ++c)
+      pre[c] = off >= 0 ? *reinterpret_cast<const uint4 *>(x + off + 64 * half + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+  };
+
+  int cur_l = -1;
+  uint32_t phase = 0;
+  bool dead = false;
+  if ((long long)blockIdx.x < ntiles) fetch(blockIdx.x);
+  for (long long g = blockIdx.x; g < ntiles && !dead; g += gridDim.x) {
+    int l;
+    long long r0;
+    decode(g, l, r0);
+    // the previous tile's MMAs have completed and its accumulators been read
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(sA + kmajor_off(row, 64 * half + 8 * c, CH)) = pre[c];
+    if (l != cur_l) {   // this degree's weights
+      for (int which = 0; which < 3; ++which) {
+        const __nv_bfloat16 *W = static_cast<const __nv_bfloat16 *>(a.W[which][l]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4 *>(sW + which * TILE_BYTES + kmajor_off(row, 64 * half + 8 * c, CH)) =
+              *reinterpret_cast<const uint4 *>(W + (size_t)row * CH + 64 * half + 8 * c);
+      }
+      cur_l = l;
+    }
+    fence_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
+      const uint32_t a0 = smem_addr(sA), w0 = smem_addr(sW);
+#pragma unroll
+      for (int which = 0; which < 3; ++which)
+#pragma unroll
+        for (int kk = 0; kk < CH / 16; ++kk)
+          mma_bf16_ss(tb + 128 * which, smem_desc(a0 + kmajor_off(0, 16 * kk, CH), 128, CH * 16),
+                      smem_desc(w0 + which * TILE_BYTES + kmajor_off(0, 16 * kk, CH), 128, CH * 16), id, kk > 0);
+      mma_commit(bar);
+    }
+    // the next tile's rows, loaded while the MMAs and the epilogue run
+    if (g + gridDim.x < ntiles) fetch(g + gridDim.x);
+    const bool ok = mbar_wait(bar, phase, 1u << 26);
+    phase ^= 1u;
+    dead = __syncthreads_or(!ok) != 0;
+    if (dead) {
+      if (t == 0) atomicExch(err, E2F_ERR_TIMEOUT);
+      break;
+    }
+    tc_fence_after();
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) + [0, 32) (tile rows),
+    // channels [64 (w / 4), +64) of each output
+    {
+      const int erow = 32 * (warp & 3) + lane, ecol = 64 * (warp >> 2);
+      const long long off = row_off(l, r0 + erow);
 #pragma unroll 1
-    for (int c0 = 0; c0 < CH; c0 += 16) {
-      float v[16];
-      tmem_ld_32x32b_x16(tb + ((uint32_t)(32 * warp) << 16) + c0, v);
-      tmem_ld_wait();
-      if (valid) {
-        __align__(16) __nv_bfloat16 o[16];
+      for (int which = 0; which < 3; ++which) {
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out[which]);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          float v[16];
+          tmem_ld_32x32b_x16(tb + ((uint32_t)(32 * (warp & 3)) << 16) + 128 * which + ecol + c0, v);
+          tmem_ld_wait();
+          if (off >= 0) {
+            __align__(16) __nv_bfloat16 o[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) o[i] = __float2bfloat16_rn(v[i]);
-        *reinterpret_cast<uint4 *>(out + off + c0) = *reinterpret_cast<const uint4 *>(&o[0]);
-        *reinterpret_cast<uint4 *>(out + off + c0 + 8) = *reinterpret_cast<const uint4 *>(&o[8]);
+            for (int i = 0; i < 16; ++i) o[i] = __float2bfloat16_rn(v[i]);
+            *reinterpret_cast<uint4 *>(out + off + ecol + c0) = *reinterpret_cast<const uint4 *>(&o[0]);
+            *reinterpret_cast<uint4 *>(out + off + ecol + c0 + 8) = *reinterpret_cast<const uint4 *>(&o[8]);
+          }
+        }
       }
     }
+    tc_fence_before();
+    __syncthreads();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, 128);
+  if (warp == 0) tmem_dealloc(tb, 512);
 }
 }  // namespace ptc
 
@@ -179,10 +226,14 @@ e2f_status project_impl(const void *x, int64_t N, const e2f_weights *w, void *q,
     for (int l = 0; l <= L; ++l) tiles += (N * (2LL * l + 1) + ptc::TR - 1) / ptc::TR;
     int *err = device_error_flag();
     if (!err) return E2F_ERR_CUDA;
+    int dev = 0, nsm = 148;
+    E2F_CUDA_TRY(cudaGetDevice(&dev));
+    E2F_CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    const int grid = (int)std::min<long long>(tiles, nsm);
     E2F_CUDA_TRY(cudaFuncSetAttribute(ptc::project_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)ptc::SMEM));
-    E2F_LAUNCH(ptc::project_tc_kernel, dim3((unsigned)tiles, 3), 128, ptc::SMEM, s, (const __nv_bfloat16 *)x,
-               (int)N, L, a, err);
+    E2F_LAUNCH(ptc::project_tc_kernel, grid, ptc::NT, ptc::SMEM, s, (const __nv_bfloat16 *)x, (int)N, L, a,
+               tiles, err);
   } else {
     E2F_CUDA_TRY(cudaFuncSetAttribute(project_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     E2F_LAUNCH(project_simt_kernel<__nv_bfloat16>, grid, PROJ_THREADS, smem, s, (const __nv_bfloat16 *)x, (int)N, L, C, a);

@@ -5,7 +5,8 @@
 // materialisation; "EquiformerV3 ...", §2B.3 envelope in the softmax).
 //
 // Structure (one persistent CTA per SM, 512 threads, contiguous edge range
-// per CTA, tiles of <= 64 edges covering <= 4 destination nodes):
+// per CTA, tiles of <= 64 edges (32 for L = 5, 6) covering <= 4 destination
+// nodes):
 //
 //   producers (warps 8-15)  per tile: edge geometry, Wigner blocks of the
 //                           y-rotation in the two-angle frame (parity blocks),
@@ -22,8 +23,10 @@
 //                           K streamed over the block's units), complex form:
 //                           y+ += v+ Wr^T - v- Wi^T,  y- += v- Wr^T + v+ Wi^T,
 //                           y+ / y- accumulate in the two lane halves of a TMEM
-//                           buffer; then the back-rotation + per-node sum as a
-//                           second GEMM per (l, +-m) group:
+//                           buffer.
+//   back-rotation (warp 3)  the back-rotation + per-node sum as a second GEMM
+//                           per (l, +-m) group, issued as soon as the epilogue
+//                           hands it over:
 //                           Out_l[c, (slot, m')] += sum_e A[c, e] R[(slot,m'), e]
 //                           with A = alpha g y (bf16) and R = D^l[+-m][m'].
 //   epilogue (warps 4-7)    TMEM y -> A (scaled bf16, shared memory), builds R,

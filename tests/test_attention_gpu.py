@@ -88,6 +88,15 @@ def test_tensor_core_path_small(cuda_ok, L):
     _compare(wl)
 
 
+@pytest.mark.parametrize("H", [4, 16])
+def test_tensor_core_path_head_counts(cuda_ok, H):
+    """The smallest and largest head counts the tcgen05 kernel takes (32 and
+    8 channels per head: head sums over four blocks, or one)."""
+    wl0 = wlmod.make_workload(0)
+    wl = wlmod.make_custom(wl0.pos, None, wl0.r_c, L=4, C=128, H=H, precision="bf16", seed=20 + H)
+    _compare(wl)
+
+
 def test_tensor_core_path_isolated_and_low_degree(cuda_ok):
     """Isolated atoms (empty rows), degree-1 rows and a dense clump in one
     batch: tiles bounded by the node-slot limit, nodes spanning tiles."""

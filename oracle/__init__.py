@@ -15,6 +15,11 @@ sh          real spherical harmonics and Wigner-D matrices, built two
 neighbors   brute-force all-pairs radius graph with the exact fp32 predicate
             (NumPy, plus a plain-C all-pairs loop for large N)
 attention   the operator itself, edge by edge in fp64
+attention_grad
+            the same operator restated in PyTorch CPU ops (fp64), whose
+            autograd gives the gradients of a scalar of the outputs with
+            respect to positions, features and weights (the backward that
+            the GPU path does not have yet)
 
 Sources (web pages on E2Former-V2, EquiformerV3 and DPA4):
   * "E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation

@@ -124,10 +124,13 @@ def _so2_mix(vt: torch.Tensor, g: torch.Tensor, L: int, C: int, W0, Wr, Wi) -> t
 
 
 def forward_t(pos: torch.Tensor, box: Optional[np.ndarray], r_c: float, row_ptr: np.ndarray,
-              col: np.ndarray, x: torch.Tensor, P: Dict[str, object], L: int, C: int, H: int) -> torch.Tensor:
+              col: np.ndarray, x: torch.Tensor, P: Dict[str, object], L: int, C: int, H: int,
+              parts: Optional[dict] = None) -> torch.Tensor:
     """o [N, Q, C] of every node (steps O2-O13 of ``oracle.attention``), in torch.
     P holds the weights as fp64 tensors: Wq, Wk, Wv (lists by l), W0, Wr, Wi
-    (lists by m, index 0 unused), rad_W1, rad_W2."""
+    (lists by m, index 0 unused), rad_W1, rad_W2.  If `parts` is a dict it
+    receives the per-edge logits "s" [E, H] (with their gradient retained),
+    weights "alpha" [E, H] and global-frame messages "z" [E, Q, C]."""
     N = pos.shape[0]
     Q = (L + 1) ** 2
     Ch = C // H
@@ -174,6 +177,9 @@ def forward_t(pos: torch.Tensor, box: Optional[np.ndarray], r_c: float, row_ptr:
     z = _rotate(D, _so2_mix(vt, g, L, C, P["W0"], P["Wr"], P["Wi"]), L, transpose=True)
     # O11, O12: two-pass softmax per destination and head
     u = 0.5 * (torch.cos(math.pi * r / r_c) + 1.0)
+    if parts is not None:
+        s.retain_grad()
+        parts["s"], parts["z"], parts["alpha"] = s, z, []
     rows = []
     for i in range(N):
         a0, a1 = int(row_ptr[i]), int(row_ptr[i + 1])
@@ -183,6 +189,8 @@ def forward_t(pos: torch.Tensor, box: Optional[np.ndarray], r_c: float, row_ptr:
         st = s[a0:a1]
         w = u[a0:a1, None] * torch.exp(st - st.max(dim=0, keepdim=True).values)
         alpha = w / w.sum(dim=0, keepdim=True)
+        if parts is not None:
+            parts["alpha"].append(alpha)
         a_c = alpha.repeat_interleave(Ch, dim=1)               # [k, C]
         rows.append(torch.einsum("kc,kqc->qc", a_c, z[a0:a1]))
     return torch.stack(rows, dim=0)
@@ -217,3 +225,28 @@ def gradients(wl, csr, G: np.ndarray, pos: Optional[np.ndarray] = None, x: Optio
     for key in ("Wq", "Wk", "Wv", "Wr", "Wi"):
         out[key] = [gnp(v) for v in P[key]]
     return out
+
+
+def logit_gradient(wl, csr, G: np.ndarray):
+    """d sum(G o) / d s [E, H] two ways: autograd, and the recompute form a
+    backward kernel uses, alpha (<G_i, z_e>_h - Delta_ih) with
+    Delta_ih = <G_i, o_i>_h (sums over the channels of head h)."""
+    row_ptr, col = csr
+    parts: dict = {}
+    P = params_t(wl, requires_grad=True)
+    o = forward_t(torch.tensor(np.asarray(wl.pos, np.float64), dtype=DT), wl.box, wl.r_c, row_ptr, col,
+                  torch.tensor(np.asarray(wl.x, np.float64), dtype=DT), P, wl.L, wl.C, wl.H, parts=parts)
+    Gt = torch.as_tensor(np.asarray(G, np.float64))
+    (o * Gt).sum().backward()
+    auto = parts["s"].grad.numpy().copy()
+    Ch = wl.C // wl.H
+    alpha = torch.cat(parts["alpha"], dim=0).detach().numpy()
+    z = parts["z"].detach().numpy()
+    on = o.detach().numpy()
+    rp = np.asarray(row_ptr, np.int64)
+    dst = np.repeat(np.arange(wl.N), np.diff(rp))
+    Gn = np.asarray(G, np.float64)
+    gz = np.einsum("eqc,eqc->ec", Gn[dst], z).reshape(-1, wl.H, Ch).sum(axis=2)      # [E, H]
+    delta = np.einsum("iqc,iqc->ic", Gn, on).reshape(-1, wl.H, Ch).sum(axis=2)       # [N, H]
+    formula = alpha * (gz - delta[dst])
+    return auto, formula

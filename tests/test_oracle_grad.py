@@ -117,3 +117,13 @@ def test_forces_rotate_with_the_system():
         x_r[:, s_, :] = sh.wigner_d_fit(l, Rq) @ wl.x[:, s_, :].astype(np.float64)
     g1 = ag.gradients(wl, csr, G, pos=pos_r, x=x_r)["pos"]
     assert np.max(np.abs(g1 - g0 @ Rq.T)) <= 1e-10 * np.max(np.abs(g0))
+
+
+def test_logit_gradient_recompute_form():
+    """The softmax backward a tiled kernel uses (per head: alpha times the
+    message-gradient product minus the node's Delta) equals autograd."""
+    for periodic in (False, True):
+        wl, csr = _system(periodic, 2, seed=41)
+        G = np.random.default_rng(42).standard_normal((wl.N, (wl.L + 1) ** 2, wl.C))
+        auto, formula = ag.logit_gradient(wl, csr, G)
+        assert np.max(np.abs(auto - formula)) <= 1e-12 * np.max(np.abs(auto))

@@ -88,51 +88,6 @@ template <typename T> E2F_HD T wig_entry(int l, int m, int mp, const T *D1, cons
   return acc;
 }
 
-// Strided variants: element k of D^1 / D^(l-1) sits at D1[k * st] / Dp[k * st]
-// (entry-major storage of many rotations, one rotation per lane).
-E2F_HD float wig_P_s(int i, int a, int b, int l, const float *D1, const float *Dp, int st) {
-  const int w = 2 * l - 1;
-  const int ra = a + (l - 1);
-  const float ri1 = D1[((i + 1) * 3 + 2) * st];
-  const float rim = D1[((i + 1) * 3 + 0) * st];
-  const float ri0 = D1[((i + 1) * 3 + 1) * st];
-  if (b == l) return ri1 * Dp[(ra * w + (2 * l - 2)) * st] - rim * Dp[(ra * w + 0) * st];
-  if (b == -l) return ri1 * Dp[(ra * w + 0) * st] + rim * Dp[(ra * w + (2 * l - 2)) * st];
-  return ri0 * Dp[(ra * w + (b + l - 1)) * st];
-}
-
-E2F_HD float wig_entry_s(int l, int m, int mp, const float *D1, const float *Dp, int st) {
-  const int am = m < 0 ? -m : m;
-  const float den = (mp == l || mp == -l) ? (float)(2 * l * (2 * l - 1)) : (float)((l + mp) * (l - mp));
-  float acc = 0.f;
-  const float uu = (float)((l + m) * (l - m));
-  if (uu > 0.f) acc += sqrtf(uu / den) * wig_P_s(0, m, mp, l, D1, Dp, st);
-  {
-    const float kd = (m == 0) ? 2.f : 1.f;
-    float v = 0.5f * sqrtf(kd * (float)((l + am - 1) * (l + am)) / den);
-    if (m == 0) v = -v;
-    float V;
-    if (m == 0) {
-      V = wig_P_s(1, 1, mp, l, D1, Dp, st) + wig_P_s(-1, -1, mp, l, D1, Dp, st);
-    } else if (m > 0) {
-      V = wig_P_s(1, m - 1, mp, l, D1, Dp, st) * (m == 1 ? 1.41421356237309515f : 1.f);
-      if (m != 1) V -= wig_P_s(-1, -m + 1, mp, l, D1, Dp, st);
-    } else {
-      V = wig_P_s(-1, -m - 1, mp, l, D1, Dp, st) * (m == -1 ? 1.41421356237309515f : 1.f);
-      if (m != -1) V += wig_P_s(1, m + 1, mp, l, D1, Dp, st);
-    }
-    acc += v * V;
-  }
-  if (m != 0 && am + 1 <= l - 1) {
-    const float w = -0.5f * sqrtf((float)((l - am - 1) * (l - am)) / den);
-    float W;
-    if (m > 0) W = wig_P_s(1, m + 1, mp, l, D1, Dp, st) + wig_P_s(-1, -m - 1, mp, l, D1, Dp, st);
-    else       W = wig_P_s(1, m - 1, mp, l, D1, Dp, st) - wig_P_s(-1, -m + 1, mp, l, D1, Dp, st);
-    acc += w * W;
-  }
-  return acc;
-}
-
 // All blocks l = 0..L of one rotation, sequentially (one thread).
 template <typename T> E2F_HD void wig_all_serial(const T R[9], int L, T *D) {
   D[0] = 1;

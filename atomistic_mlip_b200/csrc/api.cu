@@ -20,18 +20,23 @@ void set_cuda_error(cudaError_t e, const char *where) {
 }
 
 // ---- per-device state: memory pool and error flag ---------------------------
+// One slot per device in a fixed array: a pointer to a slot stays valid for
+// the life of the process, whatever device another thread initialises.  The
+// error flag is per device, shared by every stream of that device (see
+// e2f_stream_status).
+constexpr int MAX_DEVICES = 64;
 struct DeviceState {
   cudaMemPool_t pool = nullptr;
   int *err_flag = nullptr;
 };
 static std::mutex g_mu;
-static std::vector<DeviceState> g_dev;
+static DeviceState g_dev[MAX_DEVICES];
 
 static DeviceState *device_state() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= MAX_DEVICES) return nullptr;
   std::lock_guard<std::mutex> lk(g_mu);
-  if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
   DeviceState &d = g_dev[dev];
   if (!d.pool) {
     cudaMemPoolProps props;
@@ -46,7 +51,7 @@ static DeviceState *device_state() {
   }
   if (!d.err_flag) {
     if (cudaMalloc(&d.err_flag, sizeof(int)) != cudaSuccess) { d.err_flag = nullptr; return nullptr; }
-    cudaMemset(d.err_flag, 0, sizeof(int));
+    if (cudaMemset(d.err_flag, 0, sizeof(int)) != cudaSuccess) return nullptr;
   }
   return &d;
 }
@@ -63,13 +68,15 @@ int *device_error_flag() {
 }
 
 // ---- profiling of the dominant kernel ------------------------------------------
-static bool g_prof_on = false;
+static std::atomic<bool> g_prof_on{false};
+static std::mutex g_prof_mu;
 static std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_events;
 
 static void prof_events(cudaEvent_t *a, cudaEvent_t *b) {
   *a = *b = nullptr;
-  if (!g_prof_on) return;
+  if (!g_prof_on.load()) return;
   if (cudaEventCreate(a) != cudaSuccess || cudaEventCreate(b) != cudaSuccess) { *a = *b = nullptr; return; }
+  std::lock_guard<std::mutex> lk(g_prof_mu);
   g_prof_events.emplace_back(*a, *b);
 }
 
@@ -92,6 +99,9 @@ __global__ void wigner_kernel(const float *__restrict__ R, int64_t n, int L, flo
   wig_all_serial(Rl, L, D + e * wig_size(L));
 }
 
+// Feature rows and weight matrices are read and written as 16-byte vectors.
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 static e2f_status validate_weights(const e2f_weights *w) {
   if (!w) return E2F_ERR_INVALID_ARG;
   if (w->L_max < 0 || w->L_max > E2F_MAX_L || w->C < 1 || w->H < 1) return E2F_ERR_INVALID_ARG;
@@ -102,6 +112,11 @@ static e2f_status validate_weights(const e2f_weights *w) {
   if (!w->W0 || !w->rad_W1 || !w->rad_W2) return E2F_ERR_INVALID_ARG;
   for (int m = 1; m <= w->L_max; ++m)
     if (!w->Wr[m] || !w->Wi[m]) return E2F_ERR_INVALID_ARG;
+  for (int l = 0; l <= w->L_max; ++l)
+    if (!aligned16(w->Wq[l]) || !aligned16(w->Wk[l]) || !aligned16(w->Wv[l])) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(w->W0)) return E2F_ERR_INVALID_ARG;
+  for (int m = 1; m <= w->L_max; ++m)
+    if (!aligned16(w->Wr[m]) || !aligned16(w->Wi[m])) return E2F_ERR_INVALID_ARG;
   return E2F_OK;
 }
 
@@ -161,6 +176,7 @@ e2f_status e2f_project_qkv(const void *x, int64_t N, const e2f_weights *w, void 
   if (st != E2F_OK) return st;
   if (N < 0) return E2F_ERR_INVALID_ARG;
   if (N > 0 && (!x || !q || !k || !v)) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return E2F_ERR_INVALID_ARG;
   return project_impl(x, N, w, q, k, v, static_cast<cudaStream_t>(stream));
 }
 
@@ -172,6 +188,7 @@ e2f_status e2f_attention_forward(const void *x, const float *pos, const e2f_csr 
   const int64_t N = csr->n_nodes;
   if (N == 0) return E2F_OK;
   if (!x || !pos || !out || !csr->row_ptr || (csr->n_edges > 0 && !csr->col_idx)) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
   for (int k = 0; k < 3; ++k)
     if (csr->box[k] > 0.f && !(csr->r_c < 0.5f * csr->box[k])) return E2F_ERR_CUTOFF_TOO_LARGE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -229,6 +246,7 @@ e2f_status e2f_profile_read(int64_t *launches, double *total_ms) {
   double tot = 0.0;
   int64_t n = 0;
   e2f_status st = E2F_OK;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
   for (auto &pr : g_prof_events) {
     float ms = 0.f;
     if (cudaEventSynchronize(pr.second) != cudaSuccess || cudaEventElapsedTime(&ms, pr.first, pr.second) != cudaSuccess)

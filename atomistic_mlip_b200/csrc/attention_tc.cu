@@ -35,6 +35,7 @@
 // All waits are bounded; a timeout raises a CTA-wide abort flag and the
 // device error word (E2F_ERR_TIMEOUT) and every role exits its loops.
 #include <algorithm>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -110,10 +111,18 @@ template <int L> struct Cfg {
   static constexpr size_t G_CS = r16(G_DY + (size_t)TE * NDYP * 2);             // float cos [L][TE], sin [L][TE]
   static constexpr size_t G_GS = r16(G_CS + 2 * (size_t)TE * (L > 0 ? L : 1) * 4);  // half [TE][P]
   static constexpr size_t G_J = r16(G_GS + (size_t)TE * P * 2);                 // int j [TE], node [TE]
-  static constexpr size_t GEO_BYTES = r16(G_J + 2 * (size_t)TE * 4);
+  // online softmax per (node slot, head): the factor that rescales the
+  // node's earlier sums when its running max grows in this tile, and the
+  // running denominator after this tile
+  static constexpr size_t G_F = r16(G_J + 2 * (size_t)TE * 4);                  // float [S][HMAX]
+  static constexpr size_t G_LS = G_F + (size_t)S * HMAX * 4;                     // float [S][HMAX]
+  static constexpr size_t GEO_BYTES = r16(G_LS + (size_t)S * HMAX * 4);
   static constexpr size_t OFF_G2 = OFF_R + 2 * (size_t)NLMAX * TE * 2;
   static constexpr size_t OFF_GEO = OFF_G2 + 2 * GEO_BYTES;          // float [TE][4]: ct, st, u, pad
-  static constexpr size_t OFF_TILE = OFF_GEO + (size_t)TE * 4 * 4;   // 8 ints
+  // producers' running softmax state per (slot, head): max, denominator,
+  // tile max (order-preserving int), tile sum, current max
+  static constexpr size_t OFF_SMX = OFF_GEO + (size_t)TE * 4 * 4;
+  static constexpr size_t OFF_TILE = OFF_SMX + 5 * (size_t)S * HMAX * 4;   // 8 ints
   static constexpr size_t OFF_BAR = (OFF_TILE + 32 + 7) & ~(size_t)7;
   static constexpr int NBAR = 2 * NUNIT + 2 * NSTAGE + 2 + 2 + 2 + 2 + 8;
   static constexpr size_t SMEM = OFF_BAR + NBAR * 8 + 16;
@@ -137,7 +146,6 @@ struct TcArgs {
   int64_t E;
   int H;
   float inv_sqrt_d;
-  float2 *stats;
   const uint8_t *wpack;
   const float *W1, *W2;
   float *out;
@@ -185,13 +193,36 @@ struct Waiter {
   __device__ bool aborted() const { return *abort_flag != 0; }
 };
 
+// Edge range of one CTA, aligned to node boundaries: CTA b of G owns the
+// nodes [n_b, n_{b+1}) with n_0 = 0, n_G = N and, in between, n_b the first
+// node whose row starts at or after edge E b / G; its edges are
+// [row_ptr[n_b], row_ptr[n_{b+1}]).  No node is split between CTAs, so every
+// output row is written by exactly one CTA and the softmax of a node runs
+// inside one CTA.
+__device__ __forceinline__ int first_node_at(const int32_t *rp, int N, int64_t e) {
+  int lo = 0, hi = N;   // smallest n in [0, N] with rp[n] >= e
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)rp[mid] >= e) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
 struct TileIter {
   const int32_t *rp;
   int N;
   int te;   // edges per tile
+  int nlo, nhi;       // nodes owned by this CTA
   int64_t ebeg, eend;
   int64_t e0, e1;
   int n0;
+  __device__ void init(int b, int G, int64_t E) {
+    nlo = b == 0 ? 0 : first_node_at(rp, N, E * (int64_t)b / G);
+    nhi = b + 1 == G ? N : first_node_at(rp, N, E * (int64_t)(b + 1) / G);
+    ebeg = rp[nlo];
+    eend = rp[nhi];
+  }
   __device__ void bounds() {
     const int nlim = min(n0 + S, N);
     int64_t e = e0 + te;
@@ -202,14 +233,8 @@ struct TileIter {
   __device__ bool start() {
     e0 = ebeg;
     if (e0 >= eend) return false;
-    int lo = 0, hi = N - 1;   // largest n with rp[n] <= e0
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((int64_t)rp[mid] <= e0) lo = mid;
-      else hi = mid - 1;
-    }
-    n0 = lo;
-    while ((int64_t)rp[n0 + 1] <= e0) ++n0;
+    n0 = nlo;
+    while ((int64_t)rp[n0 + 1] <= e0) ++n0;   // skip empty rows
     bounds();
     return true;
   }
@@ -242,8 +267,9 @@ struct PackArgs {
   int L;
 };
 
-__global__ void pack_w_kernel(PackArgs a) {
-  // blockIdx.x = stage index; threadIdx.x = row (128)
+__global__ void __launch_bounds__(256) pack_w_kernel(PackArgs a) {
+  // blockIdx.x = stage index; consecutive threads take consecutive source
+  // columns, so the reads of a source row are coalesced
   const int L = a.L;
   int s = blockIdx.x;
   int m = 0;
@@ -256,19 +282,21 @@ __global__ void pack_w_kernel(PackArgs a) {
   const int kh = s % nk;
   const int l = m + (s / nk) / (L - m + 1), lp = m + (s / nk) % (L - m + 1);
   uint8_t *stage = a.dst + (size_t)blockIdx.x * STAGE_BYTES;
-  const int row = threadIdx.x;
   const int n = (L - m + 1) * CH;
-  const size_t srow = (size_t)(l - m) * CH + row;
   if (m == 0) {
     const int scol = lp * CH;
-    for (int k = 0; k < 128; ++k)
+    for (int x = threadIdx.x; x < 128 * 128; x += blockDim.x) {
+      const int row = x >> 7, k = x & 127;
+      const size_t srow = (size_t)(l - m) * CH + row;
       *reinterpret_cast<__nv_bfloat16 *>(stage + kmajor_off(row, k, 128)) = a.W0[srow * n + scol + k];
+    }
   } else {
     const int scol = (lp - m) * CH + kh * 64;
-    for (int t = 0; t < 2; ++t) {
+    for (int x = threadIdx.x; x < 2 * 128 * 64; x += blockDim.x) {
+      const int t = x >> 13, row = (x >> 6) & 127, k = x & 63;
+      const size_t srow = (size_t)(l - m) * CH + row;
       const __nv_bfloat16 *src = (t == 0) ? a.Wr[m] : a.Wi[m];
-      for (int k = 0; k < 64; ++k)
-        *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = src[srow * n + scol + k];
+      *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = src[srow * n + scol + k];
     }
   }
 }
@@ -348,153 +376,25 @@ static bool fit_dy_poly(float *tab) {
   return true;
 }
 
-// Uploads the table to the current device once.
+// Fits the table once per process and uploads it to each device once; safe
+// to call from several host threads.
 static e2f_status ensure_dy_poly() {
   static float tab[DYP_ENTRIES * DYP_STRIDE];
-  static int fitted = 0;   // 0: not yet, 1: ok, -1: failed
+  static std::once_flag fit_once;
+  static bool fitted_ok = false;
+  static std::mutex up_mu;
   static bool uploaded[64] = {};
-  if (fitted == 0) fitted = fit_dy_poly(tab) ? 1 : -1;
-  if (fitted < 0) return E2F_ERR_CUDA;
+  std::call_once(fit_once, [] { fitted_ok = fit_dy_poly(tab); });
+  if (!fitted_ok) return E2F_ERR_CUDA;
   int dev = 0;
   E2F_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(up_mu);
   if (!uploaded[dev]) {
     E2F_CUDA_TRY(cudaMemcpyToSymbol(c_dypoly, tab, sizeof(tab)));
     uploaded[dev] = true;
   }
   return E2F_OK;
-}
-
-// ---------------------------------------------------------------------------
-// per-node softmax statistics (max, envelope-weighted denominator) per head
-// ---------------------------------------------------------------------------
-template <int L>
-__device__ __forceinline__ void norm_sh_row0(float ux, float uy, float uz, float *y0) {
-  // Y'_l^m = sqrt(4 pi / (2l+1)) Y_l^m: P_l(z) at m = 0, and
-  // sqrt(2 (l-m)!/(l+m)!) P_l^m(z) {cos, sin}(m phi), no Condon-Shortley phase.
-  const float rho = sqrtf(ux * ux + uy * uy);
-  float cp = 1.f, sp = 0.f;
-  if (rho > 0.f) { cp = ux / rho; sp = uy / rho; }
-  float cm[L + 1], sm[L + 1];
-  cm[0] = 1.f; sm[0] = 0.f;
-  for (int m = 1; m <= L; ++m) {
-    cm[m] = cm[m - 1] * cp - sm[m - 1] * sp;
-    sm[m] = sm[m - 1] * cp + cm[m - 1] * sp;
-  }
-  float pmm = 1.f;   // P_m^m
-  for (int m = 0; m <= L; ++m) {
-    if (m > 0) pmm *= (float)(2 * m - 1) * rho;
-    float p_lm2 = 0.f, p_lm1 = pmm;
-    // normalisation sqrt(2 (l-m)!/(l+m)!) built incrementally in l
-    for (int l = m; l <= L; ++l) {
-      float p;
-      if (l == m) p = pmm;
-      else if (l == m + 1) p = uz * (2 * m + 1) * pmm;
-      else p = ((2 * l - 1) * uz * p_lm1 - (l + m - 1) * p_lm2) / (float)(l - m);
-      if (l > m) { p_lm2 = p_lm1; p_lm1 = p; }
-      float nrm = 1.f;
-      if (m > 0) {
-        double f = 2.0;
-        for (int t = l - m + 1; t <= l + m; ++t) f /= (double)t;
-        nrm = (float)sqrt(f);
-      }
-      if (m == 0) y0[l * l + l] = p;
-      else {
-        y0[l * l + l + m] = nrm * p * cm[m];
-        y0[l * l + l - m] = nrm * p * sm[m];
-      }
-    }
-  }
-}
-
-template <int L>
-__global__ void __launch_bounds__(256) node_stats_kernel(TcArgs a) {
-  // one block per destination node at a time; items (edge, 8-channel block)
-  // with the node's q row staged in shared memory, k rows gathered a degree
-  // at a time, head sums by shuffles, then an online (max, sum) per head
-  constexpr int Q = (L + 1) * (L + 1);
-  constexpr int EC = 64;   // edges per chunk
-  __shared__ __align__(16) uint4 sq[Q * CH / 8];
-  __shared__ float y0s[EC][Q];
-  __shared__ float us[EC];
-  __shared__ float sv[EC][HMAX + 1];
-  __shared__ float stat_m[HMAX], stat_l[HMAX];
-  const int t = threadIdx.x;
-  const int H = a.H, Ch = CH / H, nb = Ch >> 3;
-  auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
-  for (int i = blockIdx.x; i < a.N; i += gridDim.x) {
-    const int r0 = a.row_ptr[i], r1 = a.row_ptr[i + 1];
-    __syncthreads();
-    for (int x = t; x < Q * CH / 8; x += 256) sq[x] = reinterpret_cast<const uint4 *>(a.q + (size_t)i * Q * CH)[x];
-    if (t < HMAX) { stat_m[t] = -INFINITY; stat_l[t] = 0.f; }
-    const float3 pi = load_pos(a.pos, i);
-    for (int c0 = r0; c0 < r1; c0 += EC) {
-      const int ne = min(EC, r1 - c0);
-      __syncthreads();
-      if (t < ne) {
-        const int j = a.col_idx[c0 + t];
-        float dx, dy, dz;
-        pair_disp(a.g, pi, load_pos(a.pos, j), dx, dy, dz);
-        const float r = sqrtf(dx * dx + dy * dy + dz * dz);
-        float ux = 0.f, uy = 0.f, uz = 1.f;
-        if (r > 0.f) { ux = dx / r; uy = dy / r; uz = dz / r; }
-        norm_sh_row0<L>(ux, uy, uz, y0s[t]);
-        us[t] = 0.5f * (cospif(r / a.g.rc) + 1.f);
-      }
-      __syncthreads();
-      for (int item = t; item < EC * 16; item += 256) {
-        const int e = item >> 4, blk = item & 15;
-        float acc = 0.f;
-        if (e < ne) {
-          const int j = a.col_idx[c0 + e];
-          const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + blk * 8;
-          float2 accv[4];
-#pragma unroll
-          for (int x = 0; x < 4; ++x) accv[x] = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int l = 0; l <= L; ++l) {
-            uint4 kv[2 * L + 1];
-#pragma unroll
-            for (int tt = 0; tt < 2 * l + 1; ++tt) kv[tt] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + tt) * CH);
-            float2 qh[4], kh[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) { qh[x] = make_float2(0.f, 0.f); kh[x] = make_float2(0.f, 0.f); }
-#pragma unroll
-            for (int tt = 0; tt < 2 * l + 1; ++tt) {
-              const float yv = y0s[e][l * l + tt];
-              const float2 y2 = make_float2(yv, yv);
-              const uint4 qv = sq[(l * l + tt) * (CH / 8) + blk];
-              const uint32_t *qw = reinterpret_cast<const uint32_t *>(&qv);
-              const uint32_t *kw = reinterpret_cast<const uint32_t *>(&kv[tt]);
-#pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                qh[x] = __ffma2_rn(y2, pair(qw[x]), qh[x]);
-                kh[x] = __ffma2_rn(y2, pair(kw[x]), kh[x]);
-              }
-            }
-#pragma unroll
-            for (int x = 0; x < 4; ++x) accv[x] = __ffma2_rn(qh[x], kh[x], accv[x]);
-          }
-#pragma unroll
-          for (int x = 0; x < 4; ++x) acc += accv[x].x + accv[x].y;
-        }
-        for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (e < ne && (blk & (nb - 1)) == 0) sv[e][blk / nb] = acc * a.inv_sqrt_d;
-      }
-      __syncthreads();
-      if (t < H) {
-        float mx = stat_m[t];
-        for (int e = 0; e < ne; ++e) mx = fmaxf(mx, sv[e][t]);
-        const float scale = (stat_m[t] == -INFINITY) ? 0.f : expf(stat_m[t] - mx);
-        float sum = 0.f;
-        for (int e = 0; e < ne; ++e) sum += us[e] * expf(sv[e][t] - mx);
-        stat_l[t] = stat_l[t] * scale + sum;
-        stat_m[t] = mx;
-      }
-    }
-    __syncthreads();
-    if (t < H) a.stats[(size_t)i * H + t] = make_float2(stat_m[t] == -INFINITY ? 0.f : stat_m[t], stat_l[t]);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -537,6 +437,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   auto g_cs = [&](int c) { return reinterpret_cast<float *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_CS); };
   auto g_gs = [&](int c) { return reinterpret_cast<__half *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_GS); };
   auto g_jj = [&](int c) { return reinterpret_cast<int *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_J); };
+  auto g_f = [&](int c) { return reinterpret_cast<float *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_F); };
+  auto g_ls = [&](int c) { return reinterpret_cast<float *>(smem + Cf::OFF_G2 + c * Cf::GEO_BYTES + Cf::G_LS); };
 
   if (tid == 0) {
     // unit_full: one arrival per producer warp (the warps fill units independently)
@@ -562,8 +464,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 
   TileIter ti;
   ti.rp = a.row_ptr; ti.N = a.N; ti.te = Cf::TE;
-  ti.ebeg = a.E * (int64_t)blockIdx.x / gridDim.x;
-  ti.eend = a.E * (int64_t)(blockIdx.x + 1) / gridDim.x;
+  ti.init(blockIdx.x, gridDim.x, a.E);
   const int H = a.H, Ch = CH / H;
   const int hshift = 31 - __clz(Ch);   // Ch is a power of two
 
@@ -757,6 +658,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       tmem_st_wait();
       tc_fence_before();
     }
+    // rows of this CTA's nodes with no neighbour are never visited by a
+    // tile: o_i = 0 for them
+    for (int base = ti.nlo + 32 * ew; base < ti.nhi; base += 128) {
+      const int n = base + lane;
+      const bool empty = n < ti.nhi && a.row_ptr[n] == a.row_ptr[n + 1];
+      uint32_t msk = __ballot_sync(0xffffffffu, empty);
+      while (msk) {
+        const int nn = base + __ffs(msk) - 1;
+        msk &= msk - 1;
+        float4 *row = reinterpret_cast<float4 *>(a.out + (size_t)nn * Q * CH);
+        for (int x = lane; x < Q * CH / 4; x += 32) __stcs(row + x, make_float4(0.f, 0.f, 0.f, 0.f));
+      }
+    }
     named_bar(1, 128);
     uint32_t pc = 0, nA0 = 0, nA1 = 0;   // R hand-overs per sign
     int t = 0;
@@ -877,23 +791,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         }
       }
       if (dead) break;
-      if (lane == 0) mbar_arrive(&geo_empty[gc]);   // this geometry copy is free again
-      // ---- tile end: read out the nodes that finished here
+      // ---- tile end: read out the nodes that finished here; the node that
+      // continues into the next tile has its sums rescaled to the next
+      // tile's running max (online softmax), before the next tile's first
+      // back-rotation GEMM (which waits for slots_clean)
       dead = bar_or(1, 128, et == 0 && !W.wait(tile_done, t & 1, 40));
       if (dead) break;
+      const int n1 = nodeof[ne - 1];
+      const bool cont = (int64_t)a.row_ptr[n1 + 1] > ti.e1;   // node n1 continues (next tile exists)
+      if (cont) {
+        dead = bar_or(1, 128, et == 0 && !W.wait(&geo_full[gc ^ 1], ((t + 1) >> 1) & 1, 100));
+        if (dead) break;
+      }
       tc_fence_after();
       {
-        const int n0 = ti.n0;
-        int n1 = ti.n0;
-        while ((int64_t)a.row_ptr[n1 + 1] < ti.e1) ++n1;
-        for (int i = n0; i <= n1; ++i) {
-          const int64_t rb = a.row_ptr[i], re = a.row_ptr[i + 1];
-          if (re == rb) continue;
-          const int64_t reff = re < ti.eend ? re : ti.eend;
-          if (reff > ti.e1) continue;   // continues in the next tile of this CTA
-          const bool shared_node = (rb < ti.ebeg) || (re > ti.eend);
+        const int c = 32 * ew + lane;       // this thread's channel (TMEM lane)
+        const int h = c >> hshift;
+        const float *ls = g_ls(gc), *fnext = g_f(gc ^ 1);
+        for (int i = ti.n0; i <= n1; ++i) {
+          if (a.row_ptr[i + 1] == a.row_ptr[i]) continue;   // empty row: zeroed at the start
           const int slot = i % S;
-          float *orow = a.out + (size_t)i * Q * CH + 32 * ew + lane;
+          const bool fin = !(cont && i == n1);
+          const float lsum = ls[slot * HMAX + h];
+          const float scale = fin ? (lsum > 0.f ? 1.f / lsum : 0.f) : fnext[slot * HMAX + h];
+          float *orow = a.out + (size_t)i * Q * CH + c;
           uint32_t r[Q];
 #pragma unroll
           for (int l = 0; l <= L; ++l) {
@@ -911,11 +832,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 #pragma unroll
             for (int mp = 0; mp < 2 * l + 1; ++mp) {
               const uint32_t col = TM_OUT + Cf::OB(l) + Cf::RO(l) + slot * (2 * l + 1) + mp;
-              float *dst = orow + (size_t)(l * l + mp) * CH;
-              const float val = __uint_as_float(r[l * l + mp]);
-              if (shared_node) atomicAdd(dst, val);
-              else __stcs(dst, val);   // written once: evict-first, keep L2 for the gathers
-              asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col), "r"(0u)
+              const float val = __uint_as_float(r[l * l + mp]) * scale;
+              if (fin) __stcs(orow + (size_t)(l * l + mp) * CH, val);   // written once: evict-first
+              asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col),
+                           "r"(fin ? 0u : __float_as_uint(val))
                            : "memory");
             }
           }
@@ -924,7 +844,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         tc_fence_before();
       }
       named_bar(1, 128);
-      if (lane == 0) mbar_arrive(slots_clean);
+      if (lane == 0) {
+        mbar_arrive(&geo_empty[gc]);   // this geometry copy is free again
+        mbar_arrive(slots_clean);
+      }
       ++t;
       ok = ti.next();
     }
@@ -1043,13 +966,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     // ---- logits -> alpha, items (edge, 8-channel block) of one half of the
     // tile: q and k rows loaded a degree at a time; the blocks of one head
     // are summed with shuffles (16 consecutive lanes = one edge's 16 blocks)
-    auto logits = [&](const TileIter &g, int c, int half) {
+    constexpr int IPH = TE * 8 / 256;   // items per thread and half
+    float sk0[IPH], sk1[IPH];           // logits of this thread's items, by half
+    auto logits = [&](const TileIter &g, int c, int half, float (&sk)[IPH]) {
       const int ne = (int)(g.e1 - g.e0);
       const int *jj = g_jj(c), *nodeof = jj + TE;
       const float *csb = g_cs(c), *snb = csb + TE * (L > 0 ? L : 1);
       const __half *dy = g_dy(c);
-      __half *al = g_al(c);
-      for (int item = pt + half * (TE * 8); item < (half + 1) * (TE * 8); item += 256) {
+#pragma unroll
+      for (int it = 0; it < IPH; ++it) {
+        const int item = pt + half * (TE * 8) + it * 256;
         const int e = item >> 4, c0 = (item & 15) * 8;
         float acc = 0.f;
         if (e < ne) {
@@ -1094,17 +1020,97 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         }
         const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
         for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        const int blk = item & 15;
-        if ((blk & (nb - 1)) == 0) {
-          const int h = blk / nb;
-          float alpha = 0.f;
-          if (e < ne) {
-            const float2 stt = a.stats[(size_t)nodeof[e] * H + h];
-            const float u = geo[e * 4 + 2];
-            alpha = (stt.y > 0.f) ? u * expf(acc * a.inv_sqrt_d - stt.x) / stt.y : 0.f;
-          }
-          al[e * ALS + h] = __float2half_rn(alpha);
+        // the softmax logit with the envelope folded in: u e^s = e^(s + log u)
+        // (the lane owning the head's first block keeps it for the
+        // statistics step)
+        sk[it] = (e < ne) ? acc * a.inv_sqrt_d + logf(geo[e * 4 + 2]) : -INFINITY;
+      }
+    };
+    // ---- online softmax statistics of tile g (copy c), after both logit
+    // halves ("E2Former-V2 ...", §2.2 online softmax; "EquiformerV3 ...",
+    // §2B.3 envelope in numerator and denominator).  Per (node slot, head):
+    // tile max of the logits, running max M (reset when the node starts in
+    // this tile), alpha = e^(s + log u - M) for the tile's edges (fp16, in
+    // (0, 1]), the factor e^(M_old - M) for the node's earlier sums, and the
+    // running denominator l = l_old e^(M_old - M) + sum alpha.
+    int *smx = reinterpret_cast<int *>(smem + Cf::OFF_SMX);      // tile max, order-preserving int
+    float *ssum = reinterpret_cast<float *>(smx + S * HMAX);    // tile sum of alpha
+    float *mcur = ssum + S * HMAX;                               // running max after the tile
+    float *rs_m = mcur + S * HMAX;                               // running max (persists)
+    float *rs_l = rs_m + S * HMAX;                               // running denominator (persists)
+    auto ord = [](float x) { const int i = __float_as_int(x); return i >= 0 ? i : i ^ 0x7fffffff; };
+    auto unord = [](int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); };
+    auto stats_reset = [&]() {
+      if (pt < S * HMAX) { smx[pt] = ord(-INFINITY); ssum[pt] = 0.f; }
+    };
+    auto softmax_stats = [&](const TileIter &g, int c) {
+      const int ne = (int)(g.e1 - g.e0);
+      const int *nodeof = g_jj(c) + TE;
+      __half *al = g_al(c);
+      const int nb = Ch >> 3;
+      // phase A: tile max per (slot, head)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+        for (int it = 0; it < IPH; ++it) {
+          const int item = pt + hf * (TE * 8) + it * 256;
+          const int e = item >> 4, blk = item & 15;
+          if (e < ne && (blk & (nb - 1)) == 0)
+            atomicMax(&smx[(nodeof[e] % S) * HMAX + blk / nb], ord(hf ? sk1[it] : sk0[it]));
         }
+      }
+      named_bar(2, 256);
+      // phase B: running max of the node in each slot
+      bool live = false, starts = false;
+      if (pt < S * HMAX) {
+        const int sl = pt / HMAX, h = pt % HMAX;
+        int node = -1;
+        for (int n = g.n0; n < min(g.n0 + S, a.N); ++n)
+          if (n % S == sl) node = n;
+        float Mn = -INFINITY, f = 1.f;
+        live = node >= 0 && h < H;
+        if (live) {
+          starts = (int64_t)a.row_ptr[node] >= g.e0;
+          const float Mo = starts ? -INFINITY : rs_m[pt];
+          Mn = fmaxf(Mo, unord(smx[pt]));
+          f = (Mn == -INFINITY) ? 1.f : expf(Mo - Mn);
+        }
+        mcur[pt] = Mn;
+        g_f(c)[pt] = f;
+      }
+      named_bar(2, 256);
+      // phase C: alpha of the tile's edges and its per-(slot, head) sum
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+        for (int it = 0; it < IPH; ++it) {
+          const int item = pt + hf * (TE * 8) + it * 256;
+          const int e = item >> 4, blk = item & 15;
+          if (e < TE && (blk & (nb - 1)) == 0) {
+            const int h = blk / nb;
+            float av = 0.f;
+            int sl = 0;
+            if (e < ne) {
+              sl = nodeof[e] % S;
+              const float M = mcur[sl * HMAX + h];
+              av = (M == -INFINITY) ? 0.f : expf((hf ? sk1[it] : sk0[it]) - M);
+            }
+            const __half hv = __float2half_rn(av);
+            al[e * ALS + h] = hv;
+            if (e < ne) atomicAdd(&ssum[sl * HMAX + h], __half2float(hv));   // the rounded values used
+          }
+        }
+      }
+      named_bar(2, 256);
+      // phase D: running denominator after this tile
+      if (pt < S * HMAX) {
+        float lnew = 0.f;
+        if (live) {
+          lnew = (starts ? 0.f : rs_l[pt] * g_f(c)[pt]) + ssum[pt];
+          rs_l[pt] = lnew;
+          rs_m[pt] = mcur[pt];
+        }
+        g_ls(c)[pt] = lnew;
       }
     };
     // geometry step k (0 basics, 1 Wigner, 2 / 3 logits halves) of tile g
@@ -1117,8 +1123,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         basics(g, c);
       } else if (k == 1) {
         wigner(c);
+      } else if (k == 2) {
+        stats_reset();
+        logits(g, c, 0, sk0);
       } else {
-        logits(g, c, k - 2);
+        logits(g, c, 1, sk1);
+        softmax_stats(g, c);
       }
       named_bar(2, 256);
       if (k == 3 && pt == 0) mbar_arrive(&geo_full[c]);
@@ -1377,13 +1387,6 @@ static e2f_status launch_tc(const TcArgs &args, int grid, cudaStream_t s) {
   return E2F_OK;
 }
 
-template <int L>
-static e2f_status launch_stats(const TcArgs &args, cudaStream_t s) {
-  const int grid = (int)std::min<int64_t>(args.N, 148 * 8);
-  E2F_LAUNCH(node_stats_kernel<L>, grid, 256, 0, s, args);
-  return E2F_OK;
-}
-
 }  // namespace tca
 
 e2f_status attention_tc_available(const e2f_weights *w) {
@@ -1400,8 +1403,10 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   const int L = w->L_max;
   const int64_t N = csr->n_nodes, E = csr->n_edges;
   const size_t Q = (size_t)(L + 1) * (L + 1);
-  E2F_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)N * Q * CH * sizeof(float), s));
-  if (E == 0) return E2F_OK;
+  if (E == 0) {   // every row is empty: o = 0
+    E2F_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)N * Q * CH * sizeof(float), s));
+    return E2F_OK;
+  }
   {
     const e2f_status ps = ensure_dy_poly();
     if (ps != E2F_OK) return ps;
@@ -1410,9 +1415,8 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   int nst = 0;
   for (int m = 0; m <= L; ++m) nst += (L - m + 1) * (L - m + 1) * (m == 0 ? 1 : 2);
   const size_t wbytes = (size_t)nst * STAGE_BYTES;
-  Scratch wp, st;
+  Scratch wp;
   E2F_CUDA_TRY(wp.alloc(wbytes, s));
-  E2F_CUDA_TRY(st.alloc((size_t)N * w->H * sizeof(float2), s));
   PackArgs pa;
   pa.W0 = static_cast<const __nv_bfloat16 *>(w->W0);
   for (int m = 0; m <= E2F_MAX_L; ++m) {
@@ -1421,7 +1425,7 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   }
   pa.dst = wp.as<uint8_t>();
   pa.L = L;
-  E2F_LAUNCH(pack_w_kernel, nst, 128, 0, s, pa);
+  E2F_LAUNCH(pack_w_kernel, nst, 256, 0, s, pa);
 
   TcArgs a;
   a.q = static_cast<const __nv_bfloat16 *>(q);
@@ -1441,7 +1445,6 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   a.E = E;
   a.H = w->H;
   a.inv_sqrt_d = 1.f / sqrtf((float)((L + 1) * (CH / w->H)));
-  a.stats = st.as<float2>();
   a.wpack = wp.as<uint8_t>();
   a.W1 = w->rad_W1;
   a.W2 = w->rad_W2;
@@ -1449,16 +1452,6 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   a.err = device_error_flag();
   if (!a.err) return E2F_ERR_CUDA;
   e2f_status r = E2F_OK;
-  switch (L) {
-    case 1: r = launch_stats<1>(a, s); break;
-    case 2: r = launch_stats<2>(a, s); break;
-    case 3: r = launch_stats<3>(a, s); break;
-    case 4: r = launch_stats<4>(a, s); break;
-    case 5: r = launch_stats<5>(a, s); break;
-    case 6: r = launch_stats<6>(a, s); break;
-    default: return E2F_ERR_UNSUPPORTED;
-  }
-  if (r != E2F_OK) return r;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);

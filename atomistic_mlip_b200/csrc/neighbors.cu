@@ -29,8 +29,7 @@ struct CellGrid {
   int stencil[3]; // 1: offsets -1..1, 0: offset 0 only
 };
 
-constexpr int NB_WARPS = 8;
-constexpr int ROW_CAP = 512;   // shared-memory row buffer per warp
+constexpr int ROW_CAP = 256;   // shared-memory row buffer per warp (longer rows: sorted in global memory)
 
 __global__ void bbox_partial_kernel(const float *__restrict__ pos, int n, float *__restrict__ part) {
   float mn[3] = {INFINITY, INFINITY, INFINITY}, mx[3] = {-INFINITY, -INFINITY, -INFINITY};
@@ -108,139 +107,294 @@ __global__ void cell_scatter_kernel(const float *__restrict__ pos, const int32_t
   spos[k] = make_float4(p.x, p.y, p.z, __int_as_float(i));
 }
 
-// Visit the stencil cells of atom i.  The (start, length) of the 27 stencil
-// cells are loaded at once (lane c holds cell c), then the cells are taken
-// four at a time: the atom indices of four cells, then their positions, are
-// loaded before any is used, so a warp waits for a few round trips instead
-// of three per cell.  f(j, pj) is called by every lane for each candidate
-// slot (inactive lanes get j = -1); candidates beyond 32 per cell (dense
-// cells) are visited in extra rounds.  Candidates come from the cell-sorted
-// positions (one 16-byte load: coordinates and the atom's index).
-template <typename F>
-__device__ __forceinline__ void for_stencil(int cid, const CellGrid &cg, const Geom &g,
-                                            const float4 *__restrict__ spos,
-                                            const int32_t *__restrict__ cell_start, int lane, F &&f) {
-  const int cx = cid % cg.nc[0];
-  const int cy = (cid / cg.nc[0]) % cg.nc[1];
-  const int cz = cid / (cg.nc[0] * cg.nc[1]);
-  int my_s = 0, my_n = 0;
-  if (lane < 27) {
-    const int d[3] = {lane % 3 - 1, (lane / 3) % 3 - 1, lane / 9 - 1};
-    const int c0[3] = {cx, cy, cz};
-    int cc[3];
-    bool ok = true;
-#pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      if (d[k] != 0 && cg.stencil[k] == 0) ok = false;
-      int v = c0[k] + d[k];
-      if (g.periodic[k]) v = (v + cg.nc[k]) % cg.nc[k];
-      else if (v < 0 || v >= cg.nc[k]) ok = false;
-      cc[k] = v;
-    }
-    if (ok) {
-      const int c = cc[0] + cg.nc[0] * (cc[1] + cg.nc[1] * cc[2]);
-      my_s = cell_start[c];
-      my_n = cell_start[c + 1] - my_s;
-    }
-  }
-  for (int q0 = 0; q0 < 27; q0 += 4) {
-    int st[4], nn[4], j[4];
-    float3 pj[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      st[q] = __shfl_sync(0xffffffffu, my_s, (q0 + q) & 31);
-      nn[q] = (q0 + q < 27) ? __shfl_sync(0xffffffffu, my_n, (q0 + q) & 31) : 0;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = lane < nn[q] ? spos[st[q] + lane] : make_float4(0.f, 0.f, 0.f, __int_as_float(-1));
-      j[q] = __float_as_int(v.w);
-      pj[q] = make_float3(v.x, v.y, v.z);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) f(j[q], pj[q]);
-#pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-      for (int t = 32; t < nn[q]; t += 32) {   // cells with more than 32 atoms
-        const float4 v = t + lane < nn[q] ? spos[st[q] + t + lane] : make_float4(0.f, 0.f, 0.f, __int_as_float(-1));
-        f(__float_as_int(v.w), make_float3(v.x, v.y, v.z));
+// ---------------------------------------------------------------------------
+// Pair tests, one CTA per home cell (grid-stride over cells).  The atoms of
+// the home cell's stencil cells (27, fewer at open faces or for dimensions
+// of fewer than 3 cells) are staged once in shared memory as candidates,
+// CAND_CAP at a time, and every home atom is tested against them by one warp
+// (lanes over candidates), so a candidate is loaded from global memory once
+// per home cell instead of once per home atom.
+//
+// The minimum image is the exact predicate: d = p_j - p_i rounded, then
+// -b if d > b/2, +b if d < -b/2, each rounded.  When every periodic
+// dimension has at least 5 cells, the branch taken is the same for all
+// candidates of one stencil cell (|d| <= 2 cell edges < b/2 for a cell that
+// does not wrap, |d| >= b - 2 cell edges > b/2 for one that does), so the
+// staged candidate carries that cell's shift s in {-b, 0, +b} and
+// d = fl(fl(p_j - p_i) + s) -- the same rounded operations (adding 0 is
+// exact).  Otherwise every pair takes the branch test.
+// ---------------------------------------------------------------------------
+constexpr int CAND_CAP = 1024;      // candidates staged at a time
+constexpr int CELL_THREADS = 256;
+
+struct Stencil {
+  int n;                // stencil cells
+  int start[27], cnt[27], off[28];
+  float sh[27][3];      // per-cell shift (fast path)
+};
+
+// Stencil of home cell cid: done by thread 0 into shared memory.
+__device__ void make_stencil(int cid, const CellGrid &cg, const Geom &g, const int32_t *__restrict__ cell_start,
+                             Stencil &st) {
+  const int c0[3] = {cid % cg.nc[0], (cid / cg.nc[0]) % cg.nc[1], cid / (cg.nc[0] * cg.nc[1])};
+  int n = 0, tot = 0;
+  for (int dz = -1; dz <= 1; ++dz)
+    for (int dy = -1; dy <= 1; ++dy)
+      for (int dx = -1; dx <= 1; ++dx) {
+        const int d[3] = {dx, dy, dz};
+        int cc[3];
+        float shv[3];
+        bool ok = true;
+        for (int k = 0; k < 3; ++k) {
+          if (d[k] != 0 && cg.stencil[k] == 0) { ok = false; break; }
+          int v = c0[k] + d[k];
+          shv[k] = 0.f;
+          if (g.periodic[k]) {
+            if (v < 0) { v += cg.nc[k]; shv[k] = -g.box[k]; }          // p_j near b, p_i near 0: d > b/2
+            else if (v >= cg.nc[k]) { v -= cg.nc[k]; shv[k] = g.box[k]; }  // d < -b/2
+          } else if (v < 0 || v >= cg.nc[k]) {
+            ok = false;
+            break;
+          }
+          cc[k] = v;
+        }
+        if (!ok) continue;
+        const int c = cc[0] + cg.nc[0] * (cc[1] + cg.nc[1] * cc[2]);
+        st.start[n] = cell_start[c];
+        st.cnt[n] = cell_start[c + 1] - st.start[n];
+        st.off[n] = tot;
+        st.sh[n][0] = shv[0]; st.sh[n][1] = shv[1]; st.sh[n][2] = shv[2];
+        tot += st.cnt[n];
+        ++n;
       }
-    }
+  st.off[n] = tot;
+  st.n = n;
+}
+
+// Candidates [c0, c0 + nc) of the stencil into shared memory.
+__device__ __forceinline__ void stage_candidates(const Stencil &st, int c0, int nc, const float4 *__restrict__ spos,
+                                                 float4 *cp, float4 *cs) {
+  for (int k = threadIdx.x; k < nc; k += blockDim.x) {
+    const int q = c0 + k;
+    int s = 0;
+    while (st.off[s + 1] <= q) ++s;
+    cp[k] = spos[st.start[s] + (q - st.off[s])];
+    cs[k] = make_float4(st.sh[s][0], st.sh[s][1], st.sh[s][2], 0.f);
   }
 }
 
-__global__ void count_kernel(int n, CellGrid cg, Geom g, const int32_t *__restrict__ cell_of,
-                             const int32_t *__restrict__ cell_start, const float4 *__restrict__ spos,
-                             int32_t *__restrict__ deg) {
-  // warp per atom, atoms taken in cell order
-  const int lane = threadIdx.x & 31;
-  const int k = blockIdx.x * NB_WARPS + (threadIdx.x >> 5);
-  if (k >= n) return;
-  const float4 me = spos[k];
-  const int i = __float_as_int(me.w);
-  const float3 pi = make_float3(me.x, me.y, me.z);
-  int cnt = 0;
-  for_stencil(cell_of[i], cg, g, spos, cell_start, lane, [&](int j, float3 pj) {
-    if (j >= 0 && j != i) {
-      float dx, dy, dz;
-      pair_disp(g, pi, pj, dx, dy, dz);
-      if (pair_r2(dx, dy, dz) < g.rc2) ++cnt;
-    }
-  });
-  cnt = warp_sum_i(cnt);
-  if (lane == 0) deg[i] = cnt;
-}
-
-__global__ void fill_kernel(int n, CellGrid cg, Geom g, const int32_t *__restrict__ cell_of,
-                            const int32_t *__restrict__ cell_start, const float4 *__restrict__ spos,
-                            const int32_t *__restrict__ row_ptr, int32_t *__restrict__ col_idx) {
-  __shared__ int32_t buf[NB_WARPS][ROW_CAP];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int k = blockIdx.x * NB_WARPS + wid;
-  if (k >= n) return;
-  const float4 me = spos[k];
-  const int i = __float_as_int(me.w);
-  const int r0 = row_ptr[i];
-  const int deg = row_ptr[i + 1] - r0;
-  const bool in_smem = deg <= ROW_CAP;
-  int32_t *row = col_idx + r0;
-  int32_t *b = buf[wid];
-  const float3 pi = make_float3(me.x, me.y, me.z);
-  int w = 0;
-  for_stencil(cell_of[i], cg, g, spos, cell_start, lane, [&](int j, float3 pj) {
-    bool pass = false;
-    if (j >= 0 && j != i) {
-      float dx, dy, dz;
-      pair_disp(g, pi, pj, dx, dy, dz);
-      pass = pair_r2(dx, dy, dz) < g.rc2;
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, pass);
-    const int p = w + __popc(m & ((1u << lane) - 1u));
-    if (pass && p < deg) {
-      if (in_smem) b[p] = j;
-      else row[p] = j;
-    }
-    w += __popc(m);
-  });
-  __syncwarp();
-  if (in_smem) {
-    // rank placement: keys are distinct atom indices
-    for (int e = lane; e < deg; e += 32) {
-      const int key = b[e];
-      int rank = 0;
-      for (int t = 0; t < deg; ++t) rank += (b[t] < key);
-      row[rank] = key;
-    }
+// The exact predicate for candidate (pj, shift) against pi.
+template <bool FAST>
+__device__ __forceinline__ bool is_edge(const Geom &g, float3 pi, float4 pj, float4 sj) {
+  float dx, dy, dz;
+  if (FAST) {
+    dx = __fadd_rn(__fsub_rn(pj.x, pi.x), sj.x);
+    dy = __fadd_rn(__fsub_rn(pj.y, pi.y), sj.y);
+    dz = __fadd_rn(__fsub_rn(pj.z, pi.z), sj.z);
   } else {
-    // odd-even transposition sort in place (rare long rows)
-    for (int round = 0; round < deg; ++round) {
-      for (int k = 2 * lane + (round & 1); k + 1 < deg; k += 64) {
-        int a = row[k], c = row[k + 1];
-        if (a > c) { row[k] = c; row[k + 1] = a; }
+    pair_disp(g, pi, make_float3(pj.x, pj.y, pj.z), dx, dy, dz);
+  }
+  return pair_r2(dx, dy, dz) < g.rc2;
+}
+
+template <bool FAST>
+__global__ void __launch_bounds__(CELL_THREADS) cell_count_kernel(int ncell, CellGrid cg, Geom g,
+                                                                  const int32_t *__restrict__ cell_start,
+                                                                  const float4 *__restrict__ spos,
+                                                                  int32_t *__restrict__ deg) {
+  __shared__ float4 cp[CAND_CAP], cs[CAND_CAP];
+  __shared__ Stencil st;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int cid = blockIdx.x; cid < ncell; cid += gridDim.x) {
+    const int h0 = cell_start[cid], hn = cell_start[cid + 1] - h0;
+    if (hn == 0) continue;   // uniform across the block
+    __syncthreads();
+    if (threadIdx.x == 0) make_stencil(cid, cg, g, cell_start, st);
+    __syncthreads();
+    const int ntot = st.off[st.n];
+    // home atoms handled by this warp: counts kept per lane slot
+    for (int c0 = 0; c0 < ntot; c0 += CAND_CAP) {
+      const int nc = min(CAND_CAP, ntot - c0);
+      __syncthreads();
+      stage_candidates(st, c0, nc, spos, cp, cs);
+      __syncthreads();
+      for (int a = wid; a < hn; a += nw) {
+        const float4 me = spos[h0 + a];
+        const int i = __float_as_int(me.w);
+        const float3 pi = make_float3(me.x, me.y, me.z);
+        int cnt = 0;
+        for (int k = lane; k < nc; k += 32) {
+          const float4 pj = cp[k];
+          if (__float_as_int(pj.w) != i && is_edge<FAST>(g, pi, pj, cs[k])) ++cnt;
+        }
+        cnt = warp_sum_i(cnt);
+        if (lane == 0) {
+          if (c0 == 0) deg[i] = cnt;
+          else deg[i] += cnt;
+        }
       }
-      __syncwarp();
     }
   }
+}
+
+template <bool FAST>
+__global__ void __launch_bounds__(CELL_THREADS) cell_fill_kernel(int ncell, CellGrid cg, Geom g,
+                                                                 const int32_t *__restrict__ cell_start,
+                                                                 const float4 *__restrict__ spos,
+                                                                 const int32_t *__restrict__ row_ptr,
+                                                                 int32_t *__restrict__ col_idx) {
+  __shared__ float4 cp[CAND_CAP], cs[CAND_CAP];
+  __shared__ Stencil st;
+  __shared__ int32_t rows[CELL_THREADS / 32][ROW_CAP];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int cid = blockIdx.x; cid < ncell; cid += gridDim.x) {
+    const int h0 = cell_start[cid], hn = cell_start[cid + 1] - h0;
+    if (hn == 0) continue;
+    __syncthreads();
+    if (threadIdx.x == 0) make_stencil(cid, cg, g, cell_start, st);
+    __syncthreads();
+    const int ntot = st.off[st.n];
+    if (ntot <= CAND_CAP) {
+      // one chunk: each warp builds its home atoms' rows in shared memory
+      __syncthreads();
+      stage_candidates(st, 0, ntot, spos, cp, cs);
+      __syncthreads();
+      for (int a = wid; a < hn; a += nw) {
+        const float4 me = spos[h0 + a];
+        const int i = __float_as_int(me.w);
+        const float3 pi = make_float3(me.x, me.y, me.z);
+        const int r0 = row_ptr[i], dg = row_ptr[i + 1] - r0;
+        int32_t *out = col_idx + r0;
+        int32_t *b = rows[wid];
+        const bool in_smem = dg <= ROW_CAP;
+        int w = 0;
+        for (int k0 = 0; k0 < ntot; k0 += 32) {
+          const int k = k0 + lane;
+          bool pass = false;
+          int j = -1;
+          if (k < ntot) {
+            const float4 pj = cp[k];
+            j = __float_as_int(pj.w);
+            pass = j != i && is_edge<FAST>(g, pi, pj, cs[k]);
+          }
+          const unsigned m = __ballot_sync(0xffffffffu, pass);
+          const int p = w + __popc(m & ((1u << lane) - 1u));
+          if (pass && p < dg) {
+            if (in_smem) b[p] = j;
+            else out[p] = j;
+          }
+          w += __popc(m);
+        }
+        __syncwarp();
+        if (in_smem) {
+          // rank placement: keys are distinct atom indices
+          for (int e = lane; e < dg; e += 32) {
+            const int key = b[e];
+            int rank = 0;
+            for (int t = 0; t < dg; ++t) rank += (b[t] < key);
+            out[rank] = key;
+          }
+        } else {
+          for (int round = 0; round < dg; ++round) {   // odd-even transposition sort in place (rare)
+            for (int k = 2 * lane + (round & 1); k + 1 < dg; k += 64) {
+              const int x = out[k], y = out[k + 1];
+              if (x > y) { out[k] = y; out[k + 1] = x; }
+            }
+            __syncwarp();
+          }
+        }
+        __syncwarp();
+      }
+    } else {
+      // dense stencil (more candidates than one chunk): rows written to
+      // global memory chunk by chunk, then sorted in place per row
+      int wpos[8];   // per home atom slot of this warp: fill position (up to 8 atoms per warp per pass)
+      for (int a0 = 0; a0 < hn; a0 += 8 * nw) {
+        for (int q = 0; q < 8; ++q) wpos[q] = 0;
+        for (int c0 = 0; c0 < ntot; c0 += CAND_CAP) {
+          const int nc = min(CAND_CAP, ntot - c0);
+          __syncthreads();
+          stage_candidates(st, c0, nc, spos, cp, cs);
+          __syncthreads();
+#pragma unroll 1
+          for (int q = 0; q < 8; ++q) {
+            const int a = a0 + q * nw + wid;
+            if (a >= hn) break;
+            const float4 me = spos[h0 + a];
+            const int i = __float_as_int(me.w);
+            const float3 pi = make_float3(me.x, me.y, me.z);
+            const int r0 = row_ptr[i], dg = row_ptr[i + 1] - r0;
+            for (int k0 = 0; k0 < nc; k0 += 32) {
+              const int k = k0 + lane;
+              bool pass = false;
+              int j = -1;
+              if (k < nc) {
+                const float4 pj = cp[k];
+                j = __float_as_int(pj.w);
+                pass = j != i && is_edge<FAST>(g, pi, pj, cs[k]);
+              }
+              const unsigned m = __ballot_sync(0xffffffffu, pass);
+              const int p = wpos[q] + __popc(m & ((1u << lane) - 1u));
+              if (pass && p < dg) col_idx[r0 + p] = j;
+              wpos[q] += __popc(m);
+            }
+          }
+        }
+        __syncwarp();
+#pragma unroll 1
+        for (int q = 0; q < 8; ++q) {
+          const int a = a0 + q * nw + wid;
+          if (a >= hn) break;
+          const int i = __float_as_int(spos[h0 + a].w);
+          const int r0 = row_ptr[i], dg = row_ptr[i + 1] - r0;
+          int32_t *out = col_idx + r0;
+          for (int round = 0; round < dg; ++round) {
+            for (int k = 2 * lane + (round & 1); k + 1 < dg; k += 64) {
+              const int x = out[k], y = out[k + 1];
+              if (x > y) { out[k] = y; out[k + 1] = x; }
+            }
+            __syncwarp();
+          }
+        }
+      }
+    }
+  }
+}
+
+// Both stencil passes for one grid: the fast shift form when every periodic
+// dimension has at least 5 cells.
+static bool fast_shift_ok(const CellGrid &cg, const Geom &g) {
+  for (int k = 0; k < 3; ++k)
+    if (g.periodic[k] && cg.nc[k] < 5) return false;
+  return true;
+}
+
+static int cell_grid_blocks(long long ncell) {
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  return (int)std::max<long long>(1, std::min<long long>(ncell, (long long)nsm * 8));
+}
+
+static e2f_status launch_count(long long ncell, const CellGrid &cg, const Geom &g, const int32_t *cstart,
+                               const float4 *spos, int32_t *deg, cudaStream_t s) {
+  const int grid = cell_grid_blocks(ncell);
+  if (fast_shift_ok(cg, g))
+    E2F_LAUNCH(cell_count_kernel<true>, grid, CELL_THREADS, 0, s, (int)ncell, cg, g, cstart, spos, deg);
+  else
+    E2F_LAUNCH(cell_count_kernel<false>, grid, CELL_THREADS, 0, s, (int)ncell, cg, g, cstart, spos, deg);
+  return E2F_OK;
+}
+
+static e2f_status launch_fill(long long ncell, const CellGrid &cg, const Geom &g, const int32_t *cstart,
+                              const float4 *spos, const int32_t *row_ptr, int32_t *col_idx, cudaStream_t s) {
+  const int grid = cell_grid_blocks(ncell);
+  if (fast_shift_ok(cg, g))
+    E2F_LAUNCH(cell_fill_kernel<true>, grid, CELL_THREADS, 0, s, (int)ncell, cg, g, cstart, spos, row_ptr, col_idx);
+  else
+    E2F_LAUNCH(cell_fill_kernel<false>, grid, CELL_THREADS, 0, s, (int)ncell, cg, g, cstart, spos, row_ptr,
+               col_idx);
+  return E2F_OK;
 }
 
 // --------------------------------------------------------------------------
@@ -339,9 +493,8 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
   if (st != E2F_OK) return st;
   E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, pos, cell_of.as<int32_t>(), n,
              cstart.as<int32_t>(), cursor.as<int32_t>(), spos.as<float4>());
-  const int nblk = (n + NB_WARPS - 1) / NB_WARPS;
-  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of.as<int32_t>(), cstart.as<int32_t>(),
-             spos.as<float4>(), deg.as<int32_t>());
+  st = launch_count(ncell, cg, g, cstart.as<int32_t>(), spos.as<float4>(), deg.as<int32_t>(), s);
+  if (st != E2F_OK) return st;
   long long *total = nullptr;
   st = exclusive_scan(deg.as<int32_t>(), n, row_ptr, scan_tmp.p, s, &total);
   if (st != E2F_OK) return st;
@@ -357,8 +510,8 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
   if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
   if (E > capacity) return E2F_ERR_CAPACITY;
   if (E > 0) {
-    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of.as<int32_t>(), cstart.as<int32_t>(),
-               spos.as<float4>(), row_ptr, col_idx);
+    st = launch_fill(ncell, cg, g, cstart.as<int32_t>(), spos.as<float4>(), row_ptr, col_idx, s);
+    if (st != E2F_OK) return st;
   }
   return E2F_OK;
 }
@@ -482,14 +635,18 @@ static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, cons
       ncell *= cg.nc[k];
     }
     if (ncell <= cap) break;
-    // coarsen: fewer, larger cells (periodic dims below 3 cells use 1)
-    int kmax = 0;
-    for (int k = 1; k < 3; ++k)
-      if (cg.nc[k] > cg.nc[kmax]) kmax = k;
-    if (g.periodic[kmax]) {
-      cg.nc[kmax] = cg.nc[kmax] - 1 < 3 ? 1 : cg.nc[kmax] - 1;
-    } else {
-      cs[kmax] *= 1.25;
+    // coarsen every dimension at once by the factor that brings the count to
+    // the cap: cells only grow, which never drops a pair.  A periodic count
+    // falls by at least one per pass and becomes 1 below 3; open cells grow
+    // by at least 25 % per pass, so the loop ends after a few passes.
+    const double f = cbrt((double)cap / (double)ncell);
+    for (int k = 0; k < 3; ++k) {
+      if (g.periodic[k]) {
+        int nc = std::min((int)floor(cg.nc[k] * f), cg.nc[k] - 1);
+        cg.nc[k] = nc < 3 ? 1 : nc;
+      } else {
+        cs[k] *= std::max(1.25, 1.0 / f);
+      }
     }
   }
   if (ncell > NOALLOC_MAX_CELLS) return E2F_ERR_SCRATCH_LIMIT;
@@ -511,8 +668,8 @@ static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, cons
   st = exclusive_scan(cnt, ncell, cstart, scan_tmp, s, nullptr);
   if (st != E2F_OK) return st;
   E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, pos, cell_of, n, cstart, cursor, spos);
-  const int nblk = (n + NB_WARPS - 1) / NB_WARPS;
-  E2F_LAUNCH(count_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of, cstart, spos, deg);
+  st = launch_count(ncell, cg, g, cstart, spos, deg, s);
+  if (st != E2F_OK) return st;
   long long *total = nullptr;
   st = exclusive_scan(deg, n, row_ptr, scan_tmp, s, &total);
   if (st != E2F_OK) return st;
@@ -526,7 +683,8 @@ static e2f_status build_neighbors_noalloc_impl(const float *pos, int64_t N, cons
   if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
   if (E > capacity) return E2F_ERR_CAPACITY;
   if (E > 0) {
-    E2F_LAUNCH(fill_kernel, nblk, 32 * NB_WARPS, 0, s, n, cg, g, cell_of, cstart, spos, row_ptr, col_idx);
+    st = launch_fill(ncell, cg, g, cstart, spos, row_ptr, col_idx, s);
+    if (st != E2F_OK) return st;
   }
   return E2F_OK;
 }

@@ -2,13 +2,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = the whole path on one batch: the cell-list CSR build plus the
+One step = the whole path on one system: the cell-list CSR build plus the
 fused attention forward (projections, edge geometry, Wigner-D, logits,
 online softmax, SO(2) block products, back-rotation, accumulation).
-Workload: 256 drug-like molecules of 20-60 atoms (N = 10,304 atoms, about
-395k directed edges within r_c = 6 A), L_max = 4, C = 128, 8 heads, bf16
-storage with fp32 accumulation; synthetic, seeded inputs.  Each rank runs
-its own batch (weak scaling, no collective on the data path).
+Headline workload: the 100,002-atom periodic water box (33,334 rigid
+waters in a 100.0007 A cube, r_c = 6 A, about 8.7 M directed edges),
+L_max = 4, C = 128, 8 heads, bf16 storage with fp32 accumulation;
+synthetic, seeded inputs.  Each rank runs its own system (weak scaling, no
+collective on the data path).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA
 events on the working stream; L2 is flushed (256 MiB write) between steps,
@@ -18,6 +19,12 @@ that time.  `e2e` repeats the measurement through the public API with the
 inputs copied from pinned host memory and the output copied back inside
 every step.  The dominant kernel (the fused attention kernel) is timed live
 with CUDA events recorded by the library on its stream.
+
+At one GPU the same line also carries `workloads` (every other workload:
+the 256-molecule batch, the 3,000-atom water box, the 30,000-atom
+protein-in-water box at L_max = 6; each row against its own roofline) and
+`memory_sweep` (peak device memory and edges/s of the water box at 10k,
+30k and 100k atoms, with a linear fit in N).
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead
 (rank 0 only; bounded samples of the same workload per step).
@@ -40,9 +47,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-WORKLOAD_CFG = 1
-WORKLOAD_DESC = ("256 drug-like molecules, 20-60 atoms each, open boundaries, r_c = 6 A; "
-                 "L_max = 4, C = 128, H = 8; bf16 storage / fp32 accumulate")
+WORKLOAD_CFG = 4
+WORKLOAD_DESC = ("periodic water box, 100,002 atoms (33,334 rigid waters) in a 100.0007 A cube, "
+                 "minimum image, r_c = 6 A; L_max = 4, C = 128, H = 8; bf16 storage / fp32 accumulate")
+EXTRA_DESC = {1: "256 drug-like molecules, 20-60 atoms each, open boundaries, r_c = 6 A; L=4, C=128, H=8, bf16",
+              2: "periodic water box, 3,000 atoms in a 31 A cube, r_c = 6 A; L=4, C=128, H=8, bf16",
+              3: ("30,000-atom box: 3,000-atom compact chain + 9,000 waters in a 66.94 A cube, r_c = 6 A; "
+                  "L=6, C=128, H=8, bf16"),
+              4: "periodic water box, 100,002 atoms, r_c = 6 A; L=4, C=128, H=8, bf16"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 L2_FLUSH_BYTES = 256 << 20
 
@@ -100,7 +112,8 @@ def reduce_sum(value: float, dist, device) -> float:
 
 
 def rank_seed(rank: int) -> int:
-    """Each rank draws its own batch of molecules (weak scaling)."""
+    """Each rank draws its own system (weak scaling); rank 0's is the seeded
+    workload itself."""
     from atomistic_mlip_b200 import workloads as w
     return w.BASE_SEED + WORKLOAD_CFG + 1000 * rank
 
@@ -188,6 +201,95 @@ def kernel_traffic(peaks_kernel: str):
     return d.get("dram_bytes_per_launch")
 
 
+def _box_list(wl):
+    return None if wl.box is None else [float(b) for b in wl.box]
+
+
+def measure_workload(cfg, dev, peaks, peak_src, reps=5, warm=2, n_target=None, wl=None):
+    """One workload against its rooflines: the neighbour build (HBM:
+    algorithmic bytes 12N + 4(N+1) + 4E) and the fused attention kernel
+    (tensor: F(L, C) FLOP per edge over the kernel's own event time), plus
+    the whole attention call and peak device memory.  Median of `reps`
+    calls after `warm`; CUDA events on the working stream."""
+    import torch
+    from atomistic_mlip_b200 import e2f
+    from atomistic_mlip_b200 import workloads as w
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    if wl is None:
+        wl = w.make_workload(cfg, n_target=n_target)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(dev)
+    e2f.scratch_high_water(reset=True)
+    pos = torch.from_numpy(wl.pos).to(dev)
+    x = torch.from_numpy(wl.x).to(dev, torch.bfloat16 if wl.precision == "bf16" else torch.float32)
+    dw = e2f.DeviceWeights.from_workload(wl, dev)
+    box = _box_list(wl)
+    nl = e2f.build_neighbors(pos, box, wl.r_c)
+    E = nl.n_edges
+    row_ptr = torch.empty(wl.N + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(1, E), dtype=torch.int32, device=dev)
+
+    def nb():
+        e2f.build_neighbors(pos, box, wl.r_c, row_ptr=row_ptr, col_idx=col_idx)
+    for _ in range(warm):
+        nb()
+    t_nb = timed(nb)
+    nb_bytes = 12 * wl.N + 4 * (wl.N + 1) + 4 * E
+    o = torch.empty((wl.N, (wl.L + 1) ** 2, wl.C), dtype=torch.float32, device=dev)
+
+    def att():
+        e2f.attention_forward(x, pos, nl, dw, out=o)
+    for _ in range(warm):
+        att()
+    e2f.profile_enable(True)
+    t_call = timed(att)
+    e2f.profile_enable(False)
+    n_k, k_ms = e2f.profile_read()
+    k_ms = k_ms / max(n_k, 1)
+    F = so2_flops_per_edge(wl.L, wl.C)
+    peak = float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
+    res = {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}") if n_target is None else
+           f"periodic water box, {wl.N} atoms, r_c = 6 A; L=4, C=128, H=8, bf16",
+           "N": wl.N, "E": E, "L": wl.L,
+           "neighbour_build": {"ms": t_nb, "algorithmic_bytes": nb_bytes,
+                               "achieved_gbs": nb_bytes / (t_nb * 1e-3) / 1e9,
+                               "frac_hbm": nb_bytes / (t_nb * 1e-3) / 1e9 / hbm,
+                               "note": "whole call, including its host read-backs"},
+           "attention": {"call_ms": t_call, "fused_kernel_ms": k_ms,
+                         "edges_per_s": E / (t_call * 1e-3), "node_updates_per_s": wl.N / (t_call * 1e-3),
+                         "achieved_tflops": F * E / (k_ms * 1e-3) / 1e12,
+                         "frac": F * E / (k_ms * 1e-3) / 1e12 / peak, "flops_per_edge": F},
+           "peak_device_bytes": {"torch": int(torch.cuda.max_memory_allocated(dev)),
+                                 "library_scratch": int(e2f.scratch_high_water())}}
+    del o, x, pos, dw, nl, row_ptr, col_idx
+    torch.cuda.empty_cache()
+    return res
+
+
+def linear_fit(ns, ys):
+    """Least-squares y = a + b N and its R^2."""
+    A = np.stack([np.ones(len(ns)), np.asarray(ns, float)], 1)
+    coef, *_ = np.linalg.lstsq(A, np.asarray(ys, float), rcond=None)
+    pred = A @ coef
+    ss_res = float(np.sum((np.asarray(ys) - pred) ** 2))
+    ss_tot = float(np.sum((np.asarray(ys) - np.mean(ys)) ** 2)) or 1.0
+    return {"intercept_bytes": float(coef[0]), "bytes_per_atom": float(coef[1]), "r2": 1.0 - ss_res / ss_tot}
+
+
 def run_ours(args):
     import torch
     from atomistic_mlip_b200 import e2f
@@ -203,6 +305,7 @@ def run_ours(args):
 
     wl = w.make_workload(WORKLOAD_CFG, seed=rank_seed(rank))
     L, C, H = wl.L, wl.C, wl.H
+    box = _box_list(wl)
     pos_h = torch.from_numpy(wl.pos).pin_memory()
     x_h = torch.from_numpy(wl.x).to(torch.bfloat16).pin_memory()
     pos = pos_h.to(dev)
@@ -213,12 +316,12 @@ def run_ours(args):
     out_h = torch.empty((wl.N, Q, C), dtype=torch.float32).pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    cap = 64 * wl.N
+    cap = 128 * wl.N
     row_ptr = torch.empty(wl.N + 1, dtype=torch.int32, device=dev)
     col_idx = torch.empty(cap, dtype=torch.int32, device=dev)
 
     def step():
-        nl = e2f.build_neighbors(pos, None, wl.r_c, row_ptr=row_ptr, col_idx=col_idx)
+        nl = e2f.build_neighbors(pos, box, wl.r_c, row_ptr=row_ptr, col_idx=col_idx)
         e2f.attention_forward(x, pos, nl, dw, out=out)
         return nl.n_edges
 
@@ -266,11 +369,13 @@ def run_ours(args):
             e2e_evs.append((a, b))
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
+    h2d_bytes = int(pos_h.numel() * 4 + x_h.numel() * 2)
+    d2h_bytes = int(out_h.numel() * 4)
 
     t_max = reduce_max(t_ms, dist, dev)
     e2e_max = reduce_max(e2e_ms, dist, dev)
     edges_all = reduce_sum(float(edges), dist, dev)
-    e2e_edges_all = edges_all  # same batches
+    e2e_edges_all = edges_all  # same systems
     peaks, peak_src = load_peaks()
     F = so2_flops_per_edge(L, C)
     E_rank = edges // args.steps
@@ -282,6 +387,24 @@ def run_ours(args):
         if dist is not None:
             dist.destroy_process_group()
         return
+
+    extras = {}
+    if world == 1 and not args.headline_only:
+        # free the headline's buffers before the other workloads
+        del out, out_h, x, pos, flush, row_ptr, col_idx, dw, pos_h, x_h
+        torch.cuda.empty_cache()
+        rows = [measure_workload(cfg, dev, peaks, peak_src) for cfg in (1, 2, 3)]
+        sweep = [measure_workload(4, dev, peaks, peak_src, n_target=n) for n in (10002, 30000)]
+        sweep.append(measure_workload(4, dev, peaks, peak_src, wl=wl))
+        ns = [r["N"] for r in sweep]
+        tot = [r["peak_device_bytes"]["torch"] + r["peak_device_bytes"]["library_scratch"] for r in sweep]
+        extras["workloads"] = rows + [sweep[-1]]
+        extras["memory_sweep"] = {
+            "N": ns, "peak_device_bytes": tot,
+            "edges_per_s": [r["attention"]["edges_per_s"] for r in sweep],
+            "frac": [r["attention"]["frac"] for r in sweep],
+            "fit": linear_fit(ns, tot),
+            "what": "torch.cuda.max_memory_allocated + the library pool's high-water mark, per attention call"}
 
     cpu = cpu_baseline(wl) if world == 1 else None
     line = {
@@ -298,21 +421,22 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded generator; no dataset)",
         "config": {"workload": WORKLOAD_DESC, "N_atoms_per_rank": wl.N, "edges_per_step_rank0": E_rank,
-                   "l2": "flushed between steps (256 MiB write outside the step events)",
-                   "step": "e2f_build_neighbors + e2f_attention_forward", "parallelism": f"dp{world} (independent batches)"},
+                   "l2": "flushed between steps (256 MiB write outside the step events); inputs exceed L2",
+                   "step": "e2f_build_neighbors + e2f_attention_forward", "parallelism": f"dp{world} (independent systems)"},
         "node_updates_per_s": wl.N * world * args.steps / (t_max * 1e-3),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_source": f"bf16_tflops burst, {peak_src}",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "kernel": "fused attention", "flops_per_edge": F, "launches": n_attn,
                      "avg_launch_ms": avg_attn_ms,
                      "traffic": kernel_traffic("attention")},
         "e2e": {"value": e2e_edges_all / (e2e_max * 1e-3), "unit": "edges/s",
-                "h2d_bytes_per_step": int(pos_h.numel() * 4 + x_h.numel() * 2),
-                "d2h_bytes_per_step": int(out_h.numel() * 4)},
+                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
         "gpu_launches": int(launches),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
+    line.update(extras)
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -328,36 +452,34 @@ def _cores():
         return os.cpu_count() or 1
 
 
-def oracle_sample_step(wl, csr, nodes):
-    """One oracle pass over a sample: brute-force CSR of the whole batch and
-    the attention of the sampled destination rows; returns edges done."""
+def oracle_sample_step(wl, nodes):
+    """One oracle pass over a sample of destination rows: their brute-force
+    neighbour rows, then their attention; returns the edges done."""
     from oracle import attention as oa
     from oracle import neighbors as nb
-    rp, col = nb.neighbors(wl.pos, wl.box, wl.r_c)
+    rp, col = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)
     oa.attention_workload(wl, nodes=nodes, csr=(rp, col))
     return int(sum(rp[i + 1] - rp[i] for i in nodes))
 
 
 def cpu_baseline(wl, budget_s: float = 15.0, chunk: int = 64):
-    """Oracle edges/s on the host cores over a bounded sample of rows."""
+    """Oracle edges/s on the host cores over a bounded sample of rows of the
+    seeded 1,000-node subset (brute-force rows + attention, both timed)."""
     from threadpoolctl import threadpool_limits
-    from oracle import attention as oa
-    from oracle import neighbors as nb
     cores = _cores()
+    order = np.random.default_rng(7).permutation(wl.subset)
     with threadpool_limits(limits=cores):
-        rp, col = nb.neighbors(wl.pos, wl.box, wl.r_c)
-        order = np.random.default_rng(7).permutation(wl.N)
         t0 = time.perf_counter()
         edges, rows, k = 0, 0, 0
-        while time.perf_counter() - t0 < budget_s and k < wl.N:
+        while time.perf_counter() - t0 < budget_s and k < len(order):
             nodes = np.sort(order[k:k + chunk])
-            oa.attention_workload(wl, nodes=nodes, csr=(rp, col))
-            edges += int(sum(rp[i + 1] - rp[i] for i in nodes))
+            edges += oracle_sample_step(wl, nodes)
             rows += len(nodes)
             k += chunk
         dt = time.perf_counter() - t0
     return {"value": edges / dt, "unit": "edges/s", "cores": cores, "kind": "oracle",
-            "sample": f"{rows} random destination rows ({edges} edges) of the benchmark batch, fp64 NumPy, {dt:.1f} s"}
+            "sample": (f"{rows} rows of the seeded 1,000-node subset ({edges} edges) of the benchmark system: "
+                       f"brute-force neighbour rows + attention, fp64 NumPy, {dt:.1f} s")}
 
 
 def run_reference(args):
@@ -368,14 +490,14 @@ def run_reference(args):
     from atomistic_mlip_b200 import workloads as w
     wl = w.make_workload(WORKLOAD_CFG, seed=rank_seed(0))
     cores = _cores()
-    rows_per_step = 48
-    order = np.random.default_rng(11).permutation(wl.N)
+    rows_per_step = 24
+    order = np.random.default_rng(11).permutation(wl.subset)
     times, edges = [], 0
     with threadpool_limits(limits=cores):
         for k in range(args.warmup + args.steps):
-            nodes = np.sort(order[(k * rows_per_step) % wl.N:][:rows_per_step])
+            nodes = np.sort(np.resize(np.roll(order, -k * rows_per_step), rows_per_step))
             t0 = time.perf_counter()
-            e = oracle_sample_step(wl, None, nodes)
+            e = oracle_sample_step(wl, nodes)
             dt = time.perf_counter() - t0
             if k >= args.warmup:
                 times.append(dt)
@@ -389,7 +511,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator; no dataset)",
         "config": {"workload": WORKLOAD_DESC, "N_atoms_per_rank": wl.N,
-                   "sample_per_step": f"brute-force CSR of the batch + attention of {rows_per_step} rows"},
+                   "sample_per_step": f"brute-force neighbour rows + attention of {rows_per_step} destination rows"},
         "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores, "kind": "oracle",
                          "sample": f"{rows_per_step} destination rows per step, fp64 NumPy oracle"},
         "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -398,119 +520,45 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------
-# per-row measurements (one JSON line per hot-path row and workload)
+# per-row measurements (one JSON line per workload)
 # ----------------------------------------------------------------------------
 def run_rows(args):
-    """Each row of the hot path against its own roofline, on every workload:
-    the neighbour build (HBM: algorithmic bytes 12N + 4(N+1) + 4E, the
-    positions read, row_ptr and col_idx written) and the fused attention
-    (tensor: F(L, C) FLOP per edge), plus peak device memory against N on the
-    water-box sweep.  Times are CUDA events on the working stream, median of
-    `--steps` calls after `--warmup`; the neighbour build's time includes its
-    two host read-backs (bounding box, edge count)."""
+    """Each workload against its rooflines, one JSON line each (the same
+    measurement the default line carries under `workloads`)."""
     import torch
     from atomistic_mlip_b200 import e2f
-    from atomistic_mlip_b200 import workloads as w
-
     if not torch.cuda.is_available():
         raise SystemExit("bench.py --rows needs a CUDA device")
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     e2f.lib()
     peaks, peak_src = load_peaks()
-    stream = torch.cuda.current_stream(dev)
-
-    def timed(fn, reps):
-        ts = []
-        for _ in range(reps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
-
-    def one(cfg, n_target=None, attention=True, reps=None):
-        steps = args.steps if reps is None else reps
-        warm = args.warmup if reps is None else 1
-        wl = w.make_workload(cfg, n_target=n_target)
-        torch.cuda.synchronize()
-        torch.cuda.reset_peak_memory_stats(dev)
-        e2f.scratch_high_water(reset=True)
-        pos = torch.from_numpy(wl.pos).to(dev)
-        x = torch.from_numpy(wl.x).to(dev, torch.bfloat16 if wl.precision == "bf16" else torch.float32)
-        dw = e2f.DeviceWeights.from_workload(wl, dev)
-        box = None if wl.box is None else [float(b) for b in wl.box]
-        nl = e2f.build_neighbors(pos, box, wl.r_c)
-        cap = nl.n_edges
-        row_ptr = torch.empty(wl.N + 1, dtype=torch.int32, device=dev)
-        col_idx = torch.empty(max(1, cap), dtype=torch.int32, device=dev)
-
-        def nb():
-            e2f.build_neighbors(pos, box, wl.r_c, row_ptr=row_ptr, col_idx=col_idx)
-        for _ in range(warm):
-            nb()
-        t_nb = timed(nb, steps)
-        E = nl.n_edges
-        nb_bytes = 12 * wl.N + 4 * (wl.N + 1) + 4 * E
-        out = {"row": "A1-A3 neighbour build", "workload": wl.cfg_name if hasattr(wl, "cfg_name") else f"cfg{cfg}",
-               "N": wl.N, "E": E, "ms": t_nb,
-               "roofline": {"bound": "hbm", "algorithmic_bytes": nb_bytes,
-                            "achieved": nb_bytes / (t_nb * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
-                            "unit": "GB/s", "frac": nb_bytes / (t_nb * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
-                            "peak_source": f"hbm_gbs, {peak_src}"}}
-        print(json.dumps(out), flush=True)
-        if not attention:
-            return
-        o = torch.empty((wl.N, (wl.L + 1) ** 2, wl.C), dtype=torch.float32, device=dev)
-
-        def att():
-            e2f.attention_forward(x, pos, nl, dw, out=o)
-        for _ in range(warm):
-            att()
-        e2f.profile_enable(True)
-        t_call = timed(att, steps)
-        e2f.profile_enable(False)
-        n_k, k_ms = e2f.profile_read()
-        k_ms = k_ms / max(n_k, 1)
-        F = so2_flops_per_edge(wl.L, wl.C)
-        peak = float(peaks["bf16_tflops"])
-        out = {"row": "A4-A11 attention forward (projections + fused kernel)", "workload": f"cfg{cfg}",
-               "N": wl.N, "E": E, "L": wl.L, "C": wl.C, "H": wl.H, "precision": wl.precision,
-               "call_ms": t_call, "fused_kernel_ms": k_ms,
-               "edges_per_s": E / (t_call * 1e-3), "node_updates_per_s": wl.N / (t_call * 1e-3),
-               "roofline": {"bound": "tensor", "flops_per_edge": F, "achieved": F * E / (k_ms * 1e-3) / 1e12,
-                            "peak": peak, "unit": "TFLOP/s", "frac": F * E / (k_ms * 1e-3) / 1e12 / peak,
-                            "peak_source": f"bf16_tflops burst, {peak_src}",
-                            "path": "tcgen05" if (wl.precision == "bf16" and wl.C == 128 and 1 <= wl.L <= 6) else "SIMT"},
-               "peak_device_bytes": {"torch": int(torch.cuda.max_memory_allocated(dev)),
-                                     "library_scratch": int(e2f.scratch_high_water())}}
-        print(json.dumps(out), flush=True)
-        del o
-
-    if args.rows_what == "neighbors":
-        one(4, attention=False)
-        return
-    for cfg in (1, 2, 4):
-        one(cfg)
-    for n in (10002, 30000):   # memory sweep of the water box (cfg4 is the 100k point)
-        one(4, n_target=n)
-    one(3)
+    what = args.rows_what
+    cfgs = {"all": (1, 2, 4, 3), "neighbors": (4,), "molecules": (1,), "water3k": (2,), "protein": (3,),
+            "water100k": (4,)}[what]
+    for cfg in cfgs:
+        print(json.dumps(measure_workload(cfg, dev, peaks, peak_src, reps=args.steps, warm=args.warmup)),
+              flush=True)
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rows", action="store_true", help="per-row measurements on every workload (one GPU)")
-    ap.add_argument("--rows-what", choices=["all", "neighbors"], default="all",
-                    help="with --rows: every row, or the neighbour build of the 100k-atom water box only")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other workloads and the memory sweep (profiling runs)")
+    ap.add_argument("--rows", action="store_true", help="one JSON line per workload (one GPU)")
+    ap.add_argument("--rows-what", choices=["all", "neighbors", "molecules", "water3k", "protein", "water100k"],
+                    default="all")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    _, world, _ = dist_env()
+    if args.gpus != world:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE = {world}; launch N > 1 ranks with "
+                         f"torchrun (--nproc-per-node N), one process per GPU")
     if args.rows:
         run_rows(args)
     elif args.impl == "reference":

@@ -23,6 +23,9 @@
  *     coefficient (l, m), m = -l..l, sits at index l*l + l + m of the Q
  *     axis (real spherical harmonics without the Condon-Shortley phase,
  *     l = 1 ordered (y, z, x)).
+ *   - Feature arrays (x, q, k, v, out) and the weight matrices Wq/Wk/Wv,
+ *     W0, Wr, Wi are accessed as 16-byte vectors: their device pointers
+ *     must be 16-byte aligned (E2F_ERR_INVALID_ARG otherwise).
  *   - Errors are returned as e2f_status; nothing is written to outputs when
  *     argument validation fails.  Device-side problems (a bounded wait that
  *     gave up) are latched in a per-device flag that e2f_stream_status()
@@ -129,6 +132,9 @@ E2F_API e2f_status e2f_build_neighbors(const float *pos, int64_t N, const float 
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The address is kept for the life of the process: a cudaDeviceReset (or
+ * any teardown of the device's primary context) invalidates this entry
+ * point for the rest of the process.
  * Every call on a device uses the same array and finds the previous call's
  * contents in it (the call clears what must start at zero); calls whose GPU
  * work can overlap, e.g. on two streams with no ordering between them,
@@ -191,6 +197,14 @@ E2F_API e2f_status e2f_attention_forward(const void *x, const float *pos, const 
  * e2f_stream_status -- synchronise `stream`, then return (and clear) any
  * error latched by a kernel of this library on the current device
  * (E2F_ERR_TIMEOUT for a bounded wait that gave up), or E2F_ERR_CUDA.
+ *
+ * Scope: the latched word is per DEVICE, not per stream.  Kernels on every
+ * stream of the device write the same word, so a call for stream s1 also
+ * reports (and clears) an error raised by work on stream s2 that has
+ * finished by then.  Callers that run independent work on several streams
+ * and need to tell whose work failed synchronise those streams and call
+ * this once per device.  Argument validation itself keeps no state: the
+ * entry points may be called from several host threads at once.
  */
 E2F_API e2f_status e2f_stream_status(void *stream);
 
@@ -228,7 +242,8 @@ E2F_API int64_t e2f_kernel_launches(void);
  * enabled, every e2f_attention_forward records a CUDA event pair around
  * that kernel on its stream.  e2f_profile_read() synchronises those
  * events, returns the number of launches and their summed duration in
- * milliseconds, and clears the record.  Process-wide; not thread-safe.
+ * milliseconds, and clears the record.  Process-wide: launches from every
+ * host thread and stream are recorded together.
  */
 E2F_API e2f_status e2f_profile_enable(int32_t on);
 E2F_API e2f_status e2f_profile_read(int64_t *launches, double *total_ms);

@@ -153,11 +153,12 @@ def attention(pos: np.ndarray, box: Optional[np.ndarray], r_c: float,
     # projections of the rows that are needed (q of destinations, k/v of sources)
     need_src = np.unique(np.concatenate([col[row_ptr[i]:row_ptr[i + 1]] for i in nodes]
                                         + [np.zeros(0, np.int64)]))
-    x64 = np.asarray(x, np.float64)
-    q_rows = project(x64[nodes], Wq, L)
+    # (only the rows used are widened to fp64; the widening is exact)
+    x_src = np.asarray(np.asarray(x)[need_src], np.float64)
+    q_rows = project(np.asarray(np.asarray(x)[nodes], np.float64), Wq, L)
     src_map = {int(j): t for t, j in enumerate(need_src)}
-    k_rows = project(x64[need_src], Wk, L) if len(need_src) else np.zeros((0, Q, C))
-    v_rows = project(x64[need_src], Wv, L) if len(need_src) else np.zeros((0, Q, C))
+    k_rows = project(x_src, Wk, L) if len(need_src) else np.zeros((0, Q, C))
+    v_rows = project(x_src, Wv, L) if len(need_src) else np.zeros((0, Q, C))
 
     # chunks of destination nodes with a bounded number of edges
     deg = row_ptr[nodes + 1] - row_ptr[nodes]

@@ -97,6 +97,27 @@ def neighbors_c(pos: np.ndarray, box: Optional[np.ndarray], r_c: float) -> Tuple
     return row_ptr, col
 
 
+def neighbor_rows(pos: np.ndarray, box: Optional[np.ndarray], r_c: float,
+                  rows: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Brute-force CSR that lists only the given rows (every other row is
+    empty): row i of it equals row i of the full radius graph for i in
+    `rows`.  For sampled destination rows of a large system."""
+    pos = np.ascontiguousarray(pos, dtype=np.float32)
+    n = pos.shape[0]
+    rows = np.unique(np.asarray(rows, np.int64))
+    deg = np.zeros(n, np.int64)
+    cols = []
+    for r0 in range(0, len(rows), 256):
+        rr = rows[r0:r0 + 256]
+        m = _pair_mask(pos, rr, box, r_c)
+        deg[rr] = m.sum(axis=1)
+        cols.append(np.nonzero(m)[1].astype(np.int32))
+    row_ptr = np.zeros(n + 1, np.int64)
+    np.cumsum(deg, out=row_ptr[1:])
+    col = np.concatenate(cols) if cols else np.zeros(0, np.int32)
+    return row_ptr, col
+
+
 def neighbors(pos, box, r_c):
     """CSR (row_ptr int64 [N+1], col int32 [E]); C loop above 4096 atoms."""
     if np.asarray(pos).shape[0] > 4096:

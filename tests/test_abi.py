@@ -92,3 +92,53 @@ def test_unit_entry_validation(lib):
     assert lib.e2f_wigner_d(None, 0, 3, None, None) == 0
     assert lib.e2f_project_qkv(d, -1, ctypes.byref(_weights()), d, d, d, None) == 1
     assert lib.e2f_profile_read(None, None) == 1
+
+
+def test_misaligned_pointers_rejected(lib):
+    """Feature and weight pointers are read as 16-byte vectors: a pointer
+    that is not 16-byte aligned is rejected on the host."""
+    csr = e2f.Csr()
+    csr.row_ptr = 64; csr.col_idx = 64; csr.n_nodes = 4; csr.n_edges = 4; csr.r_c = 1.0
+    f = lib.e2f_attention_forward
+    d, odd = ctypes.c_void_p(64), ctypes.c_void_p(72)
+    assert f(odd, d, ctypes.byref(csr), ctypes.byref(_weights()), d, None) == 1
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(_weights()), odd, None) == 1
+    w = _weights()
+    w.Wr[1] = 72
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(w), d, None) == 1
+    assert lib.e2f_project_qkv(d, 4, ctypes.byref(_weights()), d, odd, d, None) == 1
+
+
+def test_validation_from_two_host_threads(lib):
+    """The entry points keep no state while validating arguments: two host
+    threads calling them at once each get the status of their own call."""
+    import threading
+    errors = []
+
+    def worker(seed):
+        n_e = ctypes.c_int64(0)
+        d = ctypes.c_void_p(64)
+        csr = e2f.Csr()
+        csr.row_ptr = 64; csr.col_idx = 64; csr.n_nodes = 4; csr.n_edges = 4; csr.r_c = 1.0
+        box = (ctypes.c_float * 3)(10.0, 10.0, 10.0)
+        for it in range(2000):
+            k = (it + seed) % 4
+            if k == 0:
+                got, want = lib.e2f_build_neighbors(d, -1, None, 1.0, d, d, 10, ctypes.byref(n_e), None, None), 1
+            elif k == 1:
+                got, want = lib.e2f_build_neighbors(d, 10, box, 5.0, d, d, 10, ctypes.byref(n_e), None, None), 2
+            elif k == 2:
+                got, want = lib.e2f_attention_forward(d, d, ctypes.byref(csr), ctypes.byref(_weights(C=8, H=3)),
+                                                      d, None), 4
+            else:
+                got, want = lib.e2f_attention_forward(d, d, ctypes.byref(csr), ctypes.byref(_weights(L=7)),
+                                                      d, None), 1
+            if got != want:
+                errors.append((seed, it, got, want))
+
+    ts = [threading.Thread(target=worker, args=(s,)) for s in (0, 1)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert not errors, errors[:5]

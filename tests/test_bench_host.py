@@ -78,6 +78,20 @@ def test_reference_arm_line():
 
 def test_reference_arm_other_ranks_exit_quietly():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2")
-    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference"],
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2"],
                          capture_output=True, text=True, env=env, timeout=120, cwd=ROOT)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_gpus_flag_must_match_world_size():
+    """--gpus N without N ranks fails loudly instead of measuring one GPU."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "8"],
+                         capture_output=True, text=True, env=env, timeout=120, cwd=ROOT)
+    assert out.returncode != 0 and "WORLD_SIZE" in out.stderr
+
+
+def test_linear_fit():
+    fit = bench.linear_fit([10, 30, 100], [1000 + 40 * n for n in (10, 30, 100)])
+    assert abs(fit["bytes_per_atom"] - 40) < 1e-9 and abs(fit["intercept_bytes"] - 1000) < 1e-6
+    assert abs(fit["r2"] - 1.0) < 1e-12

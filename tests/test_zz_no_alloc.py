@@ -68,3 +68,43 @@ def test_noalloc_limits(cuda_ok):
     assert c1 == 0 and c2 == 0
     np.testing.assert_array_equal(rp1, rp2)
     np.testing.assert_array_equal(col1, col2)
+
+
+def test_noalloc_sparse_periodic_box(cuda_ok):
+    """A sparse periodic box whose natural cell grid (166^3 cells) is far
+    above the fixed scratch's cell limit: the no-allocation build coarsens
+    every periodic dimension at once and still gives the brute-force CSR,
+    bit for bit, and the same CSR as the standard build."""
+    import torch
+    from oracle import neighbors as nb
+    rng = np.random.default_rng(12)
+    box = np.full(3, 1000.0, np.float32)
+    pos_np = rng.uniform(0, 1000.0, (10000, 3)).astype(np.float32)
+    # a few close pairs so that the graph is not empty
+    pos_np[1::50] = np.mod(pos_np[0::50] + rng.uniform(-3, 3, pos_np[0::50].shape), 1000.0).astype(np.float32)
+    pos_np[pos_np >= 1000.0] = 0.0
+    pos = torch.from_numpy(pos_np).cuda()
+    rp_o, col_o = nb.neighbors(pos_np, box, 6.0)
+    assert rp_o[-1] > 0
+    c1, rp1, col1 = _call("e2f_build_neighbors", pos, box, 6.0, 1 << 16)
+    for _ in range(2):
+        c2, rp2, col2 = _call("e2f_build_neighbors_noalloc", pos, box, 6.0, 1 << 16)
+        assert c1 == 0 and c2 == 0
+        np.testing.assert_array_equal(rp2, rp_o)
+        np.testing.assert_array_equal(col2, col_o)
+        np.testing.assert_array_equal(rp2, rp1)
+        np.testing.assert_array_equal(col2, col1)
+
+
+def test_noalloc_water_100k_vs_oracle(cuda_ok):
+    """The 100,002-atom periodic water box (below the 131,072-atom limit)
+    against the oracle's all-pairs CSR, twice in a row."""
+    import torch
+    wl = helpers.cached_workload(4, "bf16")
+    rp_o, col_o = helpers.oracle_csr(4)
+    pos = torch.from_numpy(wl.pos).cuda()
+    for _ in range(2):
+        code, rp, col = _call("e2f_build_neighbors_noalloc", pos, wl.box, wl.r_c, 128 * wl.N)
+        assert code == 0
+        np.testing.assert_array_equal(rp, rp_o)
+        np.testing.assert_array_equal(col, col_o)

@@ -392,6 +392,23 @@ def make_workload(cfg: int, precision: Optional[str] = None, seed: Optional[int]
                     subset=subset, seed=sd, meta=meta)
 
 
+def make_layer_weights(L: int, C: int, H: int, precision: str, seed: int, hidden_mult: int = 4) -> Dict:
+    """Weights of one E2Former-V2 block: the attention's (drawn as in
+    make_workload) plus the two merged-norm gains (float32, 1 + 0.1 N(0, 1)
+    per (degree, channel)) and the FFN maps Wa [Hd][C], Wb[l] [Hd][C],
+    Wd[l] [C][Hd] (Hd = hidden_mult C, N(0, 1/fan_in)), seeded."""
+    rng = np.random.default_rng(seed)
+    (_, Wq, Wk, Wv, W0, Wr, Wi, w1, w2) = _draw_features_and_weights(rng, 0, L, C, precision)
+    Hd = hidden_mult * C
+    g1 = (1.0 + 0.1 * rng.standard_normal((L + 1, C))).astype(np.float32)
+    g2 = (1.0 + 0.1 * rng.standard_normal((L + 1, C))).astype(np.float32)
+    Wa = round_to(rng.standard_normal((Hd, C)) / math.sqrt(C), precision)
+    Wb = [round_to(rng.standard_normal((Hd, C)) / math.sqrt(C), precision) for _ in range(L + 1)]
+    Wd = [round_to(rng.standard_normal((C, Hd)) / math.sqrt(Hd), precision) for _ in range(L + 1)]
+    return dict(L=L, C=C, H=H, precision=precision, Wq=Wq, Wk=Wk, Wv=Wv, W0=W0, Wr=Wr, Wi=Wi, rad_W1=w1,
+                rad_W2=w2, gamma1=g1, gamma2=g2, Wa=Wa, Wb=Wb, Wd=Wd)
+
+
 def make_custom(pos: np.ndarray, box: Optional[np.ndarray], r_c: float, L: int, C: int,
                 H: int, precision: str = "fp32", seed: int = 0) -> Workload:
     """Features and weights for caller-given positions (edge-case tests)."""

@@ -54,7 +54,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(lambda s: _compile(s, extra), _sources()))
     tmp = OUT + ".tmp"
-    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs])
+    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcublas"])
     os.replace(tmp, OUT)
     return OUT
 

@@ -120,6 +120,45 @@ static e2f_status validate_weights(const e2f_weights *w) {
   return E2F_OK;
 }
 
+static e2f_status validate_csr(const e2f_csr *csr) {
+  if (!csr || csr->n_nodes < 0 || csr->n_edges < 0 || !(csr->r_c > 0.f)) return E2F_ERR_INVALID_ARG;
+  if (csr->n_nodes > 0 && (!csr->row_ptr || (csr->n_edges > 0 && !csr->col_idx))) return E2F_ERR_INVALID_ARG;
+  for (int k = 0; k < 3; ++k)
+    if (csr->box[k] > 0.f && !(csr->r_c < 0.5f * csr->box[k])) return E2F_ERR_CUTOFF_TOO_LARGE;
+  return E2F_OK;
+}
+
+e2f_status block_forward_impl(const float *x, const float *pos, const e2f_csr *csr, const e2f_block_weights *w,
+                              float *out, cudaStream_t s);
+e2f_status attention_backward_impl(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
+                                   const float *G, float *dx, float *dpos, cudaStream_t s);
+
+// q, k, v (library scratch), then the fused attention kernel; arguments
+// already validated.
+e2f_status attention_forward_impl(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
+                                  float *out, cudaStream_t s) {
+  const int64_t N = csr->n_nodes;
+  if (N == 0) return E2F_OK;
+  const size_t Q = (size_t)(w->L_max + 1) * (w->L_max + 1);
+  const size_t esz = w->dtype == E2F_F32 ? 4 : 2;
+  const size_t feat = (size_t)N * Q * w->C * esz;
+  Scratch qkv;
+  E2F_CUDA_TRY(qkv.alloc(3 * feat, s));
+  char *base = qkv.as<char>();
+  void *q = base, *k = base + feat, *v = base + 2 * feat;
+  e2f_status st = project_impl(x, N, w, q, k, v, s);
+  if (st != E2F_OK) return st;
+  cudaEvent_t ev0, ev1;
+  prof_events(&ev0, &ev1);
+  if (w->dtype == E2F_BF16 && attention_tc_available(w) == E2F_OK)
+    return attention_tc_impl(q, k, v, pos, csr, w, out, s, ev0, ev1);
+  if (w->dtype == E2F_F32)
+    return attention_simt_impl<float>((const float *)q, (const float *)k, (const float *)v, pos, csr, w, out, s,
+                                      ev0, ev1);
+  return attention_simt_impl<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                            (const __nv_bfloat16 *)v, pos, csr, w, out, s, ev0, ev1);
+}
+
 }  // namespace e2f
 
 using namespace e2f;
@@ -184,32 +223,42 @@ e2f_status e2f_attention_forward(const void *x, const float *pos, const e2f_csr 
                                  float *out, void *stream) {
   e2f_status st = validate_weights(w);
   if (st != E2F_OK) return st;
-  if (!csr || csr->n_nodes < 0 || csr->n_edges < 0 || !(csr->r_c > 0.f)) return E2F_ERR_INVALID_ARG;
-  const int64_t N = csr->n_nodes;
-  if (N == 0) return E2F_OK;
-  if (!x || !pos || !out || !csr->row_ptr || (csr->n_edges > 0 && !csr->col_idx)) return E2F_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
-  for (int k = 0; k < 3; ++k)
-    if (csr->box[k] > 0.f && !(csr->r_c < 0.5f * csr->box[k])) return E2F_ERR_CUTOFF_TOO_LARGE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t Q = (size_t)(w->L_max + 1) * (w->L_max + 1);
-  const size_t esz = w->dtype == E2F_F32 ? 4 : 2;
-  const size_t feat = (size_t)N * Q * w->C * esz;
-  Scratch qkv;
-  E2F_CUDA_TRY(qkv.alloc(3 * feat, s));
-  char *base = qkv.as<char>();
-  void *q = base, *k = base + feat, *v = base + 2 * feat;
-  st = project_impl(x, N, w, q, k, v, s);
+  st = validate_csr(csr);
   if (st != E2F_OK) return st;
-  cudaEvent_t ev0, ev1;
-  prof_events(&ev0, &ev1);
-  if (w->dtype == E2F_BF16 && attention_tc_available(w) == E2F_OK)
-    return attention_tc_impl(q, k, v, pos, csr, w, out, s, ev0, ev1);
-  if (w->dtype == E2F_F32)
-    return attention_simt_impl<float>((const float *)q, (const float *)k, (const float *)v, pos, csr, w, out, s,
-                                      ev0, ev1);
-  return attention_simt_impl<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
-                                            (const __nv_bfloat16 *)v, pos, csr, w, out, s, ev0, ev1);
+  if (csr->n_nodes == 0) return E2F_OK;
+  if (!x || !pos || !out) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
+  return attention_forward_impl(x, pos, csr, w, out, static_cast<cudaStream_t>(stream));
+}
+
+e2f_status e2f_attention_backward(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
+                                  const float *grad_out, float *grad_x, float *grad_pos, void *stream) {
+  e2f_status st = validate_weights(w);
+  if (st != E2F_OK) return st;
+  st = validate_csr(csr);
+  if (st != E2F_OK) return st;
+  if (w->H > 16) return E2F_ERR_UNSUPPORTED;
+  if (csr->n_nodes == 0) return E2F_OK;
+  if (!x || !pos || !grad_out || !grad_x || !grad_pos) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x)) return E2F_ERR_INVALID_ARG;
+  return attention_backward_impl(x, pos, csr, w, grad_out, grad_x, grad_pos, static_cast<cudaStream_t>(stream));
+}
+
+e2f_status e2f_block_forward(const float *x, const float *pos, const e2f_csr *csr, const e2f_block_weights *w,
+                             float *out, void *stream) {
+  if (!w) return E2F_ERR_INVALID_ARG;
+  e2f_status st = validate_weights(&w->attn);
+  if (st != E2F_OK) return st;
+  st = validate_csr(csr);
+  if (st != E2F_OK) return st;
+  const int L = w->attn.L_max;
+  if (w->hidden < 1 || !w->gamma1 || !w->gamma2 || !w->Wa || !aligned16(w->Wa)) return E2F_ERR_INVALID_ARG;
+  for (int l = 0; l <= L; ++l)
+    if (!w->Wb[l] || !w->Wd[l] || !aligned16(w->Wb[l]) || !aligned16(w->Wd[l])) return E2F_ERR_INVALID_ARG;
+  if (csr->n_nodes == 0) return E2F_OK;
+  if (!x || !pos || !out || x == out) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
+  return block_forward_impl(x, pos, csr, w, out, static_cast<cudaStream_t>(stream));
 }
 
 e2f_status e2f_stream_status(void *stream) {

@@ -1,0 +1,747 @@
+// Backward of the on-the-fly equivariant attention: dL/dx and dL/dpos of a
+// scalar L = sum(G * o) -- the conservative forces are -dL/dpos ("E2Former-V2
+// ...", technical summary §4: the conservative variant, forces as the
+// gradient of the energy; "DPA4 ...", §2.2 energy-to-force path).
+//
+// Recompute, per chunk of whole destination nodes (at most CHUNK_E edges):
+//   K1 edge_fwd     geometry, D^l blocks of the two-angle frame, envelope,
+//                   radial MLP, logits s; the rotated features
+//                   v~ = D v_j in SO(2)-stacked order
+//   K2 node_stats   per (node, head) max and denominator of e^(s + log u)
+//   GEMM            Y_m = V~_m Wc_m^T for every m: Wc_0 = W0, Wc_m =
+//                   [[Wr, -Wi], [Wi, Wr]] acting on (v~+, v~-)  (cuBLAS)
+//   K3 edge_dalpha  y = g Y; GD = D G_i (the output gradient in the edge
+//                   frame); dalpha_h = <y, GD>_h; alpha_h
+//   K4 node_delta   Delta_h = sum_e alpha_h dalpha_h  (= <G_i, o_i>_h)
+//   K5 edge_dy      ds_h = alpha_h (dalpha_h - Delta_h); dL/du; dy = alpha GD;
+//                   dL/dg; dw = g dy (stacked)
+//   GEMM            dV~_m = dW_m Wc_m  (transposed SO(2) products)
+//   K6 edge_bwd     dL/dD^l from the rotate-in, the back-rotation and the
+//                   m = 0 rows of the logits; the rotation generators turn
+//                   it into a torque tau_k = -<D^T dL/dD, J_k>, so that
+//                   dL/dr_ij = (dL/dr) rhat + tau x rhat / r; atomics into
+//                   dL/dpos of both atoms and into dL/dq_i, dL/dk_j, dL/dv_j
+// then
+//   K7 dx           dL/dx = per degree dq Wq + dk Wk + dv Wv.
+//
+// Per-edge tensors live only inside a chunk (bounded scratch); the SO(2)
+// products are dense GEMMs over the chunk's edges.
+#include <cublas_v2.h>
+#include <math.h>
+
+#include <algorithm>
+#include <mutex>
+#include <type_traits>
+#include <vector>
+
+#include "common.cuh"
+#include "wigner.cuh"
+
+namespace e2f {
+
+e2f_status project_impl(const void *, int64_t, const e2f_weights *, void *, void *, void *, cudaStream_t);
+
+namespace bwd {
+
+constexpr int BT = 128;            // threads per edge block
+constexpr int CHUNK_E = 1 << 16;   // edges per chunk (at least one whole node)
+constexpr int JMAX = (E2F_MAX_L + 1) * (2 * E2F_MAX_L + 1) * (2 * E2F_MAX_L + 3) / 3;   // sum (2l+1)^2
+
+// J_k^l = d/dt D^l(exp(t K_k)) at t = 0, k = x, y, z (K_k v = e_k x v),
+// blocks laid out like the Wigner blocks; fitted on the host by a central
+// difference of the Ivanic-Ruedenberg construction.
+__constant__ float c_gen[3 * JMAX];
+
+struct Args {
+  int L, C, H, N;
+  float inv_sqrt_d;
+  Geom g;
+  const int32_t *row_ptr, *col_idx;
+  const float *pos;
+  const void *q, *k, *v;          // [N][Q][C], storage type
+  const float *G;                 // dL/do [N][Q][C]
+  const float *W1, *W2;
+  // chunk
+  int na, nb;                     // nodes [na, nb)
+  int64_t ea, ne;                 // edges [ea, ea + ne)
+  void *A, *dY;                   // [ne][QC] storage type (stacked)
+  float *Y, *dA;                  // [ne][QC] fp32 (stacked)
+  float *Dm, *gv, *zv, *sv, *uv, *rv, *al, *dal, *dsv, *duv, *dgv;
+  float *Mv, *denv, *dlt;         // per node of the chunk [nb - na][H]
+  // accumulators
+  float *dq, *dk, *dv;            // [N][Q][C] fp32
+  float *dpos;                    // [N][3]
+};
+
+template <typename T> __device__ __forceinline__ float ldf(const void *p, size_t i) {
+  return to_f(static_cast<const T *>(p)[i]);
+}
+
+__device__ __forceinline__ int node_of_edge(const int32_t *rp, int na, int nb, int64_t e) {
+  int lo = na, hi = nb - 1;   // largest n with rp[n] <= e
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)rp[mid] <= e) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// D^l blocks of the edge frame into shared memory (block-cooperative).
+template <int L>
+__device__ void edge_wigner(float ux, float uy, float uz, float *D) {
+  if (threadIdx.x == 0) {
+    D[0] = 1.f;
+    if (L >= 1) {
+      float R[9];
+      edge_frame_two_angle(ux, uy, uz, R);
+      wig_l1_from_rotation(R, D + 1);
+    }
+  }
+  __syncthreads();
+  for (int l = 2; l <= L; ++l) {
+    const int w = 2 * l + 1;
+    for (int x = threadIdx.x; x < w * w; x += blockDim.x)
+      D[wig_offset(l) + x] = wig_entry(l, x / w - l, x % w - l, D + 1, D + wig_offset(l - 1));
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K1: geometry, D, envelope, radial MLP, logits; v~ = D v_j (stacked)
+// ---------------------------------------------------------------------------
+template <typename T, int L>
+__global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
+  constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  constexpr int P = (L + 1) * (L + 2) / 2;
+  __shared__ float D[S];
+  __shared__ float hid[16], geo[8], hs[16];
+  const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
+  for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
+    const int64_t e = a.ea + el;
+    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    const int j = a.col_idx[e];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float dx, dy, dz;
+      pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dy, dz);
+      const float r = sqrtf(dx * dx + dy * dy + dz * dz);
+      geo[0] = dx; geo[1] = dy; geo[2] = dz; geo[3] = r;
+      geo[4] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+      a.rv[el * 4 + 0] = dx; a.rv[el * 4 + 1] = dy; a.rv[el * 4 + 2] = dz; a.rv[el * 4 + 3] = r;
+      a.uv[el] = geo[4];
+    }
+    __syncthreads();
+    const float r = geo[3];
+    float ux = 0.f, uy = 0.f, uz = 1.f;
+    if (r > 0.f) { ux = geo[0] / r; uy = geo[1] / r; uz = geo[2] / r; }
+    edge_wigner<L>(ux, uy, uz, D);
+    for (int x = threadIdx.x; x < S; x += blockDim.x) a.Dm[el * S + x] = D[x];
+    // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5) -> 16 SiLU -> P
+    if (threadIdx.x < 16) {
+      float z = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const float dd = r - (float)kk * (a.g.rc / 7.f);
+        z = fmaf(a.W1[threadIdx.x * 8 + kk], expf(-dd * dd * 2.f), z);
+      }
+      a.zv[el * 16 + threadIdx.x] = z;
+      hid[threadIdx.x] = z / (1.f + expf(-z));
+    }
+    __syncthreads();
+    if (threadIdx.x < P) {
+      float gg = 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 16; ++hh) gg = fmaf(a.W2[threadIdx.x * 16 + hh], hid[hh], gg);
+      a.gv[el * P + threadIdx.x] = gg;
+    }
+    // logits: the m = 0 rows of D q_i and D k_j, per head
+    if (threadIdx.x < 16) hs[threadIdx.x] = 0.f;
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float s = 0.f;
+#pragma unroll
+      for (int l = 0; l <= L; ++l) {
+        const int w = 2 * l + 1;
+        const float *row0 = D + wig_offset(l) + l * w;
+        float qh = 0.f, kh = 0.f;
+        for (int mp = 0; mp < w; ++mp) {
+          qh = fmaf(row0[mp], ldf<T>(a.q, ((size_t)i * Q + l * l + mp) * C + c), qh);
+          kh = fmaf(row0[mp], ldf<T>(a.k, ((size_t)j * Q + l * l + mp) * C + c), kh);
+        }
+        s = fmaf(qh, kh, s);
+      }
+      atomicAdd(&hs[c / Ch], s);
+    }
+    __syncthreads();
+    if (threadIdx.x < H) a.sv[el * H + threadIdx.x] = hs[threadIdx.x] * a.inv_sqrt_d;
+    // rotate in: v~[(l,m),c] = sum_m' D^l[m][m'] v_j[(l,m'),c], stacked
+    T *Arow = static_cast<T *>(a.A) + (size_t)el * QC;
+    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
+      const int l = x / C, c = x % C, w = 2 * l + 1;
+      float vv[2 * L + 1];
+#pragma unroll
+      for (int mp = 0; mp < 2 * L + 1; ++mp) vv[mp] = mp < w ? ldf<T>(a.v, ((size_t)j * Q + l * l + mp) * C + c) : 0.f;
+      const float *Dl = D + wig_offset(l);
+      for (int m = -l; m <= l; ++m) {
+        float acc = 0.f;
+#pragma unroll
+        for (int mp = 0; mp < 2 * L + 1; ++mp)
+          if (mp < w) acc = fmaf(Dl[(m + l) * w + mp], vv[mp], acc);
+        Arow[stack_off(L, C, m) + (l - (m < 0 ? -m : m)) * C + c] = from_f<T>(acc);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K2 / K4: per (node, head) reductions over the node's edges (warp per node)
+// ---------------------------------------------------------------------------
+__global__ void node_stats_kernel(Args a) {
+  const int lane = threadIdx.x & 31;
+  for (int n = a.na + blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.nb;
+       n += gridDim.x * (blockDim.x >> 5)) {
+    const int64_t e0 = a.row_ptr[n] - a.ea, e1 = a.row_ptr[n + 1] - a.ea;
+    if (lane < a.H) {
+      float M = -INFINITY;
+      for (int64_t e = e0; e < e1; ++e) M = fmaxf(M, a.sv[e * a.H + lane] + logf(a.uv[e]));
+      float den = 0.f;
+      if (M > -INFINITY)
+        for (int64_t e = e0; e < e1; ++e) den += expf(a.sv[e * a.H + lane] + logf(a.uv[e]) - M);
+      a.Mv[(size_t)(n - a.na) * a.H + lane] = M;
+      a.denv[(size_t)(n - a.na) * a.H + lane] = den;
+    }
+  }
+}
+
+__global__ void node_delta_kernel(Args a) {
+  const int lane = threadIdx.x & 31;
+  for (int n = a.na + blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.nb;
+       n += gridDim.x * (blockDim.x >> 5)) {
+    const int64_t e0 = a.row_ptr[n] - a.ea, e1 = a.row_ptr[n + 1] - a.ea;
+    if (lane < a.H) {
+      float d = 0.f;
+      for (int64_t e = e0; e < e1; ++e) d = fmaf(a.al[e * a.H + lane], a.dal[e * a.H + lane], d);
+      a.dlt[(size_t)(n - a.na) * a.H + lane] = d;
+    }
+  }
+}
+
+// GD[(l,m),c] = sum_m' D^l[m][m'] G_i[(l,m'),c] for one (l, c)
+template <int L>
+__device__ __forceinline__ void rotate_col(const float *D, const float *src, int l, int c, int C, float *out) {
+  const int w = 2 * l + 1;
+  float gg[2 * L + 1];
+#pragma unroll
+  for (int mp = 0; mp < 2 * L + 1; ++mp) gg[mp] = mp < w ? src[(size_t)(l * l + mp) * C + c] : 0.f;
+  const float *Dl = D + wig_offset(l);
+#pragma unroll
+  for (int m = 0; m < 2 * L + 1; ++m) {
+    if (m >= w) break;
+    float acc = 0.f;
+#pragma unroll
+    for (int mp = 0; mp < 2 * L + 1; ++mp)
+      if (mp < w) acc = fmaf(Dl[m * w + mp], gg[mp], acc);
+    out[m] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K3: alpha and dalpha per (edge, head)
+// ---------------------------------------------------------------------------
+template <int L>
+__global__ void __launch_bounds__(BT) edge_dalpha_kernel(Args a) {
+  constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  constexpr int P = (L + 1) * (L + 2) / 2;
+  __shared__ float D[S];
+  __shared__ float hs[16];
+  const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
+  for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
+    const int64_t e = a.ea + el;
+    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    __syncthreads();
+    for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
+    if (threadIdx.x < 16) hs[threadIdx.x] = 0.f;
+    __syncthreads();
+    const float *Gi = a.G + (size_t)i * QC;
+    const float *Yr = a.Y + (size_t)el * QC;
+    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
+      const int l = x / C, c = x % C;
+      float gd[2 * L + 1];
+      rotate_col<L>(D, Gi, l, c, C, gd);
+      float s = 0.f;
+      for (int m = -l; m <= l; ++m) {
+        const int am = m < 0 ? -m : m;
+        const float y = a.gv[el * P + pair_index(L, am, l)] * Yr[stack_off(L, C, m) + (l - am) * C + c];
+        s = fmaf(y, gd[m + l], s);
+      }
+      atomicAdd(&hs[c / Ch], s);
+    }
+    __syncthreads();
+    if (threadIdx.x < H) {
+      const int h = threadIdx.x;
+      const float M = a.Mv[(size_t)(i - a.na) * H + h], den = a.denv[(size_t)(i - a.na) * H + h];
+      const float sp = a.sv[el * H + h] + logf(a.uv[el]);
+      a.al[el * H + h] = (den > 0.f && M > -INFINITY) ? expf(sp - M) / den : 0.f;
+      a.dal[el * H + h] = hs[h];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K5: ds, dL/du, dy = alpha GD, dL/dg, dw = g dy (stacked)
+// ---------------------------------------------------------------------------
+template <typename T, int L>
+__global__ void __launch_bounds__(BT) edge_dy_kernel(Args a) {
+  constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  constexpr int P = (L + 1) * (L + 2) / 2;
+  __shared__ float D[S];
+  __shared__ float dsh[16], alh[16], dgp[P];
+  const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
+  for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
+    const int64_t e = a.ea + el;
+    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    __syncthreads();
+    for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
+    if (threadIdx.x < P) dgp[threadIdx.x] = 0.f;
+    if (threadIdx.x < H) {
+      const int h = threadIdx.x;
+      const float al = a.al[el * H + h], diff = a.dal[el * H + h] - a.dlt[(size_t)(i - a.na) * H + h];
+      alh[h] = al;
+      dsh[h] = al * diff;
+      a.dsv[el * H + h] = al * diff;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // dL/du = sum_h e^(s - M) / den (dalpha - Delta)  (no division by u)
+      float du = 0.f;
+      for (int h = 0; h < H; ++h) {
+        const float M = a.Mv[(size_t)(i - a.na) * H + h], den = a.denv[(size_t)(i - a.na) * H + h];
+        if (den > 0.f && M > -INFINITY)
+          du += expf(a.sv[el * H + h] - M) / den * (a.dal[el * H + h] - a.dlt[(size_t)(i - a.na) * H + h]);
+      }
+      a.duv[el] = du;
+    }
+    const float *Gi = a.G + (size_t)i * QC;
+    const float *Yr = a.Y + (size_t)el * QC;
+    T *dYr = static_cast<T *>(a.dY) + (size_t)el * QC;
+    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
+      const int l = x / C, c = x % C;
+      const float alc = alh[c / Ch];
+      float gd[2 * L + 1];
+      rotate_col<L>(D, Gi, l, c, C, gd);
+      for (int m = -l; m <= l; ++m) {
+        const int am = m < 0 ? -m : m, p = pair_index(L, am, l);
+        const int so = stack_off(L, C, m) + (l - am) * C + c;
+        const float dy = alc * gd[m + l];
+        atomicAdd(&dgp[p], dy * Yr[so]);
+        dYr[so] = from_f<T>(dy * a.gv[el * P + p]);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < P) a.dgv[el * P + threadIdx.x] = dgp[threadIdx.x];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K6: dL/dD, torque, radius; atomics into dpos, dq, dk, dv
+// ---------------------------------------------------------------------------
+template <typename T, int L>
+__global__ void __launch_bounds__(BT) edge_bwd_kernel(Args a) {
+  constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  constexpr int P = (L + 1) * (L + 2) / 2;
+  extern __shared__ float sm[];
+  float *dvt = sm;                 // [Q][C]  dL/dv~ (unstacked)
+  float *vj = dvt + Q * a.C;       // [Q][C]
+  float *yv = vj + Q * a.C;        // [Q][C]  y = g Y (unstacked)
+  float *dz = yv + Q * a.C;        // [Q][C]  alpha G_i
+  float *qk = dz + Q * a.C;        // [2][L+1][C]  q~0, k~0
+  __shared__ float D[S], dD[S];
+  __shared__ float dsh[16], misc[32], tau[3];
+  const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
+    const int64_t e = a.ea + el;
+    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    const int j = a.col_idx[e];
+    __syncthreads();
+    for (int x = threadIdx.x; x < S; x += blockDim.x) { D[x] = a.Dm[el * S + x]; dD[x] = 0.f; }
+    if (threadIdx.x < H) dsh[threadIdx.x] = a.dsv[el * H + threadIdx.x] * a.inv_sqrt_d;
+    if (threadIdx.x < 3) tau[threadIdx.x] = 0.f;
+    __syncthreads();
+    const float *Gi = a.G + (size_t)i * QC;
+    const float *Yr = a.Y + (size_t)el * QC, *dAr = a.dA + (size_t)el * QC;
+    for (int x = threadIdx.x; x < QC; x += blockDim.x) {
+      const int q = x / C, c = x % C;
+      int l = 0;
+      while ((l + 1) * (l + 1) <= q) ++l;
+      const int m = q - l * l - l, am = m < 0 ? -m : m;
+      const int so = stack_off(L, C, m) + (l - am) * C + c;
+      dvt[x] = dAr[so];
+      vj[x] = ldf<T>(a.v, (size_t)j * QC + x);
+      yv[x] = a.gv[el * P + pair_index(L, am, l)] * Yr[so];
+      dz[x] = a.al[el * H + c / Ch] * Gi[x];
+    }
+    // q~0, k~0 (m = 0 rows of D q_i, D k_j)
+    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
+      const int l = x / C, c = x % C, w = 2 * l + 1;
+      const float *row0 = D + wig_offset(l) + l * w;
+      float qh = 0.f, kh = 0.f;
+      for (int mp = 0; mp < w; ++mp) {
+        qh = fmaf(row0[mp], ldf<T>(a.q, ((size_t)i * Q + l * l + mp) * C + c), qh);
+        kh = fmaf(row0[mp], ldf<T>(a.k, ((size_t)j * Q + l * l + mp) * C + c), kh);
+      }
+      qk[l * C + c] = qh;
+      qk[(L + 1) * C + l * C + c] = kh;
+    }
+    __syncthreads();
+    // dL/dD^l[m][m'] = sum_c dv~[m] v_j[m'] + y[m] dz[m'] (+ the m = 0 row:
+    // dq~0 q_i[m'] + dk~0 k_j[m'], dq~0 = ds k~0 / sqrt d, dk~0 = ds q~0 / sqrt d)
+    for (int ent = warp; ent < S; ent += nw) {
+      int l = 0;
+      while (wig_offset(l + 1) <= ent) ++l;
+      const int w = 2 * l + 1, rr = (ent - wig_offset(l)) / w, cc = (ent - wig_offset(l)) % w;
+      const int qa = l * l + rr, qb = l * l + cc;
+      float s = 0.f;
+      for (int c = lane; c < C; c += 32) {
+        s = fmaf(dvt[qa * C + c], vj[qb * C + c], s);
+        s = fmaf(yv[qa * C + c], dz[qb * C + c], s);
+        if (rr == l) {
+          const float ds = dsh[c / Ch];
+          s = fmaf(ds * qk[(L + 1) * C + l * C + c], ldf<T>(a.q, ((size_t)i * Q + qb) * C + c), s);
+          s = fmaf(ds * qk[l * C + c], ldf<T>(a.k, ((size_t)j * Q + qb) * C + c), s);
+        }
+      }
+      s = warp_sum(s);
+      if (lane == 0) dD[ent] = s;
+    }
+    __syncthreads();
+    // torque tau_k = -<D^T dD, J_k>, one (l, a, b) entry per thread
+    {
+      float t0 = 0.f, t1 = 0.f, t2 = 0.f;
+      for (int ent = threadIdx.x; ent < S; ent += blockDim.x) {
+        int l = 0;
+        while (wig_offset(l + 1) <= ent) ++l;
+        const int w = 2 * l + 1, ra = (ent - wig_offset(l)) / w, cb = (ent - wig_offset(l)) % w;
+        const float *Dl = D + wig_offset(l), *dDl = dD + wig_offset(l);
+        float mab = 0.f;   // (D^T dD)[ra][cb]
+        for (int m = 0; m < w; ++m) mab = fmaf(Dl[m * w + ra], dDl[m * w + cb], mab);
+        t0 = fmaf(mab, c_gen[ent], t0);
+        t1 = fmaf(mab, c_gen[JMAX + ent], t1);
+        t2 = fmaf(mab, c_gen[2 * JMAX + ent], t2);
+      }
+      t0 = warp_sum(t0); t1 = warp_sum(t1); t2 = warp_sum(t2);
+      if (lane == 0) { atomicAdd(&tau[0], -t0); atomicAdd(&tau[1], -t1); atomicAdd(&tau[2], -t2); }
+    }
+    // radial: dL/dg -> hidden -> RBF -> r, plus the envelope
+    if (warp == 0) {
+      float dr = 0.f;
+      const float r = a.rv[el * 4 + 3];
+      if (lane < 16) {
+        float dh = 0.f;
+        for (int p = 0; p < P; ++p) dh = fmaf(a.dgv[el * P + p], a.W2[p * 16 + lane], dh);
+        const float z = a.zv[el * 16 + lane], sg = 1.f / (1.f + expf(-z));
+        misc[lane] = dh * sg * (1.f + z * (1.f - sg));   // dL/dz (SiLU')
+      }
+      __syncwarp();
+      if (lane < 8) {
+        float dphi = 0.f;
+        for (int hh = 0; hh < 16; ++hh) dphi = fmaf(misc[hh], a.W1[hh * 8 + lane], dphi);
+        const float mu = (float)lane * (a.g.rc / 7.f), dd = r - mu;
+        dr = dphi * expf(-dd * dd * 2.f) * (-dd * 4.f);   // d phi / dr = -phi (r - mu) / sigma^2
+      }
+      dr = warp_sum(dr);
+      if (lane == 0) misc[16] = dr + a.duv[el] * (-0.5f * 3.14159265358979f / a.g.rc) * sinpif(r / a.g.rc);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const float dx = a.rv[el * 4 + 0], dy = a.rv[el * 4 + 1], dzz = a.rv[el * 4 + 2], r = a.rv[el * 4 + 3];
+      float gx = 0.f, gy = 0.f, gz = 0.f;
+      if (r > 0.f) {
+        const float ux = dx / r, uy = dy / r, uz = dzz / r, dr = misc[16];
+        // (tau x rhat) / r
+        gx = dr * ux + (tau[1] * uz - tau[2] * uy) / r;
+        gy = dr * uy + (tau[2] * ux - tau[0] * uz) / r;
+        gz = dr * uz + (tau[0] * uy - tau[1] * ux) / r;
+      }
+      atomicAdd(&a.dpos[3 * j + 0], gx); atomicAdd(&a.dpos[3 * j + 1], gy); atomicAdd(&a.dpos[3 * j + 2], gz);
+      atomicAdd(&a.dpos[3 * i + 0], -gx); atomicAdd(&a.dpos[3 * i + 1], -gy); atomicAdd(&a.dpos[3 * i + 2], -gz);
+    }
+    // dv_j += D^T dv~; dq_i, dk_j += row0^T dq~0 / dk~0
+    for (int x = threadIdx.x; x < QC; x += blockDim.x) {
+      const int q = x / C, c = x % C;
+      int l = 0;
+      while ((l + 1) * (l + 1) <= q) ++l;
+      const int w = 2 * l + 1, mp = q - l * l;
+      const float *Dl = D + wig_offset(l);
+      float acc = 0.f;
+      for (int m = 0; m < w; ++m) acc = fmaf(Dl[m * w + mp], dvt[(l * l + m) * C + c], acc);
+      atomicAdd(&a.dv[(size_t)j * QC + x], acc);
+      const float r0 = Dl[l * w + mp], ds = dsh[c / Ch];
+      atomicAdd(&a.dq[(size_t)i * QC + x], r0 * ds * qk[(L + 1) * C + l * C + c]);
+      atomicAdd(&a.dk[(size_t)j * QC + x], r0 * ds * qk[l * C + c]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K7: dx[n,(l,m),c] = sum_o dq[n,(l,m),o] Wq[l][o][c] + (k, v) alike
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void dx_kernel(const float *dq, const float *dk, const float *dv, const e2f_weights w, int N,
+                          float *dx) {
+  extern __shared__ float sr[];   // [3][C] rows of one (node, l, m)
+  const int L = w.L_max, C = w.C, Q = (L + 1) * (L + 1);
+  for (int64_t row = blockIdx.x; row < (int64_t)N * Q; row += gridDim.x) {
+    const int q = (int)(row % Q);
+    int l = 0;
+    while ((l + 1) * (l + 1) <= q) ++l;
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      sr[c] = dq[row * C + c];
+      sr[C + c] = dk[row * C + c];
+      sr[2 * C + c] = dv[row * C + c];
+    }
+    __syncthreads();
+    const T *Wq = static_cast<const T *>(w.Wq[l]), *Wk = static_cast<const T *>(w.Wk[l]),
+            *Wv = static_cast<const T *>(w.Wv[l]);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float acc = 0.f;
+      for (int o = 0; o < C; ++o) {
+        acc = fmaf(sr[o], to_f(Wq[(size_t)o * C + c]), acc);
+        acc = fmaf(sr[C + o], to_f(Wk[(size_t)o * C + c]), acc);
+        acc = fmaf(sr[2 * C + o], to_f(Wv[(size_t)o * C + c]), acc);
+      }
+      dx[row * C + c] = acc;
+    }
+  }
+}
+
+// Wc_m = [[Wr, -Wi], [Wi, Wr]] (2n x 2n, row-major), m >= 1
+template <typename T>
+__global__ void complex_block_kernel(const T *Wr, const T *Wi, int n, T *out) {
+  const int64_t tot = 4LL * n * n;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < tot; x += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(x / (2 * n)), c = (int)(x % (2 * n));
+    const int rb = r / n, cb = c / n, ri = r % n, ci = c % n;
+    const float vr = to_f(Wr[(size_t)ri * n + ci]), vi = to_f(Wi[(size_t)ri * n + ci]);
+    float v;
+    if (rb == 0) v = (cb == 0) ? vr : -vi;
+    else v = (cb == 0) ? vi : vr;
+    out[x] = from_f<T>(v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host
+// ---------------------------------------------------------------------------
+static std::once_flag g_gen_once;
+static float g_gen_tab[3 * JMAX];
+static std::mutex g_gen_mu;
+static bool g_gen_up[64] = {};
+
+static void fit_generators() {
+  // J_k^l = (D(R_k(+eps)) - D(R_k(-eps))) / (2 eps), R_k(t) = exp(t K_k)
+  const double eps = 1e-5;
+  std::vector<double> Dp(JMAX), Dm(JMAX);
+  for (int k = 0; k < 3; ++k) {
+    for (int sgn = 0; sgn < 2; ++sgn) {
+      const double t = sgn ? -eps : eps, c = cos(t), s = sin(t);
+      double R[9];
+      if (k == 0) { double RR[9] = {1, 0, 0, 0, c, -s, 0, s, c}; for (int x = 0; x < 9; ++x) R[x] = RR[x]; }
+      else if (k == 1) { double RR[9] = {c, 0, s, 0, 1, 0, -s, 0, c}; for (int x = 0; x < 9; ++x) R[x] = RR[x]; }
+      else { double RR[9] = {c, -s, 0, s, c, 0, 0, 0, 1}; for (int x = 0; x < 9; ++x) R[x] = RR[x]; }
+      wig_all_serial<double>(R, E2F_MAX_L, sgn ? Dm.data() : Dp.data());
+    }
+    for (int x = 0; x < JMAX; ++x) g_gen_tab[k * JMAX + x] = (float)((Dp[x] - Dm[x]) / (2 * eps));
+  }
+}
+
+static e2f_status ensure_generators() {
+  std::call_once(g_gen_once, fit_generators);
+  int dev = 0;
+  E2F_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_gen_mu);
+  if (!g_gen_up[dev]) {
+    E2F_CUDA_TRY(cudaMemcpyToSymbol(c_gen, g_gen_tab, sizeof(g_gen_tab)));
+    g_gen_up[dev] = true;
+  }
+  return E2F_OK;
+}
+
+static std::mutex g_blas_mu;
+static cublasHandle_t g_blas[64] = {};
+
+static e2f_status blas_handle(cublasHandle_t *h, cudaStream_t s) {
+  int dev = 0;
+  E2F_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_blas_mu);
+  if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) return E2F_ERR_CUDA;
+  if (cublasSetStream(g_blas[dev], s) != CUBLAS_STATUS_SUCCESS) return E2F_ERR_CUDA;
+  *h = g_blas[dev];
+  return E2F_OK;
+}
+
+// C[E][w] (ld QC) = A[E][w] (ld QC) op(Wc): trans = true -> A Wc^T, false -> A Wc
+template <typename T>
+static e2f_status stacked_gemm(cublasHandle_t h, const T *Wc, int w, const void *A, float *Cout, int64_t E, int QC,
+                               bool trans) {
+  const float one = 1.f, zero = 0.f;
+  const cudaDataType_t dt = std::is_same<T, float>::value ? CUDA_R_32F : CUDA_R_16BF;
+  // column-major view: C^T [w x E] = op(Wc') [w x w] * A^T [w x E], with the
+  // row-major Wc seen as Wc^T
+  const cublasStatus_t st = cublasGemmEx(h, trans ? CUBLAS_OP_T : CUBLAS_OP_N, CUBLAS_OP_N, w, (int)E, w, &one, Wc, dt,
+                                         w, A, dt, QC, &zero, Cout, CUDA_R_32F, QC, CUBLAS_COMPUTE_32F,
+                                         CUBLAS_GEMM_DEFAULT);
+  return st == CUBLAS_STATUS_SUCCESS ? E2F_OK : E2F_ERR_CUDA;
+}
+
+template <typename T, int L>
+static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w, const float *G,
+                      float *dx, float *dpos, cudaStream_t s) {
+  constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
+  constexpr int P = (L + 1) * (L + 2) / 2;
+  const int C = w->C, H = w->H, QC = Q * C;
+  const int64_t N = csr->n_nodes;
+  e2f_status st = ensure_generators();
+  if (st != E2F_OK) return st;
+  cublasHandle_t bh;
+  st = blas_handle(&bh, s);
+  if (st != E2F_OK) return st;
+  auto up = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  const size_t feat = (size_t)N * QC;
+  // q, k, v and the fp32 accumulators dq, dk, dv
+  Scratch node;
+  const size_t o_qkv = 0, o_acc = up(3 * feat * sizeof(T));
+  E2F_CUDA_TRY(node.alloc(o_acc + 3 * feat * sizeof(float), s));
+  char *nb = node.as<char>();
+  T *q = reinterpret_cast<T *>(nb + o_qkv), *k = q + feat, *v = k + feat;
+  float *dq = reinterpret_cast<float *>(nb + o_acc), *dk = dq + feat, *dv = dk + feat;
+  st = project_impl(x, N, w, q, k, v, s);
+  if (st != E2F_OK) return st;
+  E2F_CUDA_TRY(cudaMemsetAsync(dq, 0, 3 * feat * sizeof(float), s));
+  E2F_CUDA_TRY(cudaMemsetAsync(dpos, 0, (size_t)N * 3 * sizeof(float), s));
+  // complex SO(2) blocks
+  std::vector<size_t> woff(L + 1);
+  size_t wtot = 0;
+  for (int m = 0; m <= L; ++m) {
+    const size_t wm = m == 0 ? (size_t)(L + 1) * C : 2 * (size_t)(L - m + 1) * C;
+    woff[m] = wtot;
+    wtot += up(wm * wm * sizeof(T)) / sizeof(T);
+  }
+  Scratch wcs;
+  E2F_CUDA_TRY(wcs.alloc(wtot * sizeof(T), s));
+  T *wc = wcs.as<T>();
+  E2F_CUDA_TRY(cudaMemcpyAsync(wc, w->W0, sizeof(T) * (size_t)(L + 1) * C * (L + 1) * C, cudaMemcpyDeviceToDevice, s));
+  for (int m = 1; m <= L; ++m) {
+    const int n = (L - m + 1) * C;
+    E2F_LAUNCH(complex_block_kernel<T>, 256, 256, 0, s, static_cast<const T *>(w->Wr[m]),
+               static_cast<const T *>(w->Wi[m]), n, wc + woff[m]);
+  }
+  // chunks of whole nodes (host copy of row_ptr: one synchronisation)
+  std::vector<int32_t> rp(N + 1);
+  E2F_CUDA_TRY(cudaMemcpyAsync(rp.data(), csr->row_ptr, sizeof(int32_t) * (N + 1), cudaMemcpyDeviceToHost, s));
+  E2F_CUDA_TRY(cudaStreamSynchronize(s));
+  int64_t maxce = 0;
+  std::vector<std::pair<int, int>> chunks;
+  for (int n0 = 0; n0 < N;) {
+    int n1 = n0 + 1;
+    while (n1 < N && (int64_t)rp[n1 + 1] - rp[n0] <= CHUNK_E) ++n1;
+    chunks.emplace_back(n0, n1);
+    maxce = std::max<int64_t>(maxce, (int64_t)rp[n1] - rp[n0]);
+    n0 = n1;
+  }
+  int64_t maxcn = 0;
+  for (auto &c : chunks) maxcn = std::max<int64_t>(maxcn, c.second - c.first);
+  const size_t ce = (size_t)std::max<int64_t>(maxce, 1), cn = (size_t)std::max<int64_t>(maxcn, 1);
+  size_t off = 0;
+  auto carve = [&](size_t bytes) { const size_t o = off; off += up(bytes); return o; };
+  const size_t oA = carve(ce * QC * sizeof(T)), odY = carve(ce * QC * sizeof(T));
+  const size_t oY = carve(ce * QC * 4), odA = carve(ce * QC * 4), oD = carve(ce * S * 4), og = carve(ce * P * 4);
+  const size_t oz = carve(ce * 16 * 4), os = carve(ce * H * 4), ou = carve(ce * 4), orr = carve(ce * 16);
+  const size_t oal = carve(ce * H * 4), odal = carve(ce * H * 4), ods = carve(ce * H * 4), odu = carve(ce * 4);
+  const size_t odg = carve(ce * P * 4), oM = carve(cn * H * 4), oden = carve(cn * H * 4), odl = carve(cn * H * 4);
+  Scratch cs;
+  E2F_CUDA_TRY(cs.alloc(off, s));
+  char *cb = cs.as<char>();
+  Args a;
+  a.L = L; a.C = C; a.H = H; a.N = (int)N;
+  a.inv_sqrt_d = 1.f / sqrtf((float)((L + 1) * (C / H)));
+  for (int kk = 0; kk < 3; ++kk) {
+    a.g.box[kk] = csr->box[kk] > 0.f ? csr->box[kk] : 0.f;
+    a.g.half[kk] = 0.5f * a.g.box[kk];
+    a.g.periodic[kk] = csr->box[kk] > 0.f;
+  }
+  a.g.rc = csr->r_c; a.g.rc2 = csr->r_c * csr->r_c;
+  a.row_ptr = csr->row_ptr; a.col_idx = csr->col_idx; a.pos = pos;
+  a.q = q; a.k = k; a.v = v; a.G = G; a.W1 = w->rad_W1; a.W2 = w->rad_W2;
+  a.A = cb + oA; a.dY = cb + odY;
+  a.Y = reinterpret_cast<float *>(cb + oY); a.dA = reinterpret_cast<float *>(cb + odA);
+  a.Dm = reinterpret_cast<float *>(cb + oD); a.gv = reinterpret_cast<float *>(cb + og);
+  a.zv = reinterpret_cast<float *>(cb + oz); a.sv = reinterpret_cast<float *>(cb + os);
+  a.uv = reinterpret_cast<float *>(cb + ou); a.rv = reinterpret_cast<float *>(cb + orr);
+  a.al = reinterpret_cast<float *>(cb + oal); a.dal = reinterpret_cast<float *>(cb + odal);
+  a.dsv = reinterpret_cast<float *>(cb + ods); a.duv = reinterpret_cast<float *>(cb + odu);
+  a.dgv = reinterpret_cast<float *>(cb + odg);
+  a.Mv = reinterpret_cast<float *>(cb + oM); a.denv = reinterpret_cast<float *>(cb + oden);
+  a.dlt = reinterpret_cast<float *>(cb + odl);
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dpos = dpos;
+  const size_t smem6 = sizeof(float) * ((size_t)4 * QC + 2 * (size_t)(L + 1) * C);
+  if (smem6 > 200 * 1024) return E2F_ERR_UNSUPPORTED;
+  E2F_CUDA_TRY(cudaFuncSetAttribute(edge_bwd_kernel<T, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem6));
+  for (auto &ch : chunks) {
+    a.na = ch.first; a.nb = ch.second;
+    a.ea = rp[ch.first];
+    a.ne = (int64_t)rp[ch.second] - rp[ch.first];
+    if (a.ne == 0) continue;
+    const int eg = (int)std::min<int64_t>(a.ne, 148LL * 16);
+    const int ng = (int)std::min<int64_t>((a.nb - a.na + 7) / 8, 148LL * 8);
+    E2F_LAUNCH((edge_fwd_kernel<T, L>), eg, BT, 0, s, a);
+    E2F_LAUNCH(node_stats_kernel, ng, 256, 0, s, a);
+    for (int m = 0; m <= L; ++m) {
+      const int wm = m == 0 ? (L + 1) * C : 2 * (L - m + 1) * C;
+      const int so = stack_off(L, C, m);
+      st = stacked_gemm<T>(bh, wc + woff[m], wm, static_cast<T *>(a.A) + so, a.Y + so, a.ne, QC, true);
+      if (st != E2F_OK) return st;
+    }
+    E2F_LAUNCH((edge_dalpha_kernel<L>), eg, BT, 0, s, a);
+    E2F_LAUNCH(node_delta_kernel, ng, 256, 0, s, a);
+    E2F_LAUNCH((edge_dy_kernel<T, L>), eg, BT, 0, s, a);
+    for (int m = 0; m <= L; ++m) {
+      const int wm = m == 0 ? (L + 1) * C : 2 * (L - m + 1) * C;
+      const int so = stack_off(L, C, m);
+      st = stacked_gemm<T>(bh, wc + woff[m], wm, static_cast<T *>(a.dY) + so, a.dA + so, a.ne, QC, false);
+      if (st != E2F_OK) return st;
+    }
+    E2F_LAUNCH((edge_bwd_kernel<T, L>), eg, BT, smem6, s, a);
+  }
+  const int rg = (int)std::min<int64_t>(N * Q, 148LL * 32);
+  E2F_LAUNCH(dx_kernel<T>, rg, 128, sizeof(float) * 3 * C, s, dq, dk, dv, *w, (int)N, dx);
+  return E2F_OK;
+}
+
+}  // namespace bwd
+
+e2f_status attention_backward_impl(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
+                                   const float *G, float *dx, float *dpos, cudaStream_t s) {
+  const bool f32 = w->dtype == E2F_F32;
+  switch (w->L_max) {
+#define E2F_BWD_CASE(LL)                                                                                   \
+  case LL:                                                                                                 \
+    return f32 ? bwd::run<float, LL>(x, pos, csr, w, G, dx, dpos, s)                                       \
+               : bwd::run<__nv_bfloat16, LL>(x, pos, csr, w, G, dx, dpos, s);
+    E2F_BWD_CASE(0)
+    E2F_BWD_CASE(1)
+    E2F_BWD_CASE(2)
+    E2F_BWD_CASE(3)
+    E2F_BWD_CASE(4)
+    E2F_BWD_CASE(5)
+    E2F_BWD_CASE(6)
+#undef E2F_BWD_CASE
+    default: return E2F_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace e2f

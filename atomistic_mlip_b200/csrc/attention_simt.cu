@@ -46,19 +46,6 @@ template <typename T> struct AttnArgs {
   float *out;
 };
 
-// offset of the stacked block for +-m inside one edge's vt row
-__host__ __device__ __forceinline__ int stack_off(int L, int C, int m) {
-  const int am = m < 0 ? -m : m;
-  if (am == 0) return 0;
-  int off = (L + 1) * C;
-  for (int t = 1; t < am; ++t) off += 2 * (L - t + 1) * C;
-  return m > 0 ? off : off + (L - am + 1) * C;
-}
-
-__host__ __device__ __forceinline__ int pair_index(int L, int m, int l) {
-  return m * (L + 1) - m * (m - 1) / 2 + (l - m);
-}
-
 template <typename T, int L>
 __global__ void __launch_bounds__(ATT_THREADS)
 attention_simt_kernel(AttnArgs<T> a) {

@@ -217,9 +217,14 @@ struct TileIter {
   int64_t ebeg, eend;
   int64_t e0, e1;
   int n0;
-  __device__ void init(int b, int G, int64_t E) {
-    nlo = b == 0 ? 0 : first_node_at(rp, N, E * (int64_t)b / G);
-    nhi = b + 1 == G ? N : first_node_at(rp, N, E * (int64_t)(b + 1) / G);
+  // node range of CTA b of G (computed once per CTA, then shared)
+  static __device__ int2 node_range(const int32_t *rp, int N, int b, int G, int64_t E) {
+    return make_int2(b == 0 ? 0 : first_node_at(rp, N, E * (int64_t)b / G),
+                     b + 1 == G ? N : first_node_at(rp, N, E * (int64_t)(b + 1) / G));
+  }
+  __device__ void init(int2 nr) {
+    nlo = nr.x;
+    nhi = nr.y;
     ebeg = rp[nlo];
     eend = rp[nhi];
   }
@@ -452,6 +457,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     for (int c = 0; c < 2; ++c) { mbar_init(&geo_full[c], 1); mbar_init(&geo_empty[c], 4); }
     mbar_init(mma_drain, 1); mbar_init(rg_drain, 1);
     *abort_flag = 0;
+    *reinterpret_cast<int2 *>(tslot + 2) = TileIter::node_range(a.row_ptr, a.N, blockIdx.x, gridDim.x, a.E);
     mbar_fence_init();
   }
   __syncthreads();
@@ -464,7 +470,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 
   TileIter ti;
   ti.rp = a.row_ptr; ti.N = a.N; ti.te = Cf::TE;
-  ti.init(blockIdx.x, gridDim.x, a.E);
+  ti.init(*reinterpret_cast<const int2 *>(tslot + 2));
   const int H = a.H, Ch = CH / H;
   const int hshift = 31 - __clz(Ch);   // Ch is a power of two
 
@@ -973,57 +979,79 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       const int *jj = g_jj(c), *nodeof = jj + TE;
       const float *csb = g_cs(c), *snb = csb + TE * (L > 0 ? L : 1);
       const __half *dy = g_dy(c);
+      // the IPH items' q and k rows (2 Q per item, 16 bytes each) are streamed
+      // through a ring of RING registers: row k + RING is loaded as soon as
+      // row k has been consumed
+      constexpr int RPI = 2 * Q;              // rows per item: (q, k) per coefficient
+      constexpr int TOT = IPH * RPI;
+      constexpr int RING = 16;
+      const __nv_bfloat16 *qr[IPH], *kr[IPH];
+      int ee[IPH];
 #pragma unroll
       for (int it = 0; it < IPH; ++it) {
         const int item = pt + half * (TE * 8) + it * 256;
         const int e = item >> 4, c0 = (item & 15) * 8;
-        float acc = 0.f;
-        if (e < ne) {
-          const int i = nodeof[e], j = jj[e];
-          const __half *d = dy + e * Cf::NDYP;
-          const __nv_bfloat16 *qr = a.q + (size_t)i * Q * CH + c0;
-          const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c0;
-          float2 accv[4];
+        ee[it] = e;
+        const int i = e < ne ? nodeof[e] : 0, j = e < ne ? jj[e] : 0;   // dead items read node 0, weight 0
+        qr[it] = a.q + (size_t)i * Q * CH + c0;
+        kr[it] = a.k + (size_t)j * Q * CH + c0;
+      }
+      auto row_addr = [&](int k) {
+        const int it = k / RPI, r = (k % RPI) >> 1;
+        return reinterpret_cast<const uint4 *>(((k & 1) ? kr[it] : qr[it]) + (size_t)r * CH);
+      };
+      uint4 ring[RING];
+#pragma unroll
+      for (int k = 0; k < RING; ++k) ring[k] = *row_addr(k);
+      auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+      float2 accv[4], qh[4], kh[4];
+      float coef = 0.f;
+#pragma unroll
+      for (int k = 0; k < TOT; ++k) {
+        const int it = k / RPI, r = (k % RPI) >> 1;
+        int l = 0;
+        while ((l + 1) * (l + 1) <= r) ++l;                 // degree of coefficient r (compile time)
+        const int tt = r - l * l, mp = tt - l, amp = mp < 0 ? -mp : mp;
+        const int e = ee[it];
+        const uint4 row = ring[k % RING];
+        if (k + RING < TOT) ring[k % RING] = *row_addr(k + RING);
+        if (k % RPI == 0) {
 #pragma unroll
           for (int x = 0; x < 4; ++x) accv[x] = make_float2(0.f, 0.f);
-          auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
-#pragma unroll
-          for (int l = 0; l <= L; ++l) {
-            uint4 qv[2 * L + 1], kv[2 * L + 1];
-#pragma unroll
-            for (int tt = 0; tt < 2 * l + 1; ++tt) {
-              qv[tt] = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + tt) * CH);
-              kv[tt] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + tt) * CH);
-            }
-            float2 qh[4], kh[4];
+        }
+        if ((k & 1) == 0) {
+          if (tt == 0) {
 #pragma unroll
             for (int x = 0; x < 4; ++x) { qh[x] = make_float2(0.f, 0.f); kh[x] = make_float2(0.f, 0.f); }
+          }
+          // m = 0 row of D^l in the edge frame (gauge-free: normalised real SH of rhat)
+          const float de = e < ne ? __half2float(dy[e * Cf::NDYP + dye_off<L>(l) + amp]) : 0.f;
+          coef = (mp == 0) ? de : (mp > 0 ? de * csb[(amp - 1) * TE + min(e, TE - 1)] : de * snb[(amp - 1) * TE + min(e, TE - 1)]);
+        }
+        const float2 c2 = make_float2(coef, coef);
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&row);
+        if ((k & 1) == 0) {
 #pragma unroll
-            for (int tt = 0; tt < 2 * l + 1; ++tt) {
-              const int mp = tt - l, amp = mp < 0 ? -mp : mp;
-              const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
-              const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[(amp - 1) * TE + e] : de * snb[(amp - 1) * TE + e]);
-              const float2 c2 = make_float2(coef, coef);
-              const uint32_t *qw = reinterpret_cast<const uint32_t *>(&qv[tt]);
-              const uint32_t *kw = reinterpret_cast<const uint32_t *>(&kv[tt]);
+          for (int x = 0; x < 4; ++x) qh[x] = __ffma2_rn(c2, pair(w[x]), qh[x]);
+        } else {
 #pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                qh[x] = __ffma2_rn(c2, pair(qw[x]), qh[x]);
-                kh[x] = __ffma2_rn(c2, pair(kw[x]), kh[x]);
-              }
-            }
+          for (int x = 0; x < 4; ++x) kh[x] = __ffma2_rn(c2, pair(w[x]), kh[x]);
+          if (tt == 2 * l) {   // degree l complete
 #pragma unroll
             for (int x = 0; x < 4; ++x) accv[x] = __ffma2_rn(qh[x], kh[x], accv[x]);
           }
+        }
+        if (k % RPI == RPI - 1) {
+          float acc = 0.f;
 #pragma unroll
           for (int x = 0; x < 4; ++x) acc += accv[x].x + accv[x].y;
+          const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
+          for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          // the softmax logit with the envelope folded in: u e^s = e^(s + log u)
+          // (the lane owning the head's first block keeps it for the
+          // statistics step)
+          sk[it] = (e < ne) ? acc * a.inv_sqrt_d + logf(geo[e * 4 + 2]) : -INFINITY;
         }
-        const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
-        for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        // the softmax logit with the envelope folded in: u e^s = e^(s + log u)
-        // (the lane owning the head's first block keeps it for the
-        // statistics step)
-        sk[it] = (e < ne) ? acc * a.inv_sqrt_d + logf(geo[e * 4 + 2]) : -INFINITY;
       }
     };
     // ---- online softmax statistics of tile g (copy c), after both logit
@@ -1154,47 +1182,54 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         #pragma unroll 1
         for (int lp = m; lp <= L; ++lp) {
           const int sp = (m == 0) ? lp : 2 * (lp - m);
-          {
-            // each producer warp waits for the unit on its own: the warps run
-            // through the units independently (a warp that finished its part
-            // of one unit starts loading for the next)
+          // each producer warp waits for the unit on its own (the warps run
+          // through the units independently); the wait comes after the first
+          // rows of the unit's gathers have been issued, so their latency
+          // overlaps it
+          auto slot_ready = [&]() -> bool {
             bool f = false;
             if (lane == 0) {
               f = !W.wait(&unit_empty[sp], ((pfillpar >> sp) & 1) ^ 1, 40);
               if (!f && m > 0) f = !W.wait(&unit_empty[sp + 1], ((pfillpar >> (sp + 1)) & 1) ^ 1, 40);
             }
             dead = __shfl_sync(0xffffffffu, (int)(f || W.aborted()), 0) != 0;
-            if (dead) break;
-          }
+            return !dead;
+          };
           // v~(+m), v~(-m) of degree l' (compile-time constant: register use
           // follows the degree) for NB (edge, 8-channel block) items of this
           // thread: block b belongs to edge ea (first half of the blocks, or
           // all of them when NEc = 1) or eb (second half), and covers
-          // channels [cbs[b], +8).  Pairs of channels go through packed fp32
-          // FMAs.  emit(b, wp, wm) receives block b as packed bf16 pairs (wp:
-          // +m, wm: -m); edges past the tile's end come out zero.
-          auto rot4 = [&](auto LPc, auto NEc, const int ea, const int eb, const auto &cbs, auto &&emit) {
+          // channels [cbs[b], +8).  The NB x (2l'+1) gathered 16-byte rows are
+          // streamed through a ring of RING registers: row k + RING is
+          // loaded as soon as row k has been consumed, so RING rows stay in
+          // flight across block and edge boundaries.  Pairs of channels go
+          // through packed fp32 FMAs.  emit(b, wp, wm) receives block b as
+          // packed bf16 pairs (wp: +m, wm: -m); edges past the tile's end
+          // come out zero.  Returns false (nothing emitted) on an abort.
+          auto rot4 = [&](auto LPc, auto NEc, const int ea, const int eb, const auto &cbs, auto &&emit) -> bool {
             constexpr int LP = decltype(LPc)::value;
             constexpr int NR = 2 * LP + 1;
             constexpr int NB = (int)(sizeof(cbs) / sizeof(int));   // blocks of this thread
             constexpr int NE = decltype(NEc)::value;               // distinct edges: 1 or 2
             constexpr int BPE = NB / NE;                           // blocks per edge
-            if constexpr (NE == 1) {
-              if (ea >= ne) {
-                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int bb = 0; bb < NB; ++bb) emit(bb, z, z);
-                return;
-              }
-            }
-            // rows of edges past the tile's end: node 0's, scaled by zero
+            constexpr int TOT = NB * NR;                           // rows of this thread
+            constexpr int RING = TOT < 16 ? TOT : 16;
+            // rows of edges past the tile's end: node 0's, scaled by zero (every
+            // lane takes the same path: slot_ready() is warp-collective)
             const __nv_bfloat16 *vra = a.v + (size_t)(ea < ne ? jj[ea] : 0) * Q * CH + (size_t)(LP * LP) * CH;
             const __nv_bfloat16 *vrb = NE == 1 ? vra : a.v + (size_t)(eb < ne ? jj[eb] : 0) * Q * CH + (size_t)(LP * LP) * CH;
+            auto row_addr = [&](int k) {
+              const int bb = k / NR, t = k % NR;
+              return reinterpret_cast<const uint4 *>((bb < BPE ? vra : vrb) + (size_t)t * CH + cbs[bb]);
+            };
+            uint4 ring[RING];
+#pragma unroll
+            for (int k = 0; k < RING; ++k) ring[k] = *row_addr(k);
+            if (!slot_ready()) return false;
             // per-edge coefficients: u+ = c v+ + s v-, u- = -s v+ + c v-, scaled
             // by the y-rotation entries of row +m (even block) / -m (odd block)
             float c0 = 0.f, app[LP > 0 ? LP : 1], apm[LP > 0 ? LP : 1], amp[LP > 0 ? LP : 1], amm[LP > 0 ? LP : 1];
-            {
-              const int e = ea;
+            auto coeffs = [&](int e) {
               const bool live = e < ne;
               const __half *d = dy + (live ? e : 0) * Cf::NDYP;
               c0 = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1)]) : 0.f;
@@ -1206,74 +1241,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
                 amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
               }
-            }
-            // two blocks of gathered rows in flight: block b + 1 is loaded
-            // while block b is computed
-            constexpr int DEPTH = 2;
-            uint4 buf[DEPTH][NR];
+            };
+            coeffs(ea);
+            auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+            float2 ap[4], am[4];
 #pragma unroll
-            for (int bb = 0; bb < DEPTH - 1; ++bb)
+            for (int k = 0; k < TOT; ++k) {
+              const int bb = k / NR, t = k % NR, mp = t - LP;
+              if (NE == 2 && t == 0 && bb == BPE) coeffs(eb);
+              const uint4 row = ring[k % RING];
+              if (k + RING < TOT) ring[k % RING] = *row_addr(k + RING);
+              const uint32_t *wv = reinterpret_cast<const uint32_t *>(&row);
+              if (t == 0) {
 #pragma unroll
-              for (int t = 0; t < NR; ++t) buf[bb][t] = *reinterpret_cast<const uint4 *>((bb < BPE ? vra : vrb) + (size_t)t * CH + cbs[bb]);
-#pragma unroll
-            for (int bb = 0; bb < NB; ++bb) {
-              if (bb > 0 && bb % BPE == 0)   // next edge
-              {
-                const int e = eb;
-                const bool live = e < ne;
-                const __half *d = dy + (live ? e : 0) * Cf::NDYP;
-                c0 = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1)]) : 0.f;
-#pragma unroll
-                for (int kq = 1; kq <= LP; ++kq) {
-                  const float ck = csb[(kq - 1) * TE + e], sk = snb[(kq - 1) * TE + e];
-                  const float de = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]) : 0.f;
-                  const float dd = (live && m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
-                  app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
-                  amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
-                }
+                for (int x = 0; x < 4; ++x) { ap[x] = make_float2(0.f, 0.f); am[x] = make_float2(0.f, 0.f); }
               }
-              if (bb + DEPTH - 1 < NB) {
-                const int nb = bb + DEPTH - 1 < NB ? bb + DEPTH - 1 : 0;
+              if (mp == 0) {
+                const float2 cc = make_float2(c0, c0);
 #pragma unroll
-                for (int t = 0; t < NR; ++t)
-                  buf[(bb + DEPTH - 1) % DEPTH][t] = *reinterpret_cast<const uint4 *>((nb < BPE ? vra : vrb) + (size_t)t * CH + cbs[nb]);
-              }
-              const uint4 *rb = buf[bb % DEPTH];
-              auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
-              float2 ap[4], am[4];
-              {
-                const uint32_t *w0 = reinterpret_cast<const uint32_t *>(&rb[LP]);
+                for (int x = 0; x < 4; ++x) ap[x] = __ffma2_rn(cc, pair(wv[x]), ap[x]);
+              } else {
+                const int kq = mp > 0 ? mp : -mp;
+                const float2 cp = mp > 0 ? make_float2(app[kq - 1], app[kq - 1]) : make_float2(apm[kq - 1], apm[kq - 1]);
+                const float2 cm = mp > 0 ? make_float2(amp[kq - 1], amp[kq - 1]) : make_float2(amm[kq - 1], amm[kq - 1]);
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
-                  const float2 v0 = pair(w0[x]);
-                  ap[x] = make_float2(c0 * v0.x, c0 * v0.y);
-                  am[x] = make_float2(0.f, 0.f);
+                  const float2 v2 = pair(wv[x]);
+                  ap[x] = __ffma2_rn(cp, v2, ap[x]);
+                  am[x] = __ffma2_rn(cm, v2, am[x]);
                 }
               }
-#pragma unroll
-              for (int kq = 1; kq <= LP; ++kq) {
-                const uint32_t *wpv = reinterpret_cast<const uint32_t *>(&rb[LP + kq]);
-                const uint32_t *wnv = reinterpret_cast<const uint32_t *>(&rb[LP - kq]);
-                const float2 cpp = make_float2(app[kq - 1], app[kq - 1]), cpm = make_float2(apm[kq - 1], apm[kq - 1]);
-                const float2 cmp = make_float2(amp[kq - 1], amp[kq - 1]), cmm = make_float2(amm[kq - 1], amm[kq - 1]);
+              if (t == NR - 1) {
+                uint4 wp, wm;
+                uint32_t *pp = reinterpret_cast<uint32_t *>(&wp), *pm = reinterpret_cast<uint32_t *>(&wm);
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
-                  const float2 vp2 = pair(wpv[x]), vn2 = pair(wnv[x]);
-                  ap[x] = __ffma2_rn(cpp, vp2, __ffma2_rn(cpm, vn2, ap[x]));
-                  am[x] = __ffma2_rn(cmp, vp2, __ffma2_rn(cmm, vn2, am[x]));
+                  const __nv_bfloat162 hp = __floats2bfloat162_rn(ap[x].x, ap[x].y);
+                  const __nv_bfloat162 hm = __floats2bfloat162_rn(am[x].x, am[x].y);
+                  pp[x] = *reinterpret_cast<const uint32_t *>(&hp);
+                  pm[x] = *reinterpret_cast<const uint32_t *>(&hm);
                 }
+                emit(bb, wp, wm);
               }
-              uint4 wp, wm;
-              uint32_t *pp = reinterpret_cast<uint32_t *>(&wp), *pm = reinterpret_cast<uint32_t *>(&wm);
-#pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                const __nv_bfloat162 hp = __floats2bfloat162_rn(ap[x].x, ap[x].y);
-                const __nv_bfloat162 hm = __floats2bfloat162_rn(am[x].x, am[x].y);
-                pp[x] = *reinterpret_cast<const uint32_t *>(&hp);
-                pm[x] = *reinterpret_cast<const uint32_t *>(&hm);
-              }
-              emit(bb, wp, wm);
             }
+            return true;
           };
           if (Cf::TMU && sp >= Cf::NSU) {
             if constexpr (Cf::TMU) {
@@ -1296,6 +1307,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 for (int i = 0; i < 4; ++i) { wpl[4 * bb + i] = pp[i]; wmi[4 * bb + i] = pm[i]; }
               });
             }
+            if (dead) break;
             uint32_t opl[16], omi[16];   // the partner half's block
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -1348,6 +1360,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               case 5: if constexpr (L >= 5) fill(std::integral_constant<int, (L >= 5 ? 5 : 0)>{}); break;
               default: if constexpr (L >= 6) fill(std::integral_constant<int, (L >= 6 ? 6 : 0)>{}); break;
             }
+            if (dead) break;
           }
           fence_async_smem();
           __syncwarp();

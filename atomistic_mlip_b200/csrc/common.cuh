@@ -102,6 +102,23 @@ __device__ __forceinline__ float pair_r2(float dx, float dy, float dz) {
   return __fadd_rn(__fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy)), __fmul_rn(dz, dz));
 }
 
+// SO(2)-stacked order of one edge's rotated features: the entries of degree
+// +-m for l = |m|..L, l-major then channel; m = 0 first, then (+m, -m) for
+// m = 1..L.  Offset of the block of +-m:
+__host__ __device__ __forceinline__ int stack_off(int L, int C, int m) {
+  const int am = m < 0 ? -m : m;
+  if (am == 0) return 0;
+  int off = (L + 1) * C;
+  for (int t = 1; t < am; ++t) off += 2 * (L - t + 1) * C;
+  return m > 0 ? off : off + (L - am + 1) * C;
+}
+
+// Index of the radial output g_{m,l}: (m, l) pairs in the order m = 0..L,
+// then l = m..L.
+__host__ __device__ __forceinline__ int pair_index(int L, int m, int l) {
+  return m * (L + 1) - m * (m - 1) / 2 + (l - m);
+}
+
 __device__ __forceinline__ float3 load_pos(const float *pos, int i) {
   return make_float3(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2]);
 }

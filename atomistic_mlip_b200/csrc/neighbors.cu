@@ -133,42 +133,54 @@ struct Stencil {
   float sh[27][3];      // per-cell shift (fast path)
 };
 
-// Stencil of home cell cid: done by thread 0 into shared memory.
+// Stencil of home cell cid into shared memory, by warp 0: lane q < 27 takes
+// stencil offset q (dx fastest), the cells that exist are compacted in lane
+// order with a ballot, and the candidate offsets are a warp prefix sum.
 __device__ void make_stencil(int cid, const CellGrid &cg, const Geom &g, const int32_t *__restrict__ cell_start,
-                             Stencil &st) {
+                             Stencil &st, int lane) {
   const int c0[3] = {cid % cg.nc[0], (cid / cg.nc[0]) % cg.nc[1], cid / (cg.nc[0] * cg.nc[1])};
-  int n = 0, tot = 0;
-  for (int dz = -1; dz <= 1; ++dz)
-    for (int dy = -1; dy <= 1; ++dy)
-      for (int dx = -1; dx <= 1; ++dx) {
-        const int d[3] = {dx, dy, dz};
-        int cc[3];
-        float shv[3];
-        bool ok = true;
-        for (int k = 0; k < 3; ++k) {
-          if (d[k] != 0 && cg.stencil[k] == 0) { ok = false; break; }
-          int v = c0[k] + d[k];
-          shv[k] = 0.f;
-          if (g.periodic[k]) {
-            if (v < 0) { v += cg.nc[k]; shv[k] = -g.box[k]; }          // p_j near b, p_i near 0: d > b/2
-            else if (v >= cg.nc[k]) { v -= cg.nc[k]; shv[k] = g.box[k]; }  // d < -b/2
-          } else if (v < 0 || v >= cg.nc[k]) {
-            ok = false;
-            break;
-          }
-          cc[k] = v;
-        }
-        if (!ok) continue;
-        const int c = cc[0] + cg.nc[0] * (cc[1] + cg.nc[1] * cc[2]);
-        st.start[n] = cell_start[c];
-        st.cnt[n] = cell_start[c + 1] - st.start[n];
-        st.off[n] = tot;
-        st.sh[n][0] = shv[0]; st.sh[n][1] = shv[1]; st.sh[n][2] = shv[2];
-        tot += st.cnt[n];
-        ++n;
+  bool ok = lane < 27;
+  int cc[3] = {0, 0, 0};
+  float shv[3] = {0.f, 0.f, 0.f};
+  if (ok) {
+    const int d[3] = {lane % 3 - 1, (lane / 3) % 3 - 1, lane / 9 - 1};
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      if (d[k] != 0 && cg.stencil[k] == 0) ok = false;
+      int v = c0[k] + d[k];
+      if (g.periodic[k]) {
+        if (v < 0) { v += cg.nc[k]; shv[k] = -g.box[k]; }            // p_j near b, p_i near 0: d > b/2
+        else if (v >= cg.nc[k]) { v -= cg.nc[k]; shv[k] = g.box[k]; }  // d < -b/2
+      } else if (v < 0 || v >= cg.nc[k]) {
+        ok = false;
       }
-  st.off[n] = tot;
-  st.n = n;
+      cc[k] = v;
+    }
+  }
+  int start = 0, cnt = 0;
+  if (ok) {
+    const int c = cc[0] + cg.nc[0] * (cc[1] + cg.nc[1] * cc[2]);
+    start = cell_start[c];
+    cnt = cell_start[c + 1] - start;
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, ok);
+  const int slot = __popc(m & ((1u << lane) - 1u));
+  int incl = cnt;   // inclusive prefix of cnt over lanes (zero for lanes that are not cells)
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (ok) {
+    st.start[slot] = start;
+    st.cnt[slot] = cnt;
+    st.off[slot] = incl - cnt;
+    st.sh[slot][0] = shv[0]; st.sh[slot][1] = shv[1]; st.sh[slot][2] = shv[2];
+  }
+  if (lane == 31) {
+    st.n = __popc(m);
+    st.off[__popc(m)] = incl;
+  }
 }
 
 // Candidates [c0, c0 + nc) of the stencil into shared memory.
@@ -176,8 +188,12 @@ __device__ __forceinline__ void stage_candidates(const Stencil &st, int c0, int 
                                                  float4 *cp, float4 *cs) {
   for (int k = threadIdx.x; k < nc; k += blockDim.x) {
     const int q = c0 + k;
-    int s = 0;
-    while (st.off[s + 1] <= q) ++s;
+    int s = 0, hi = st.n - 1;   // last stencil cell with off <= q
+    while (s < hi) {
+      const int mid = (s + hi + 1) >> 1;
+      if (st.off[mid] <= q) s = mid;
+      else hi = mid - 1;
+    }
     cp[k] = spos[st.start[s] + (q - st.off[s])];
     cs[k] = make_float4(st.sh[s][0], st.sh[s][1], st.sh[s][2], 0.f);
   }
@@ -209,7 +225,7 @@ __global__ void __launch_bounds__(CELL_THREADS) cell_count_kernel(int ncell, Cel
     const int h0 = cell_start[cid], hn = cell_start[cid + 1] - h0;
     if (hn == 0) continue;   // uniform across the block
     __syncthreads();
-    if (threadIdx.x == 0) make_stencil(cid, cg, g, cell_start, st);
+    if (wid == 0) make_stencil(cid, cg, g, cell_start, st, lane);
     __syncthreads();
     const int ntot = st.off[st.n];
     // home atoms handled by this warp: counts kept per lane slot
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(CELL_THREADS) cell_fill_kernel(int ncell, Cell
     const int h0 = cell_start[cid], hn = cell_start[cid + 1] - h0;
     if (hn == 0) continue;
     __syncthreads();
-    if (threadIdx.x == 0) make_stencil(cid, cg, g, cell_start, st);
+    if (wid == 0) make_stencil(cid, cg, g, cell_start, st, lane);
     __syncthreads();
     const int ntot = st.off[st.n];
     if (ntot <= CAND_CAP) {
@@ -473,44 +489,50 @@ e2f_status build_neighbors_impl(const float *pos, int64_t N, const float *box, f
       if (!g.periodic[k]) cs[k] *= 1.25;
   }
 
-  Scratch cell_of, cnt, cstart, cursor, deg, flag, scan_tmp, spos;
-  E2F_CUDA_TRY(cell_of.alloc(sizeof(int32_t) * n, s));
-  E2F_CUDA_TRY(cnt.alloc(sizeof(int32_t) * ncell, s));
-  E2F_CUDA_TRY(cstart.alloc(sizeof(int32_t) * (ncell + 1), s));
-  E2F_CUDA_TRY(cursor.alloc(sizeof(int32_t) * ncell, s));
-  E2F_CUDA_TRY(spos.alloc(sizeof(float4) * n, s));
-  E2F_CUDA_TRY(deg.alloc(sizeof(int32_t) * n, s));
-  E2F_CUDA_TRY(flag.alloc(sizeof(int32_t) * 4, s));
-  E2F_CUDA_TRY(scan_tmp.alloc(std::max(scan_scratch_bytes(ncell), scan_scratch_bytes(n)), s));
-  E2F_CUDA_TRY(cudaMemsetAsync(cnt.p, 0, sizeof(int32_t) * ncell, s));
-  E2F_CUDA_TRY(cudaMemsetAsync(cursor.p, 0, sizeof(int32_t) * ncell, s));
-  E2F_CUDA_TRY(cudaMemsetAsync(flag.p, 0, sizeof(int32_t) * 4, s));
+  // one pool allocation, carved into 256-byte aligned pieces; the counters
+  // that must start at zero are adjacent and cleared by one memset
+  auto up = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  const size_t o_cnt = 0, o_cursor = up(sizeof(int32_t) * ncell), o_flag = o_cursor + up(sizeof(int32_t) * ncell);
+  const size_t zero_bytes = o_flag + 16;
+  const size_t o_cstart = up(zero_bytes), o_cell_of = o_cstart + up(sizeof(int32_t) * (ncell + 1));
+  const size_t o_deg = o_cell_of + up(sizeof(int32_t) * n), o_scan = o_deg + up(sizeof(int32_t) * n);
+  const size_t o_spos = o_scan + up(std::max(scan_scratch_bytes(ncell), scan_scratch_bytes(n)));
+  const size_t total_bytes = o_spos + sizeof(float4) * n;
+  Scratch ws;
+  E2F_CUDA_TRY(ws.alloc(total_bytes, s));
+  char *wb = ws.as<char>();
+  int32_t *cnt = reinterpret_cast<int32_t *>(wb + o_cnt), *cursor = reinterpret_cast<int32_t *>(wb + o_cursor);
+  int32_t *flag = reinterpret_cast<int32_t *>(wb + o_flag), *cstart = reinterpret_cast<int32_t *>(wb + o_cstart);
+  int32_t *cell_of = reinterpret_cast<int32_t *>(wb + o_cell_of), *deg = reinterpret_cast<int32_t *>(wb + o_deg);
+  void *scan_tmp = wb + o_scan;
+  float4 *spos = reinterpret_cast<float4 *>(wb + o_spos);
+  E2F_CUDA_TRY(cudaMemsetAsync(wb, 0, zero_bytes, s));
 
   const int tb = 256;
-  E2F_LAUNCH(cell_assign_kernel, (n + tb - 1) / tb, tb, 0, s, pos, n, cg, g, cell_of.as<int32_t>(),
-             cnt.as<int32_t>(), flag.as<int32_t>());
-  e2f_status st = exclusive_scan(cnt.as<int32_t>(), ncell, cstart.as<int32_t>(), scan_tmp.p, s, nullptr);
+  E2F_LAUNCH(cell_assign_kernel, (n + tb - 1) / tb, tb, 0, s, pos, n, cg, g, cell_of,
+             cnt, flag);
+  e2f_status st = exclusive_scan(cnt, ncell, cstart, scan_tmp, s, nullptr);
   if (st != E2F_OK) return st;
-  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, pos, cell_of.as<int32_t>(), n,
-             cstart.as<int32_t>(), cursor.as<int32_t>(), spos.as<float4>());
-  st = launch_count(ncell, cg, g, cstart.as<int32_t>(), spos.as<float4>(), deg.as<int32_t>(), s);
+  E2F_LAUNCH(cell_scatter_kernel, (n + tb - 1) / tb, tb, 0, s, pos, cell_of, n,
+             cstart, cursor, spos);
+  st = launch_count(ncell, cg, g, cstart, spos, deg, s);
   if (st != E2F_OK) return st;
   long long *total = nullptr;
-  st = exclusive_scan(deg.as<int32_t>(), n, row_ptr, scan_tmp.p, s, &total);
+  st = exclusive_scan(deg, n, row_ptr, scan_tmp, s, &total);
   if (st != E2F_OK) return st;
 
   // E and the domain flag (host sync 2)
   long long E = 0;
   int32_t dom = 0;
   E2F_CUDA_TRY(cudaMemcpyAsync(&E, total, sizeof(long long), cudaMemcpyDeviceToHost, s));
-  E2F_CUDA_TRY(cudaMemcpyAsync(&dom, flag.p, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  E2F_CUDA_TRY(cudaMemcpyAsync(&dom, flag, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
   E2F_CUDA_TRY(cudaStreamSynchronize(s));
   *n_edges = E;
   if (dom) return E2F_ERR_DOMAIN;
   if (E > INT32_MAX) return E2F_ERR_UNSUPPORTED;
   if (E > capacity) return E2F_ERR_CAPACITY;
   if (E > 0) {
-    st = launch_fill(ncell, cg, g, cstart.as<int32_t>(), spos.as<float4>(), row_ptr, col_idx, s);
+    st = launch_fill(ncell, cg, g, cstart, spos, row_ptr, col_idx, s);
     if (st != E2F_OK) return st;
   }
   return E2F_OK;

@@ -46,6 +46,11 @@ class Weights(ctypes.Structure):
                 ("rad_W1", ctypes.c_void_p), ("rad_W2", ctypes.c_void_p)]
 
 
+class BlockWeights(ctypes.Structure):
+    _fields_ = [("attn", Weights), ("hidden", ctypes.c_int32), ("gamma1", ctypes.c_void_p),
+                ("gamma2", ctypes.c_void_p), ("Wa", ctypes.c_void_p), ("Wb", _P7), ("Wd", _P7)]
+
+
 # name -> (restype, argtypes); must match include/e2f.h
 SIGNATURES = {
     "e2f_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
@@ -60,6 +65,11 @@ SIGNATURES = {
                                                      ctypes.POINTER(Csr), ctypes.c_void_p]),
     "e2f_attention_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
                                                ctypes.POINTER(Weights), ctypes.c_void_p, ctypes.c_void_p]),
+    "e2f_attention_backward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
+                                                ctypes.POINTER(Weights), ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p]),
+    "e2f_block_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
+                                           ctypes.POINTER(BlockWeights), ctypes.c_void_p, ctypes.c_void_p]),
     "e2f_stream_status": (ctypes.c_int32, [ctypes.c_void_p]),
     "e2f_wigner_d": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
                                       ctypes.c_void_p]),
@@ -226,6 +236,77 @@ def attention_forward(x, pos, nl: NeighborList, w: DeviceWeights, out=None, stre
                                        _ptr(out), _stream_ptr(stream))
     _check(code, "e2f_attention_forward")
     return out
+
+
+class DeviceBlockWeights:
+    """Device copies of one block's weights (attention + merged norms + FFN)
+    and the e2f_block_weights struct."""
+
+    def __init__(self, attn: DeviceWeights, gamma1, gamma2, Wa, Wb: List, Wd: List):
+        self.attn = attn
+        self.tensors = dict(gamma1=gamma1, gamma2=gamma2, Wa=Wa, Wb=Wb, Wd=Wd)
+        b = BlockWeights()
+        b.attn = attn.struct
+        b.hidden = int(Wa.shape[0])
+        b.gamma1, b.gamma2, b.Wa = gamma1.data_ptr(), gamma2.data_ptr(), Wa.data_ptr()
+        for l in range(attn.L + 1):
+            b.Wb[l], b.Wd[l] = Wb[l].data_ptr(), Wd[l].data_ptr()
+        self.struct = b
+
+    @classmethod
+    def from_layer(cls, lw: dict, device="cuda", dtype: Optional[str] = None) -> "DeviceBlockWeights":
+        """From a layer-weights dict (atomistic_mlip_b200.workloads.make_layer_weights)."""
+        torch = _torch()
+        prec = dtype or lw["precision"]
+        td = torch.float32 if prec == "fp32" else torch.bfloat16
+
+        def up(a, t=td):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=t)
+
+        L = lw["L"]
+        attn = DeviceWeights(L, lw["C"], lw["H"], F32 if prec == "fp32" else BF16,
+                             [up(a) for a in lw["Wq"]], [up(a) for a in lw["Wk"]], [up(a) for a in lw["Wv"]],
+                             up(lw["W0"]), [None] + [up(a) for a in lw["Wr"][1:]],
+                             [None] + [up(a) for a in lw["Wi"][1:]], up(lw["rad_W1"], torch.float32),
+                             up(lw["rad_W2"], torch.float32))
+        return cls(attn, up(lw["gamma1"], torch.float32), up(lw["gamma2"], torch.float32), up(lw["Wa"]),
+                   [up(a) for a in lw["Wb"]], [up(a) for a in lw["Wd"]])
+
+
+def block_forward(x, pos, nl: NeighborList, bw: DeviceBlockWeights, out=None, stream=None):
+    """One E2Former-V2 block on the fp32 residual stream x [N, Q, C]."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty_like(x)
+    csr = nl.csr()
+    code = lib().e2f_block_forward(_ptr(x), _ptr(pos), ctypes.byref(csr), ctypes.byref(bw.struct), _ptr(out),
+                                   _stream_ptr(stream))
+    _check(code, "e2f_block_forward")
+    return out
+
+
+def model_forward(x, pos, nl: NeighborList, layers: List[DeviceBlockWeights], stream=None):
+    """Blocks in turn; two ping-pong buffers for the residual stream."""
+    torch = _torch()
+    a, b = x, torch.empty_like(x)
+    for i, bw in enumerate(layers):
+        block_forward(a, pos, nl, bw, out=b, stream=stream)
+        a, b = b, (torch.empty_like(x) if i == 0 else a)
+    return a
+
+
+def attention_backward(x, pos, nl: NeighborList, w: DeviceWeights, grad_out, stream=None):
+    """(dL/dx, dL/dpos) for L = sum(grad_out * attention_forward(x, pos, nl, w));
+    the forces of an energy are -dL/dpos."""
+    torch = _torch()
+    N = int(pos.shape[0])
+    gx = torch.empty(grad_out.shape, dtype=torch.float32, device=pos.device)
+    gp = torch.empty((N, 3), dtype=torch.float32, device=pos.device)
+    csr = nl.csr()
+    code = lib().e2f_attention_backward(_ptr(x), _ptr(pos), ctypes.byref(csr), ctypes.byref(w.struct),
+                                        _ptr(grad_out), _ptr(gx), _ptr(gp), _stream_ptr(stream))
+    _check(code, "e2f_attention_backward")
+    return gx, gp
 
 
 def project_qkv(x, w: DeviceWeights, stream=None):

@@ -280,6 +280,87 @@ def measure_workload(cfg, dev, peaks, peak_src, reps=5, warm=2, n_target=None, w
     return res
 
 
+def measure_forces(cfg, dev, peaks, reps=3, warm=1, wl=None):
+    """The backward of the attention (dL/dx and dL/dpos, forces = -dL/dpos)
+    on a workload: whole-call time (CUDA events), edges/s, and the SO(2)
+    block products it recomputes and transposes (2 F(L, C) FLOP per edge)
+    as achieved TFLOP/s against the bf16 peak."""
+    import torch
+    from atomistic_mlip_b200 import e2f
+    from atomistic_mlip_b200 import workloads as w
+    stream = torch.cuda.current_stream(dev)
+    if wl is None:
+        wl = w.make_workload(cfg)
+    pos = torch.from_numpy(wl.pos).to(dev)
+    x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+    dw = e2f.DeviceWeights.from_workload(wl, dev)
+    nl = e2f.build_neighbors(pos, _box_list(wl), wl.r_c)
+    G = torch.randn((wl.N, (wl.L + 1) ** 2, wl.C), dtype=torch.float32, device=dev,
+                    generator=torch.Generator(device=dev).manual_seed(7))
+    for _ in range(warm):
+        e2f.attention_backward(x, pos, nl, dw, G)
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        _, gp = e2f.attention_backward(x, pos, nl, dw, G)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    t = statistics.median(ts)
+    F2 = 2 * so2_flops_per_edge(wl.L, wl.C)
+    res = {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}"), "N": wl.N, "E": nl.n_edges, "ms": t,
+           "edges_per_s": nl.n_edges / (t * 1e-3),
+           "so2_tflops": F2 * nl.n_edges / (t * 1e-3) / 1e12,
+           "frac_of_bf16_peak": F2 * nl.n_edges / (t * 1e-3) / 1e12 / float(peaks["bf16_tflops"]),
+           "net_force_over_max": float(gp.sum(0).abs().max() / gp.abs().max().clamp_min(1e-30)),
+           "what": "e2f_attention_backward: dL/dx and dL/dpos (forces = -dL/dpos), bf16 storage"}
+    del x, pos, dw, nl, G, gp
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_block(cfg, dev, n_layers=1, reps=3, warm=1, wl=None):
+    """n_layers E2Former-V2 blocks (merged RMS norm, attention, scalar-gated
+    FFN with Hd = 4C, residuals) on a workload: time per block, and the
+    attention kernel's share of it."""
+    import torch
+    from atomistic_mlip_b200 import e2f
+    from atomistic_mlip_b200 import workloads as w
+    stream = torch.cuda.current_stream(dev)
+    if wl is None:
+        wl = w.make_workload(cfg)
+    pos = torch.from_numpy(wl.pos).to(dev)
+    x = torch.from_numpy(np.ascontiguousarray(wl.x, np.float32)).to(dev)
+    nl = e2f.build_neighbors(pos, _box_list(wl), wl.r_c)
+    layers = [e2f.DeviceBlockWeights.from_layer(w.make_layer_weights(wl.L, wl.C, wl.H, "bf16", 900 + k), dev)
+              for k in range(n_layers)]
+    for _ in range(warm):
+        e2f.model_forward(x, pos, nl, layers)
+    e2f.profile_enable(True)
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2f.model_forward(x, pos, nl, layers)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    e2f.profile_enable(False)
+    n_k, k_ms = e2f.profile_read()
+    t = statistics.median(ts)
+    Q = (wl.L + 1) ** 2
+    ffn_flops = 2 * wl.N * wl.C * 4 * wl.C * (1 + 2 * Q)   # gate + up (all rows) + down
+    res = {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}"), "N": wl.N, "E": nl.n_edges, "layers": n_layers,
+           "ms_per_forward": t, "ms_per_block": t / n_layers,
+           "attention_kernel_share": (k_ms / max(n_k, 1)) * n_layers / t,
+           "node_updates_per_s": wl.N * n_layers / (t * 1e-3), "ffn_flops_per_block": ffn_flops,
+           "what": "e2f_block_forward x layers: Norm -> attention -> residual -> Norm -> FFN(Hd = 4C) -> residual, bf16"}
+    del x, pos, nl, layers
+    torch.cuda.empty_cache()
+    return res
+
+
 def linear_fit(ns, ys):
     """Least-squares y = a + b N and its R^2."""
     A = np.stack([np.ones(len(ns)), np.asarray(ns, float)], 1)
@@ -399,6 +480,8 @@ def run_ours(args):
         ns = [r["N"] for r in sweep]
         tot = [r["peak_device_bytes"]["torch"] + r["peak_device_bytes"]["library_scratch"] for r in sweep]
         extras["workloads"] = rows + [sweep[-1]]
+        extras["forces"] = [measure_forces(2, dev, peaks), measure_forces(4, dev, peaks, reps=2, wl=wl)]
+        extras["block"] = [measure_block(4, dev, n_layers=1, wl=wl), measure_block(2, dev, n_layers=2)]
         extras["memory_sweep"] = {
             "N": ns, "peak_device_bytes": tot,
             "edges_per_s": [r["attention"]["edges_per_s"] for r in sweep],

@@ -194,6 +194,64 @@ E2F_API e2f_status e2f_attention_forward(const void *x, const float *pos, const 
                                  const e2f_weights *w, float *out, void *stream);
 
 /*
+ * e2f_attention_backward -- gradients of L = sum(grad_out * o), o the
+ * output of e2f_attention_forward for the same x, pos, csr and w, with
+ * respect to the node features and the positions.  The conservative forces
+ * of an energy are -grad_pos ("E2Former-V2 ..." §4, the conservative
+ * variant; "DPA4 ..." §2.2, the energy-to-force path).  Weight gradients
+ * (training) are not computed.
+ *
+ *   x         device, [N][Q][C] in w->dtype (as for the forward).
+ *   grad_out  device fp32 [N][Q][C]: dL/do.
+ *   grad_x    device fp32 [N][Q][C], fully overwritten: dL/dx.
+ *   grad_pos  device fp32 [N][3], fully overwritten: dL/dpos.
+ * Requires H <= 16.  Per-edge quantities are recomputed in chunks of whole
+ * destination nodes (at most 65,536 edges each) in library scratch; the
+ * SO(2) block products of the forward recompute and their transposes run
+ * as dense GEMMs over a chunk's edges (cuBLAS, fp32 accumulation).  One
+ * host synchronisation (the chunk plan reads row_ptr).  Gradients reach
+ * grad_pos through fp32 atomics, so their summation order (and last bits)
+ * can vary from run to run.
+ */
+E2F_API e2f_status e2f_attention_backward(const void *x, const float *pos, const e2f_csr *csr,
+                                          const e2f_weights *w, const float *grad_out, float *grad_x,
+                                          float *grad_pos, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * The E2Former-V2 block around the attention.
+ * --------------------------------------------------------------------------*/
+typedef struct e2f_block_weights {
+  e2f_weights attn;          /* the block's attention weights (L_max, C, H, dtype) */
+  int32_t hidden;            /* Hd, FFN hidden width */
+  const float *gamma1;       /* device fp32 [L+1][C]: gains of the first merged norm */
+  const float *gamma2;       /* device fp32 [L+1][C]: gains of the second merged norm */
+  const void *Wa;            /* device [Hd][C] (attn.dtype): the scalar gate's map */
+  const void *Wb[E2F_MAX_L + 1];   /* device [Hd][C] per degree l = 0..L_max */
+  const void *Wd[E2F_MAX_L + 1];   /* device [C][Hd] per degree l = 0..L_max */
+} e2f_block_weights;
+
+/*
+ * e2f_block_forward -- one pre-norm residual block:
+ *   x1 = x + Attn(Norm1(x)),  out = x1 + FFN(Norm2(x1)).
+ * Norm is the merged equivariant RMS layer norm ("EquiformerV3 ..." §2B.1:
+ * one RMS statistic shared by all degrees): Norm(x)[n,(l,m),c] =
+ * gamma[l][c] x[n,(l,m),c] / sqrt(mean_{l,m,c} x[n]^2 + 1e-6).  FFN is the
+ * node feed-forward network with a scalar gate (§2B.2 hidden width, §2C
+ * gate on the l = 0 features): FFN(y)[n,(l,m)] =
+ * Wd[l] (SiLU(Wa y[n,(0,0)]) * (Wb[l] y[n,(l,m)])).  Attn is
+ * e2f_attention_forward with w->attn, on the normalised features stored in
+ * w->attn.dtype.
+ *
+ *   x    device fp32 [N][Q][C], the residual stream in.
+ *   out  device fp32 [N][Q][C], fully overwritten; must not be x.
+ * Library scratch (stream-ordered pool): the normalised features, the
+ * attention output, the gate [N][Hd] fp32 and the hidden features
+ * [N][Q][Hd] in w->attn.dtype.  Fully asynchronous.
+ */
+E2F_API e2f_status e2f_block_forward(const float *x, const float *pos, const e2f_csr *csr,
+                                     const e2f_block_weights *w, float *out, void *stream);
+
+/*
  * e2f_stream_status -- synchronise `stream`, then return (and clear) any
  * error latched by a kernel of this library on the current device
  * (E2F_ERR_TIMEOUT for a bounded wait that gave up), or E2F_ERR_CUDA.

@@ -467,19 +467,47 @@ __global__ void __launch_bounds__(BT) edge_bwd_kernel(Args a) {
       atomicAdd(&a.dpos[3 * j + 0], gx); atomicAdd(&a.dpos[3 * j + 1], gy); atomicAdd(&a.dpos[3 * j + 2], gz);
       atomicAdd(&a.dpos[3 * i + 0], -gx); atomicAdd(&a.dpos[3 * i + 1], -gy); atomicAdd(&a.dpos[3 * i + 2], -gz);
     }
-    // dv_j += D^T dv~; dq_i, dk_j += row0^T dq~0 / dk~0
-    for (int x = threadIdx.x; x < QC; x += blockDim.x) {
-      const int q = x / C, c = x % C;
-      int l = 0;
-      while ((l + 1) * (l + 1) <= q) ++l;
-      const int w = 2 * l + 1, mp = q - l * l;
-      const float *Dl = D + wig_offset(l);
-      float acc = 0.f;
-      for (int m = 0; m < w; ++m) acc = fmaf(Dl[m * w + mp], dvt[(l * l + m) * C + c], acc);
-      atomicAdd(&a.dv[(size_t)j * QC + x], acc);
-      const float r0 = Dl[l * w + mp], ds = dsh[c / Ch];
-      atomicAdd(&a.dq[(size_t)i * QC + x], r0 * ds * qk[(L + 1) * C + l * C + c]);
-      atomicAdd(&a.dk[(size_t)j * QC + x], r0 * ds * qk[l * C + c]);
+    // dv_j += D^T dv~; dq_i, dk_j += row0^T dq~0 / dk~0 -- four channels per
+    // thread and one 16-byte atomic per array when C is a multiple of 4
+    if ((C & 3) == 0) {
+      for (int x4 = threadIdx.x; x4 < QC / 4; x4 += blockDim.x) {
+        const int x = 4 * x4, q = x / C, c = x % C;
+        int l = 0;
+        while ((l + 1) * (l + 1) <= q) ++l;
+        const int w = 2 * l + 1, mp = q - l * l;
+        const float *Dl = D + wig_offset(l);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 0; m < w; ++m) {
+          const float dm = Dl[m * w + mp];
+          const float *src = dvt + (l * l + m) * C + c;
+          acc.x = fmaf(dm, src[0], acc.x); acc.y = fmaf(dm, src[1], acc.y);
+          acc.z = fmaf(dm, src[2], acc.z); acc.w = fmaf(dm, src[3], acc.w);
+        }
+        atomicAdd(reinterpret_cast<float4 *>(a.dv + (size_t)j * QC + x), acc);
+        const float r0 = Dl[l * w + mp];
+        float4 gq, gk;
+        const float *qt = qk + (L + 1) * C + l * C + c, *kt = qk + l * C + c;
+        gq.x = r0 * dsh[c / Ch] * qt[0];       gk.x = r0 * dsh[c / Ch] * kt[0];
+        gq.y = r0 * dsh[(c + 1) / Ch] * qt[1]; gk.y = r0 * dsh[(c + 1) / Ch] * kt[1];
+        gq.z = r0 * dsh[(c + 2) / Ch] * qt[2]; gk.z = r0 * dsh[(c + 2) / Ch] * kt[2];
+        gq.w = r0 * dsh[(c + 3) / Ch] * qt[3]; gk.w = r0 * dsh[(c + 3) / Ch] * kt[3];
+        atomicAdd(reinterpret_cast<float4 *>(a.dq + (size_t)i * QC + x), gq);
+        atomicAdd(reinterpret_cast<float4 *>(a.dk + (size_t)j * QC + x), gk);
+      }
+    } else {
+      for (int x = threadIdx.x; x < QC; x += blockDim.x) {
+        const int q = x / C, c = x % C;
+        int l = 0;
+        while ((l + 1) * (l + 1) <= q) ++l;
+        const int w = 2 * l + 1, mp = q - l * l;
+        const float *Dl = D + wig_offset(l);
+        float acc = 0.f;
+        for (int m = 0; m < w; ++m) acc = fmaf(Dl[m * w + mp], dvt[(l * l + m) * C + c], acc);
+        atomicAdd(&a.dv[(size_t)j * QC + x], acc);
+        const float r0 = Dl[l * w + mp], ds = dsh[c / Ch];
+        atomicAdd(&a.dq[(size_t)i * QC + x], r0 * ds * qk[(L + 1) * C + l * C + c]);
+        atomicAdd(&a.dk[(size_t)j * QC + x], r0 * ds * qk[l * C + c]);
+      }
     }
   }
 }

@@ -4,18 +4,20 @@
 // ...", §2.1 EAAS change of basis, §2.2 node-centric streaming with no edge
 // materialisation; "EquiformerV3 ...", §2B.3 envelope in the softmax).
 //
-// Structure (one persistent CTA per SM, 512 threads, contiguous edge range
-// per CTA, tiles of <= 64 edges (32 for L = 5, 6) covering <= 4 destination
+// Structure (one persistent CTA per SM, 512 threads; CTA b owns the nodes
+// whose rows start in its share of the edges, so no node is split between
+// CTAs; tiles of <= 64 edges (32 for L = 5, 6) covering <= 4 destination
 // nodes):
 //
 //   producers (warps 8-15)  per tile: edge geometry, Wigner blocks of the
 //                           y-rotation in the two-angle frame (parity blocks),
-//                           envelope, radial MLP, logits -> alpha (exact
-//                           softmax: per-node max / denominator come from
-//                           a pre-pass, so nothing is rescaled later); then,
-//                           block by block, the rotated neighbour features
-//                           v~ = D v_j written as bf16 MMA operands (one
-//                           64 x 128 "unit" per (degree, +-m)).
+//                           envelope, radial MLP, logits, and the online-
+//                           softmax statistics of the tile (per node and head:
+//                           the node's reference maximum, alpha, the factor
+//                           for its earlier sums, the running denominator);
+//                           then, block by block, the rotated neighbour
+//                           features v~ = D v_j written as bf16 MMA operands
+//                           (one 64 x 128 "unit" per (degree, +-m)).
 //   loaders (warps 1-2)     stream pre-packed weight tiles (Wr|Wi, or W0)
 //                           from L2 with 1-D bulk copies.
 //   MMA (warp 0)            SO(2) block products as tcgen05.mma (M = 64
@@ -29,14 +31,17 @@
 //                           hands it over:
 //                           Out_l[c, (slot, m')] += sum_e A[c, e] R[(slot,m'), e]
 //                           with A = alpha g y (bf16) and R = D^l[+-m][m'].
-//   epilogue (warps 4-7)    TMEM y -> A (scaled bf16, shared memory), builds R,
-//                           reads finished nodes' Out columns -> o_i.
+//   epilogue (warps 4-7)    TMEM y -> A (scaled bf16, shared memory), builds R;
+//                           at tile end, finished nodes' Out columns / the
+//                           denominator -> o_i, and the continuing node's
+//                           columns rescaled when its reference maximum moved.
 //
 // All waits are bounded; a timeout raises a CTA-wide abort flag and the
 // device error word (E2F_ERR_TIMEOUT) and every role exits its loops.
 #include <algorithm>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "common.cuh"
 #include "tc_common.cuh"
@@ -56,6 +61,10 @@ constexpr int NTHREADS = 512;
 constexpr int HMAX = 16;
 constexpr int ALS = HMAX + 1;     // alpha row stride (odd: conflict-free per-edge rows)
 constexpr uint32_t WAIT_LIMIT = 1u << 25;
+// online softmax: how far (in logit units) a node's later tiles may exceed
+// its reference maximum before the reference moves; alpha = e^(s - M) then
+// stays below e^8 (< 3000, exact range of the fp16 alpha store)
+constexpr float SOFTMAX_MARGIN = 8.f;
 // TMEM columns: [0, 256) two y buffers (y+ in lanes 0-15, y- in lanes 16-31 of
 // each 32-lane subpartition), [256, 256 + OUT_COLS) the per-node output sums,
 // [384, 512) one rotated-feature unit pair used as the MMA A operand.
@@ -193,6 +202,16 @@ struct Waiter {
   __device__ bool aborted() const { return *abort_flag != 0; }
 };
 
+// f(std::integral_constant<int, l>) for l = 0..L, each degree a compile-time
+// constant.
+template <int... ls, class F>
+__device__ __forceinline__ void for_degrees_impl(std::integer_sequence<int, ls...>, F &&f) {
+  (f(std::integral_constant<int, ls>{}), ...);
+}
+template <int L, class F> __device__ __forceinline__ void for_degrees(F &&f) {
+  for_degrees_impl(std::make_integer_sequence<int, L + 1>{}, f);
+}
+
 // Edge range of one CTA, aligned to node boundaries: CTA b of G owns the
 // nodes [n_b, n_{b+1}) with n_0 = 0, n_G = N and, in between, n_b the first
 // node whose row starts at or after edge E b / G; its edges are
@@ -213,7 +232,6 @@ struct TileIter {
   const int32_t *rp;
   int N;
   int te;   // edges per tile
-  int nlo, nhi;       // nodes owned by this CTA
   int64_t ebeg, eend;
   int64_t e0, e1;
   int n0;
@@ -221,12 +239,6 @@ struct TileIter {
   static __device__ int2 node_range(const int32_t *rp, int N, int b, int G, int64_t E) {
     return make_int2(b == 0 ? 0 : first_node_at(rp, N, E * (int64_t)b / G),
                      b + 1 == G ? N : first_node_at(rp, N, E * (int64_t)(b + 1) / G));
-  }
-  __device__ void init(int2 nr) {
-    nlo = nr.x;
-    nhi = nr.y;
-    ebeg = rp[nlo];
-    eend = rp[nhi];
   }
   __device__ void bounds() {
     const int nlim = min(n0 + S, N);
@@ -238,8 +250,14 @@ struct TileIter {
   __device__ bool start() {
     e0 = ebeg;
     if (e0 >= eend) return false;
-    n0 = nlo;
-    while ((int64_t)rp[n0 + 1] <= e0) ++n0;   // skip empty rows
+    int lo = 0, hi = N - 1;   // largest n with rp[n] <= e0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((int64_t)rp[mid] <= e0) lo = mid;
+      else hi = mid - 1;
+    }
+    n0 = lo;
+    while ((int64_t)rp[n0 + 1] <= e0) ++n0;
     bounds();
     return true;
   }
@@ -470,7 +488,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 
   TileIter ti;
   ti.rp = a.row_ptr; ti.N = a.N; ti.te = Cf::TE;
-  ti.init(*reinterpret_cast<const int2 *>(tslot + 2));
+  {
+    const int2 nr = *reinterpret_cast<const int2 *>(tslot + 2);
+    ti.ebeg = a.row_ptr[nr.x];
+    ti.eend = a.row_ptr[nr.y];
+  }
   const int H = a.H, Ch = CH / H;
   const int hshift = 31 - __clz(Ch);   // Ch is a power of two
 
@@ -666,9 +688,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     }
     // rows of this CTA's nodes with no neighbour are never visited by a
     // tile: o_i = 0 for them
-    for (int base = ti.nlo + 32 * ew; base < ti.nhi; base += 128) {
+    const int2 nrange = *reinterpret_cast<const int2 *>(tslot + 2);
+    for (int base = nrange.x + 32 * ew; base < nrange.y; base += 128) {
       const int n = base + lane;
-      const bool empty = n < ti.nhi && a.row_ptr[n] == a.row_ptr[n + 1];
+      const bool empty = n < nrange.y && a.row_ptr[n] == a.row_ptr[n + 1];
       uint32_t msk = __ballot_sync(0xffffffffu, empty);
       while (msk) {
         const int nn = base + __ffs(msk) - 1;
@@ -717,9 +740,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
 #pragma unroll 1
             for (int i = 0; i < 8; i += 2) {
               float v[2][16];
-              tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i, v[0]);
-              tmem_ld_32x32b_x16(tbase + lane_base + 128 * b + 16 * i + 16, v[1]);
-              tmem_ld_wait();
+              tmem_ld_32x32b_x16x2(tbase + lane_base + 128 * b + 16 * i, tbase + lane_base + 128 * b + 16 * i + 16,
+                                   v[0], v[1]);
               if (sg == which) {
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -727,12 +749,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                   // channels [c0, c0 + 8) and [c0 + 8, c0 + 16) lie in one head each
                   const float s_lo = (e < ne) ? __half2float(al[e * ALS + (c0 >> hshift)]) * ge : 0.f;
                   const float s_hi = (e < ne) ? __half2float(al[e * ALS + ((c0 + 8) >> hshift)]) * ge : 0.f;
-                  __align__(16) __nv_bfloat16 o[16];
-#pragma unroll
-                  for (int j = 0; j < 16; ++j) o[j] = __float2bfloat16_rn(v[h2][j] * (j < 8 ? s_lo : s_hi));
+                  const float *vv = v[h2];
+                  const uint4 lo = make_uint4(pack_bf16x2(vv[0] * s_lo, vv[1] * s_lo), pack_bf16x2(vv[2] * s_lo, vv[3] * s_lo),
+                                              pack_bf16x2(vv[4] * s_lo, vv[5] * s_lo), pack_bf16x2(vv[6] * s_lo, vv[7] * s_lo));
+                  const uint4 hi = make_uint4(pack_bf16x2(vv[8] * s_hi, vv[9] * s_hi), pack_bf16x2(vv[10] * s_hi, vv[11] * s_hi),
+                                              pack_bf16x2(vv[12] * s_hi, vv[13] * s_hi), pack_bf16x2(vv[14] * s_hi, vv[15] * s_hi));
                   if (e < TE) {   // TMEM rows of edges >= TE (32-edge tiles) are not real
-                    *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0, e, TE)) = *reinterpret_cast<uint4 *>(&o[0]);
-                    *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0 + 8, e, TE)) = *reinterpret_cast<uint4 *>(&o[8]);
+                    *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0, e, TE)) = lo;
+                    *reinterpret_cast<uint4 *>(A2 + mnmajor_off(c0 + 8, e, TE)) = hi;
                   }
                 }
               }
@@ -818,33 +842,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           if (a.row_ptr[i + 1] == a.row_ptr[i]) continue;   // empty row: zeroed at the start
           const int slot = i % S;
           const bool fin = !(cont && i == n1);
+          // a continuing node whose reference maximum did not move (factor 1
+          // for every head of this warp's channels) needs no rescale
+          if (!fin && __all_sync(0xffffffffu, fnext[slot * HMAX + h] == 1.f)) continue;
           const float lsum = ls[slot * HMAX + h];
           const float scale = fin ? (lsum > 0.f ? 1.f / lsum : 0.f) : fnext[slot * HMAX + h];
           float *orow = a.out + (size_t)i * Q * CH + c;
-          uint32_t r[Q];
-#pragma unroll
-          for (int l = 0; l <= L; ++l) {
-#pragma unroll
-            for (int mp = 0; mp < 2 * l + 1; ++mp) {
-              const uint32_t col = TM_OUT + Cf::OB(l) + Cf::RO(l) + slot * (2 * l + 1) + mp;
-              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
-                           : "=r"(r[l * l + mp])
-                           : "r"(tbase + lane_base + col));
-            }
-          }
-          tmem_ld_wait();
-#pragma unroll
-          for (int l = 0; l <= L; ++l) {
+          // degree by degree: the node's 2l + 1 columns are consecutive and
+          // are read as one load of the next power-of-two width (the extra
+          // columns lie inside the allocation and are ignored)
+          for_degrees<L>([&](auto lc) {
+            constexpr int l = decltype(lc)::value;
+            constexpr int NW = l == 0 ? 1 : (l == 1 ? 4 : (l <= 3 ? 8 : 16));
+            const uint32_t col0 = TM_OUT + Cf::OB(l) + Cf::RO(l) + slot * (2 * l + 1);
+            uint32_t r[NW];
+            tmem_ld_cols<NW>(tbase + lane_base + col0, r);
 #pragma unroll
             for (int mp = 0; mp < 2 * l + 1; ++mp) {
-              const uint32_t col = TM_OUT + Cf::OB(l) + Cf::RO(l) + slot * (2 * l + 1) + mp;
-              const float val = __uint_as_float(r[l * l + mp]) * scale;
+              const float val = __uint_as_float(r[mp]) * scale;
               if (fin) __stcs(orow + (size_t)(l * l + mp) * CH, val);   // written once: evict-first
-              asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col),
+              asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(tbase + lane_base + col0 + mp),
                            "r"(fin ? 0u : __float_as_uint(val))
                            : "memory");
             }
-          }
+          });
         }
         tmem_st_wait();
         tc_fence_before();
@@ -979,88 +1000,65 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       const int *jj = g_jj(c), *nodeof = jj + TE;
       const float *csb = g_cs(c), *snb = csb + TE * (L > 0 ? L : 1);
       const __half *dy = g_dy(c);
-      // the IPH items' q and k rows (2 Q per item, 16 bytes each) are streamed
-      // through a ring of RING registers: row k + RING is loaded as soon as
-      // row k has been consumed
-      constexpr int RPI = 2 * Q;              // rows per item: (q, k) per coefficient
-      constexpr int TOT = IPH * RPI;
-      constexpr int RING = 16;
-      const __nv_bfloat16 *qr[IPH], *kr[IPH];
-      int ee[IPH];
-#pragma unroll
+#pragma unroll 1
       for (int it = 0; it < IPH; ++it) {
         const int item = pt + half * (TE * 8) + it * 256;
         const int e = item >> 4, c0 = (item & 15) * 8;
-        ee[it] = e;
-        const int i = e < ne ? nodeof[e] : 0, j = e < ne ? jj[e] : 0;   // dead items read node 0, weight 0
-        qr[it] = a.q + (size_t)i * Q * CH + c0;
-        kr[it] = a.k + (size_t)j * Q * CH + c0;
-      }
-      auto row_addr = [&](int k) {
-        const int it = k / RPI, r = (k % RPI) >> 1;
-        return reinterpret_cast<const uint4 *>(((k & 1) ? kr[it] : qr[it]) + (size_t)r * CH);
-      };
-      uint4 ring[RING];
-#pragma unroll
-      for (int k = 0; k < RING; ++k) ring[k] = *row_addr(k);
-      auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
-      float2 accv[4], qh[4], kh[4];
-      float coef = 0.f;
-#pragma unroll
-      for (int k = 0; k < TOT; ++k) {
-        const int it = k / RPI, r = (k % RPI) >> 1;
-        int l = 0;
-        while ((l + 1) * (l + 1) <= r) ++l;                 // degree of coefficient r (compile time)
-        const int tt = r - l * l, mp = tt - l, amp = mp < 0 ? -mp : mp;
-        const int e = ee[it];
-        const uint4 row = ring[k % RING];
-        if (k + RING < TOT) ring[k % RING] = *row_addr(k + RING);
-        if (k % RPI == 0) {
+        float acc = 0.f;
+        if (e < ne) {
+          const int i = nodeof[e], j = jj[e];
+          const __half *d = dy + e * Cf::NDYP;
+          const __nv_bfloat16 *qr = a.q + (size_t)i * Q * CH + c0;
+          const __nv_bfloat16 *kr = a.k + (size_t)j * Q * CH + c0;
+          float2 accv[4];
 #pragma unroll
           for (int x = 0; x < 4; ++x) accv[x] = make_float2(0.f, 0.f);
-        }
-        if ((k & 1) == 0) {
-          if (tt == 0) {
+          auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+#pragma unroll
+          for (int l = 0; l <= L; ++l) {
+            uint4 qv[2 * L + 1], kv[2 * L + 1];
+#pragma unroll
+            for (int tt = 0; tt < 2 * l + 1; ++tt) {
+              qv[tt] = *reinterpret_cast<const uint4 *>(qr + (size_t)(l * l + tt) * CH);
+              kv[tt] = *reinterpret_cast<const uint4 *>(kr + (size_t)(l * l + tt) * CH);
+            }
+            float2 qh[4], kh[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) { qh[x] = make_float2(0.f, 0.f); kh[x] = make_float2(0.f, 0.f); }
-          }
-          // m = 0 row of D^l in the edge frame (gauge-free: normalised real SH of rhat)
-          const float de = e < ne ? __half2float(dy[e * Cf::NDYP + dye_off<L>(l) + amp]) : 0.f;
-          coef = (mp == 0) ? de : (mp > 0 ? de * csb[(amp - 1) * TE + min(e, TE - 1)] : de * snb[(amp - 1) * TE + min(e, TE - 1)]);
-        }
-        const float2 c2 = make_float2(coef, coef);
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(&row);
-        if ((k & 1) == 0) {
 #pragma unroll
-          for (int x = 0; x < 4; ++x) qh[x] = __ffma2_rn(c2, pair(w[x]), qh[x]);
-        } else {
+            for (int tt = 0; tt < 2 * l + 1; ++tt) {
+              const int mp = tt - l, amp = mp < 0 ? -mp : mp;
+              const float de = __half2float(d[dye_off<L>(l) + amp]);   // row 0 of the even block
+              const float coef = (mp == 0) ? de : (mp > 0 ? de * csb[(amp - 1) * TE + e] : de * snb[(amp - 1) * TE + e]);
+              const float2 c2 = make_float2(coef, coef);
 #pragma unroll
-          for (int x = 0; x < 4; ++x) kh[x] = __ffma2_rn(c2, pair(w[x]), kh[x]);
-          if (tt == 2 * l) {   // degree l complete
+              for (int x = 0; x < 4; ++x) {
+                qh[x] = __ffma2_rn(c2, pair(u4w(qv[tt], x)), qh[x]);
+                kh[x] = __ffma2_rn(c2, pair(u4w(kv[tt], x)), kh[x]);
+              }
+            }
 #pragma unroll
             for (int x = 0; x < 4; ++x) accv[x] = __ffma2_rn(qh[x], kh[x], accv[x]);
           }
-        }
-        if (k % RPI == RPI - 1) {
-          float acc = 0.f;
 #pragma unroll
           for (int x = 0; x < 4; ++x) acc += accv[x].x + accv[x].y;
-          const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
-          for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          // the softmax logit with the envelope folded in: u e^s = e^(s + log u)
-          // (the lane owning the head's first block keeps it for the
-          // statistics step)
-          sk[it] = (e < ne) ? acc * a.inv_sqrt_d + logf(geo[e * 4 + 2]) : -INFINITY;
         }
+        const int nb = Ch >> 3;   // 8-channel blocks per head: 1, 2 or 4
+        for (int o = 1; o < nb; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        // the softmax logit with the envelope folded in: u e^s = e^(s + log u)
+        // (the lane owning the head's first block keeps it for the
+        // statistics step)
+        sk[it] = (e < ne) ? acc * a.inv_sqrt_d + logf(geo[e * 4 + 2]) : -INFINITY;
       }
     };
     // ---- online softmax statistics of tile g (copy c), after both logit
     // halves ("E2Former-V2 ...", §2.2 online softmax; "EquiformerV3 ...",
     // §2B.3 envelope in numerator and denominator).  Per (node slot, head):
-    // tile max of the logits, running max M (reset when the node starts in
-    // this tile), alpha = e^(s + log u - M) for the tile's edges (fp16, in
-    // (0, 1]), the factor e^(M_old - M) for the node's earlier sums, and the
-    // running denominator l = l_old e^(M_old - M) + sum alpha.
+    // tile max of the logits, the node's reference maximum M (its first
+    // tile's maximum, moved up only when a later tile exceeds it by more than
+    // SOFTMAX_MARGIN), alpha = e^(s + log u - M) for the tile's edges (fp16,
+    // at most e^margin), the factor e^(M_old - M) for the node's earlier sums
+    // (1 unless M moved), and the running denominator l = l_old f + sum alpha.
     int *smx = reinterpret_cast<int *>(smem + Cf::OFF_SMX);      // tile max, order-preserving int
     float *ssum = reinterpret_cast<float *>(smx + S * HMAX);    // tile sum of alpha
     float *mcur = ssum + S * HMAX;                               // running max after the tile
@@ -1099,9 +1097,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         live = node >= 0 && h < H;
         if (live) {
           starts = (int64_t)a.row_ptr[node] >= g.e0;
-          const float Mo = starts ? -INFINITY : rs_m[pt];
-          Mn = fmaxf(Mo, unord(smx[pt]));
-          f = (Mn == -INFINITY) ? 1.f : expf(Mo - Mn);
+          const float Mo = starts ? -INFINITY : rs_m[pt], tmax = unord(smx[pt]);
+          // the node keeps its reference maximum while the tile's stays
+          // within SOFTMAX_MARGIN of it (alpha <= e^margin, no rescale);
+          // otherwise the reference moves up and the earlier sums are
+          // rescaled by e^(M_old - M)
+          if (Mo == -INFINITY || tmax > Mo + SOFTMAX_MARGIN) {
+            Mn = tmax;
+            f = (Mo == -INFINITY) ? 1.f : expf(Mo - Mn);
+          } else {
+            Mn = Mo;
+          }
         }
         mcur[pt] = Mn;
         g_f(c)[pt] = f;
@@ -1182,54 +1188,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
         #pragma unroll 1
         for (int lp = m; lp <= L; ++lp) {
           const int sp = (m == 0) ? lp : 2 * (lp - m);
-          // each producer warp waits for the unit on its own (the warps run
-          // through the units independently); the wait comes after the first
-          // rows of the unit's gathers have been issued, so their latency
-          // overlaps it
-          auto slot_ready = [&]() -> bool {
+          {
+            // each producer warp waits for the unit on its own: the warps run
+            // through the units independently (a warp that finished its part
+            // of one unit starts loading for the next)
             bool f = false;
             if (lane == 0) {
               f = !W.wait(&unit_empty[sp], ((pfillpar >> sp) & 1) ^ 1, 40);
               if (!f && m > 0) f = !W.wait(&unit_empty[sp + 1], ((pfillpar >> (sp + 1)) & 1) ^ 1, 40);
             }
             dead = __shfl_sync(0xffffffffu, (int)(f || W.aborted()), 0) != 0;
-            return !dead;
-          };
+            if (dead) break;
+          }
           // v~(+m), v~(-m) of degree l' (compile-time constant: register use
           // follows the degree) for NB (edge, 8-channel block) items of this
           // thread: block b belongs to edge ea (first half of the blocks, or
           // all of them when NEc = 1) or eb (second half), and covers
-          // channels [cbs[b], +8).  The NB x (2l'+1) gathered 16-byte rows are
-          // streamed through a ring of RING registers: row k + RING is
-          // loaded as soon as row k has been consumed, so RING rows stay in
-          // flight across block and edge boundaries.  Pairs of channels go
-          // through packed fp32 FMAs.  emit(b, wp, wm) receives block b as
-          // packed bf16 pairs (wp: +m, wm: -m); edges past the tile's end
-          // come out zero.  Returns false (nothing emitted) on an abort.
-          auto rot4 = [&](auto LPc, auto NEc, const int ea, const int eb, const auto &cbs, auto &&emit) -> bool {
+          // channels [cbs[b], +8).  Pairs of channels go through packed fp32
+          // FMAs.  emit(b, wp, wm) receives block b as packed bf16 pairs (wp:
+          // +m, wm: -m); edges past the tile's end come out zero.
+          auto rot4 = [&](auto LPc, auto NEc, const int ea, const int eb, const auto &cbs, auto &&emit) {
             constexpr int LP = decltype(LPc)::value;
             constexpr int NR = 2 * LP + 1;
             constexpr int NB = (int)(sizeof(cbs) / sizeof(int));   // blocks of this thread
             constexpr int NE = decltype(NEc)::value;               // distinct edges: 1 or 2
             constexpr int BPE = NB / NE;                           // blocks per edge
-            constexpr int TOT = NB * NR;                           // rows of this thread
-            constexpr int RING = TOT < 16 ? TOT : 16;
-            // rows of edges past the tile's end: node 0's, scaled by zero (every
-            // lane takes the same path: slot_ready() is warp-collective)
+            if constexpr (NE == 1) {
+              if (ea >= ne) {
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int bb = 0; bb < NB; ++bb) emit(bb, z, z);
+                return;
+              }
+            }
+            // rows of edges past the tile's end: node 0's, scaled by zero
             const __nv_bfloat16 *vra = a.v + (size_t)(ea < ne ? jj[ea] : 0) * Q * CH + (size_t)(LP * LP) * CH;
             const __nv_bfloat16 *vrb = NE == 1 ? vra : a.v + (size_t)(eb < ne ? jj[eb] : 0) * Q * CH + (size_t)(LP * LP) * CH;
-            auto row_addr = [&](int k) {
-              const int bb = k / NR, t = k % NR;
-              return reinterpret_cast<const uint4 *>((bb < BPE ? vra : vrb) + (size_t)t * CH + cbs[bb]);
-            };
-            uint4 ring[RING];
-#pragma unroll
-            for (int k = 0; k < RING; ++k) ring[k] = *row_addr(k);
-            if (!slot_ready()) return false;
             // per-edge coefficients: u+ = c v+ + s v-, u- = -s v+ + c v-, scaled
             // by the y-rotation entries of row +m (even block) / -m (odd block)
             float c0 = 0.f, app[LP > 0 ? LP : 1], apm[LP > 0 ? LP : 1], amp[LP > 0 ? LP : 1], amm[LP > 0 ? LP : 1];
-            auto coeffs = [&](int e) {
+            {
+              const int e = ea;
               const bool live = e < ne;
               const __half *d = dy + (live ? e : 0) * Cf::NDYP;
               c0 = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1)]) : 0.f;
@@ -1241,50 +1240,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
                 amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
               }
-            };
-            coeffs(ea);
-            auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
-            float2 ap[4], am[4];
-#pragma unroll
-            for (int k = 0; k < TOT; ++k) {
-              const int bb = k / NR, t = k % NR, mp = t - LP;
-              if (NE == 2 && t == 0 && bb == BPE) coeffs(eb);
-              const uint4 row = ring[k % RING];
-              if (k + RING < TOT) ring[k % RING] = *row_addr(k + RING);
-              const uint32_t *wv = reinterpret_cast<const uint32_t *>(&row);
-              if (t == 0) {
-#pragma unroll
-                for (int x = 0; x < 4; ++x) { ap[x] = make_float2(0.f, 0.f); am[x] = make_float2(0.f, 0.f); }
-              }
-              if (mp == 0) {
-                const float2 cc = make_float2(c0, c0);
-#pragma unroll
-                for (int x = 0; x < 4; ++x) ap[x] = __ffma2_rn(cc, pair(wv[x]), ap[x]);
-              } else {
-                const int kq = mp > 0 ? mp : -mp;
-                const float2 cp = mp > 0 ? make_float2(app[kq - 1], app[kq - 1]) : make_float2(apm[kq - 1], apm[kq - 1]);
-                const float2 cm = mp > 0 ? make_float2(amp[kq - 1], amp[kq - 1]) : make_float2(amm[kq - 1], amm[kq - 1]);
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                  const float2 v2 = pair(wv[x]);
-                  ap[x] = __ffma2_rn(cp, v2, ap[x]);
-                  am[x] = __ffma2_rn(cm, v2, am[x]);
-                }
-              }
-              if (t == NR - 1) {
-                uint4 wp, wm;
-                uint32_t *pp = reinterpret_cast<uint32_t *>(&wp), *pm = reinterpret_cast<uint32_t *>(&wm);
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                  const __nv_bfloat162 hp = __floats2bfloat162_rn(ap[x].x, ap[x].y);
-                  const __nv_bfloat162 hm = __floats2bfloat162_rn(am[x].x, am[x].y);
-                  pp[x] = *reinterpret_cast<const uint32_t *>(&hp);
-                  pm[x] = *reinterpret_cast<const uint32_t *>(&hm);
-                }
-                emit(bb, wp, wm);
-              }
             }
-            return true;
+            // two blocks of gathered rows in flight: block b + 1 is loaded
+            // while block b is computed
+            constexpr int DEPTH = 2;
+            uint4 buf[DEPTH][NR];
+#pragma unroll
+            for (int bb = 0; bb < DEPTH - 1; ++bb)
+#pragma unroll
+              for (int t = 0; t < NR; ++t) buf[bb][t] = *reinterpret_cast<const uint4 *>((bb < BPE ? vra : vrb) + (size_t)t * CH + cbs[bb]);
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) {
+              if (bb > 0 && bb % BPE == 0)   // next edge
+              {
+                const int e = eb;
+                const bool live = e < ne;
+                const __half *d = dy + (live ? e : 0) * Cf::NDYP;
+                c0 = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1)]) : 0.f;
+#pragma unroll
+                for (int kq = 1; kq <= LP; ++kq) {
+                  const float ck = csb[(kq - 1) * TE + e], sk = snb[(kq - 1) * TE + e];
+                  const float de = live ? __half2float(d[dye_off<L>(LP) + m * (LP + 1) + kq]) : 0.f;
+                  const float dd = (live && m > 0) ? __half2float(d[dyo_off<L>(LP) + (m - 1) * LP + (kq - 1)]) : 0.f;
+                  app[kq - 1] = de * ck; apm[kq - 1] = de * sk;
+                  amp[kq - 1] = -dd * sk; amm[kq - 1] = dd * ck;
+                }
+              }
+              if (bb + DEPTH - 1 < NB) {
+                const int nb = bb + DEPTH - 1 < NB ? bb + DEPTH - 1 : 0;
+#pragma unroll
+                for (int t = 0; t < NR; ++t)
+                  buf[(bb + DEPTH - 1) % DEPTH][t] = *reinterpret_cast<const uint4 *>((nb < BPE ? vra : vrb) + (size_t)t * CH + cbs[nb]);
+              }
+              auto pair = [](uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+              float2 ap[4], am[4];
+              {
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const float2 v0 = pair(u4w(buf[bb % DEPTH][LP], x));
+                  ap[x] = make_float2(c0 * v0.x, c0 * v0.y);
+                  am[x] = make_float2(0.f, 0.f);
+                }
+              }
+#pragma unroll
+              for (int kq = 1; kq <= LP; ++kq) {
+
+                const float2 cpp = make_float2(app[kq - 1], app[kq - 1]), cpm = make_float2(apm[kq - 1], apm[kq - 1]);
+                const float2 cmp = make_float2(amp[kq - 1], amp[kq - 1]), cmm = make_float2(amm[kq - 1], amm[kq - 1]);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const float2 vp2 = pair(u4w(buf[bb % DEPTH][LP + kq], x)), vn2 = pair(u4w(buf[bb % DEPTH][LP - kq], x));
+                  ap[x] = __ffma2_rn(cpp, vp2, __ffma2_rn(cpm, vn2, ap[x]));
+                  am[x] = __ffma2_rn(cmp, vp2, __ffma2_rn(cmm, vn2, am[x]));
+                }
+              }
+              const uint4 wp = make_uint4(pack_bf16x2(ap[0].x, ap[0].y), pack_bf16x2(ap[1].x, ap[1].y),
+                                          pack_bf16x2(ap[2].x, ap[2].y), pack_bf16x2(ap[3].x, ap[3].y));
+              const uint4 wm = make_uint4(pack_bf16x2(am[0].x, am[0].y), pack_bf16x2(am[1].x, am[1].y),
+                                          pack_bf16x2(am[2].x, am[2].y), pack_bf16x2(am[3].x, am[3].y));
+              emit(bb, wp, wm);
+            }
           };
           if (Cf::TMU && sp >= Cf::NSU) {
             if constexpr (Cf::TMU) {
@@ -1302,12 +1317,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               const int cb0 = chb + 32 * half;
               const int cbs[4] = {cb0, cb0 + 8, cb0 + 16, cb0 + 24};
               rot4(std::integral_constant<int, L>{}, std::integral_constant<int, 1>{}, e, e, cbs, [&](int bb, const uint4 &wp, const uint4 &wm) {
-                const uint32_t *pp = reinterpret_cast<const uint32_t *>(&wp), *pm = reinterpret_cast<const uint32_t *>(&wm);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) { wpl[4 * bb + i] = pp[i]; wmi[4 * bb + i] = pm[i]; }
+                for (int i = 0; i < 4; ++i) { wpl[4 * bb + i] = u4w(wp, i); wmi[4 * bb + i] = u4w(wm, i); }
               });
             }
-            if (dead) break;
             uint32_t opl[16], omi[16];   // the partner half's block
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -1360,7 +1373,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
               case 5: if constexpr (L >= 5) fill(std::integral_constant<int, (L >= 5 ? 5 : 0)>{}); break;
               default: if constexpr (L >= 6) fill(std::integral_constant<int, (L >= 6 ? 6 : 0)>{}); break;
             }
-            if (dead) break;
           }
           fence_async_smem();
           __syncwarp();
@@ -1405,6 +1417,11 @@ static e2f_status launch_tc(const TcArgs &args, int grid, cudaStream_t s) {
 e2f_status attention_tc_available(const e2f_weights *w) {
   if (w->dtype != E2F_BF16 || w->C != tca::CH) return E2F_ERR_UNSUPPORTED;
   if (w->L_max < 1 || w->L_max > 6) return E2F_ERR_UNSUPPORTED;
+  // L = 3 is not instantiated: its build of this kernel stopped on the GPU
+  // with a misaligned-address fault whose cause has not been found (every
+  // address the source forms is 16-byte aligned by construction); L = 3
+  // inputs run on the CUDA-core kernel instead
+  if (w->L_max == 3) return E2F_ERR_UNSUPPORTED;
   // heads of 8..32 channels (the head reductions run inside one warp)
   if (w->H < 4 || w->H > tca::HMAX || tca::CH % w->H != 0) return E2F_ERR_UNSUPPORTED;
   return E2F_OK;
@@ -1474,7 +1491,6 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   switch (L) {
     case 1: r = launch_tc<1>(a, grid, s); break;
     case 2: r = launch_tc<2>(a, grid, s); break;
-    case 3: r = launch_tc<3>(a, grid, s); break;
     case 4: r = launch_tc<4>(a, grid, s); break;
     case 5: r = launch_tc<5>(a, grid, s); break;
     case 6: r = launch_tc<6>(a, grid, s); break;

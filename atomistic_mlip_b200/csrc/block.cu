@@ -254,7 +254,6 @@ __global__ void __launch_bounds__(NT, 1) dgemm_tc_kernel(DG a, long long ntiles,
       for (int c0 = 0; c0 < Nout / 2; c0 += 16) {
         float v[16];
         tmem_ld_32x32b_x16(tb + ((uint32_t)(32 * (warp & 3)) << 16) + cb + c0, v);
-        tmem_ld_wait();
         if (live) {
           const size_t oi = ((size_t)node * a.out_q + l * l + m) * Nout + cb + c0;
           if (EPI == EPI_SILU) {
@@ -264,18 +263,16 @@ __global__ void __launch_bounds__(NT, 1) dgemm_tc_kernel(DG a, long long ntiles,
               o4[i] = make_float4(silu(v[4 * i]), silu(v[4 * i + 1]), silu(v[4 * i + 2]), silu(v[4 * i + 3]));
           } else if (EPI == EPI_GATE) {
             const float4 *g4 = reinterpret_cast<const float4 *>(a.gate + (size_t)node * Nout + cb + c0);
-            __align__(16) __nv_bfloat16 o[16];
+            uint32_t w[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float4 gg = g4[i];
-              o[4 * i] = __float2bfloat16_rn(v[4 * i] * gg.x);
-              o[4 * i + 1] = __float2bfloat16_rn(v[4 * i + 1] * gg.y);
-              o[4 * i + 2] = __float2bfloat16_rn(v[4 * i + 2] * gg.z);
-              o[4 * i + 3] = __float2bfloat16_rn(v[4 * i + 3] * gg.w);
+              w[2 * i] = pack_bf16x2(v[4 * i] * gg.x, v[4 * i + 1] * gg.y);
+              w[2 * i + 1] = pack_bf16x2(v[4 * i + 2] * gg.z, v[4 * i + 3] * gg.w);
             }
             __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(a.out) + oi;
-            *reinterpret_cast<uint4 *>(op) = *reinterpret_cast<const uint4 *>(&o[0]);
-            *reinterpret_cast<uint4 *>(op + 8) = *reinterpret_cast<const uint4 *>(&o[8]);
+            *reinterpret_cast<uint4 *>(op) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(op + 8) = make_uint4(w[4], w[5], w[6], w[7]);
           } else {
             float4 *o4 = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + oi);
 #pragma unroll

@@ -32,7 +32,11 @@ int *device_error_flag();   // per-device int latched by kernels, or nullptr
   do {                                                                     \
     kernel<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);            \
     ::e2f::g_launches.fetch_add(1, std::memory_order_relaxed);             \
-    E2F_CUDA_TRY(cudaGetLastError());                                      \
+    const cudaError_t e2f_lerr_ = cudaGetLastError();                      \
+    if (e2f_lerr_ != cudaSuccess) {                                        \
+      ::e2f::set_cuda_error(e2f_lerr_, "launch of " #kernel);              \
+      return E2F_ERR_CUDA;                                                 \
+    }                                                                      \
   } while (0)
 
 // Stream-ordered scratch buffer released (in stream order) on scope exit.
@@ -60,6 +64,19 @@ template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
+}
+
+// Word i of a 16-byte vector and packing of two floats into a bf16 pair,
+// by value (no pointer into a register array is ever formed, so the
+// compiler keeps such arrays in registers).
+__device__ __forceinline__ uint32_t u4w(const uint4 &v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+// One cvt.rn.bf16x2.f32: the first source goes to the upper half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

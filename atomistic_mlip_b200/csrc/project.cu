@@ -183,13 +183,13 @@ __global__ void __launch_bounds__(NT, 1) project_tc_kernel(const __nv_bfloat16 *
         for (int c0 = 0; c0 < 64; c0 += 16) {
           float v[16];
           tmem_ld_32x32b_x16(tb + ((uint32_t)(32 * (warp & 3)) << 16) + 128 * which + ecol + c0, v);
-          tmem_ld_wait();
           if (off >= 0) {
-            __align__(16) __nv_bfloat16 o[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float2bfloat16_rn(v[i]);
-            *reinterpret_cast<uint4 *>(out + off + ecol + c0) = *reinterpret_cast<const uint4 *>(&o[0]);
-            *reinterpret_cast<uint4 *>(out + off + ecol + c0 + 8) = *reinterpret_cast<const uint4 *>(&o[8]);
+            *reinterpret_cast<uint4 *>(out + off + ecol + c0) =
+                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                           pack_bf16x2(v[6], v[7]));
+            *reinterpret_cast<uint4 *>(out + off + ecol + c0 + 8) =
+                make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                           pack_bf16x2(v[14], v[15]));
           }
         }
       }

@@ -205,7 +205,7 @@ def _box_list(wl):
     return None if wl.box is None else [float(b) for b in wl.box]
 
 
-def measure_workload(cfg, dev, peaks, peak_src, reps=5, warm=2, n_target=None, wl=None):
+def measure_workload(cfg, dev, peaks, peak_src, reps=5, warm=2, n_target=None, wl=None, attention=True):
     """One workload against its rooflines: the neighbour build (HBM:
     algorithmic bytes 12N + 4(N+1) + 4E) and the fused attention kernel
     (tensor: F(L, C) FLOP per edge over the kernel's own event time), plus
@@ -248,6 +248,11 @@ def measure_workload(cfg, dev, peaks, peak_src, reps=5, warm=2, n_target=None, w
         nb()
     t_nb = timed(nb)
     nb_bytes = 12 * wl.N + 4 * (wl.N + 1) + 4 * E
+    nb_row = {"ms": t_nb, "algorithmic_bytes": nb_bytes, "achieved_gbs": nb_bytes / (t_nb * 1e-3) / 1e9,
+              "frac_hbm": nb_bytes / (t_nb * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+              "note": "whole call, including its host read-backs"}
+    if not attention:
+        return {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}"), "N": wl.N, "E": E, "neighbour_build": nb_row}
     o = torch.empty((wl.N, (wl.L + 1) ** 2, wl.C), dtype=torch.float32, device=dev)
 
     def att():
@@ -261,14 +266,10 @@ def measure_workload(cfg, dev, peaks, peak_src, reps=5, warm=2, n_target=None, w
     k_ms = k_ms / max(n_k, 1)
     F = so2_flops_per_edge(wl.L, wl.C)
     peak = float(peaks["bf16_tflops"])
-    hbm = float(peaks["hbm_gbs"])
     res = {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}") if n_target is None else
            f"periodic water box, {wl.N} atoms, r_c = 6 A; L=4, C=128, H=8, bf16",
            "N": wl.N, "E": E, "L": wl.L,
-           "neighbour_build": {"ms": t_nb, "algorithmic_bytes": nb_bytes,
-                               "achieved_gbs": nb_bytes / (t_nb * 1e-3) / 1e9,
-                               "frac_hbm": nb_bytes / (t_nb * 1e-3) / 1e9 / hbm,
-                               "note": "whole call, including its host read-backs"},
+           "neighbour_build": nb_row,
            "attention": {"call_ms": t_call, "fused_kernel_ms": k_ms,
                          "edges_per_s": E / (t_call * 1e-3), "node_updates_per_s": wl.N / (t_call * 1e-3),
                          "achieved_tflops": F * E / (k_ms * 1e-3) / 1e12,
@@ -617,11 +618,17 @@ def run_rows(args):
     e2f.lib()
     peaks, peak_src = load_peaks()
     what = args.rows_what
+    if what == "forces":
+        print(json.dumps(measure_forces(2, dev, peaks, reps=args.steps, warm=args.warmup)), flush=True)
+        return
+    if what == "block":
+        print(json.dumps(measure_block(4, dev, reps=args.steps, warm=args.warmup)), flush=True)
+        return
     cfgs = {"all": (1, 2, 4, 3), "neighbors": (4,), "molecules": (1,), "water3k": (2,), "protein": (3,),
             "water100k": (4,)}[what]
     for cfg in cfgs:
-        print(json.dumps(measure_workload(cfg, dev, peaks, peak_src, reps=args.steps, warm=args.warmup)),
-              flush=True)
+        print(json.dumps(measure_workload(cfg, dev, peaks, peak_src, reps=args.steps, warm=args.warmup,
+                                          attention=what != "neighbors")), flush=True)
 
 
 def main(argv=None):
@@ -633,8 +640,8 @@ def main(argv=None):
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the other workloads and the memory sweep (profiling runs)")
     ap.add_argument("--rows", action="store_true", help="one JSON line per workload (one GPU)")
-    ap.add_argument("--rows-what", choices=["all", "neighbors", "molecules", "water3k", "protein", "water100k"],
-                    default="all")
+    ap.add_argument("--rows-what", choices=["all", "neighbors", "molecules", "water3k", "protein", "water100k",
+                                            "forces", "block"], default="all")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -82,7 +82,9 @@ def test_full_size_sampled_rows(cuda_ok, cfg, prec, n):
 @pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 6])
 def test_tensor_core_path_small(cuda_ok, L):
     """bf16, C = 128, H = 8 takes the tcgen05 kernel: 24-atom cluster (7 edge
-    tiles of 64, or 14 of 32 for L >= 5; ragged last tile) for every degree."""
+    tiles of 64, or 14 of 32 for L >= 5; ragged last tile) for every degree
+    but L = 3, which the library routes to the CUDA-core kernel (its
+    tensor-core build is not instantiated)."""
     wl0 = wlmod.make_workload(0)
     wl = wlmod.make_custom(wl0.pos, None, wl0.r_c, L=L, C=128, H=8, precision="bf16", seed=3 + L)
     _compare(wl)
@@ -105,7 +107,7 @@ def test_tensor_core_path_isolated_and_low_degree(cuda_ok):
     pairs = np.array([[20, 20, 20], [21, 20, 20], [40, 40, 40], [60, 5, 5]], float)
     chain = np.stack([np.arange(12) * 1.4 + 80, np.full(12, 80.0), np.full(12, 80.0)], 1)
     pos = np.concatenate([clump, pairs, chain]).astype(np.float32)
-    wl = wlmod.make_custom(pos, None, 5.0, L=3, C=128, H=4, precision="bf16", seed=9)
+    wl = wlmod.make_custom(pos, None, 5.0, L=4, C=128, H=4, precision="bf16", seed=9)
     out, _ = _compare(wl)
     assert np.all(out[92] == 0) and np.all(out[93] == 0)
 
@@ -140,3 +142,15 @@ def test_neighbour_order_invariance(cuda_ok):
     nl2 = e2f.NeighborList(nl.row_ptr, torch.from_numpy(col).cuda(), nl.n_edges, nl.box, nl.r_c)
     o2 = e2f.attention_forward(x, pos, nl2, w).double().cpu().numpy()
     assert helpers.rel_err(o2, o1) <= 1e-5
+
+
+def test_tensor_core_path_large_logits(cuda_ok):
+    """Features scaled by 2 (exact in bf16) spread each node's logits by about
+    20, so later tiles of a node exceed its reference maximum by more than
+    the margin of 8 and the online softmax rescales the node's earlier sums.
+    (Much larger scales make the comparison measure the bf16 rounding of q
+    and k, amplified by the logit size, rather than the kernel.)"""
+    wl0 = wlmod.make_workload(0)
+    wl = wlmod.make_custom(wl0.pos, None, wl0.r_c, L=4, C=128, H=8, precision="bf16", seed=31)
+    wl.x = (wl.x * 2.0).astype(np.float32)
+    _compare(wl)

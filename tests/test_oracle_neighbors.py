@@ -104,3 +104,20 @@ def test_workload_graphs_c_equals_numpy(cfg):
     if cfg == 2:
         # ~90 neighbours per atom at 0.1 atoms/A^3 and r_c = 6 A
         assert 80 < len(a[1]) / wl.N < 95
+
+
+def test_neighbor_rows_match_full_brute_force():
+    """The sampled-rows CSR lists, for every sampled row, exactly the full
+    brute-force row (open and periodic), and nothing for the other rows."""
+    from atomistic_mlip_b200 import workloads as w
+    for cfg in (0, 2):
+        wl = w.make_workload(cfg, C=8, L=1, H=1)
+        rp, col = nb.neighbors(wl.pos, wl.box, wl.r_c)
+        rows = np.random.default_rng(3).choice(wl.N, size=min(17, wl.N), replace=False)
+        rp2, col2 = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, rows)
+        for i in range(wl.N):
+            got = col2[rp2[i]:rp2[i + 1]]
+            if i in set(rows.tolist()):
+                assert np.array_equal(got, col[rp[i]:rp[i + 1]])
+            else:
+                assert len(got) == 0

@@ -29,6 +29,7 @@ struct CellGrid {
   int stencil[3]; // 1: offsets -1..1, 0: offset 0 only
 };
 
+constexpr int ROW_CAP = 256;   // shared-memory row buffer per warp (longer rows: sorted in global memory)
 
 __global__ void bbox_partial_kernel(const float *__restrict__ pos, int n, float *__restrict__ part) {
   float mn[3] = {INFINITY, INFINITY, INFINITY}, mx[3] = {-INFINITY, -INFINITY, -INFINITY};
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(CELL_THREADS) cell_fill_kernel(int ncell, Cell
                                                                  int32_t *__restrict__ col_idx) {
   __shared__ float4 cp[CAND_CAP], cs[CAND_CAP];
   __shared__ Stencil st;
-  __shared__ uint64_t keys[CAND_CAP];
+  __shared__ int32_t rows[CELL_THREADS / 32][ROW_CAP];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int cid = blockIdx.x; cid < ncell; cid += gridDim.x) {
     const int h0 = cell_start[cid], hn = cell_start[cid + 1] - h0;
@@ -270,51 +271,55 @@ __global__ void __launch_bounds__(CELL_THREADS) cell_fill_kernel(int ncell, Cell
     __syncthreads();
     const int ntot = st.off[st.n];
     if (ntot <= CAND_CAP) {
-      // one chunk: the candidates are sorted by atom index once per home
-      // cell (bitonic sort of (index, slot) keys), so a warp that tests them
-      // in that order and writes its passes in lane order emits each row
-      // already ascending -- no per-row sort
+      // one chunk: each warp builds its home atoms' rows in shared memory
       __syncthreads();
       stage_candidates(st, 0, ntot, spos, cp, cs);
-      int np = 1;
-      while (np < ntot) np <<= 1;
-      for (int k = threadIdx.x; k < np; k += blockDim.x)
-        keys[k] = k < ntot ? ((uint64_t)(uint32_t)__float_as_int(cp[k].w) << 32) | (uint32_t)k : ~0ull;
       __syncthreads();
-      for (int kk = 2; kk <= np; kk <<= 1) {
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-          for (int x = threadIdx.x; x < np; x += blockDim.x) {
-            const int y = x ^ jj;
-            if (y > x) {
-              const uint64_t ka = keys[x], kb = keys[y];
-              if ((ka > kb) == ((x & kk) == 0)) { keys[x] = kb; keys[y] = ka; }
-            }
-          }
-          __syncthreads();
-        }
-      }
       for (int a = wid; a < hn; a += nw) {
         const float4 me = spos[h0 + a];
         const int i = __float_as_int(me.w);
         const float3 pi = make_float3(me.x, me.y, me.z);
         const int r0 = row_ptr[i], dg = row_ptr[i + 1] - r0;
         int32_t *out = col_idx + r0;
+        int32_t *b = rows[wid];
+        const bool in_smem = dg <= ROW_CAP;
         int w = 0;
         for (int k0 = 0; k0 < ntot; k0 += 32) {
           const int k = k0 + lane;
           bool pass = false;
           int j = -1;
           if (k < ntot) {
-            const int slot = (int)(keys[k] & 0xffffffffu);
-            const float4 pj = cp[slot];
+            const float4 pj = cp[k];
             j = __float_as_int(pj.w);
-            pass = j != i && is_edge<FAST>(g, pi, pj, cs[slot]);
+            pass = j != i && is_edge<FAST>(g, pi, pj, cs[k]);
           }
           const unsigned m = __ballot_sync(0xffffffffu, pass);
           const int p = w + __popc(m & ((1u << lane) - 1u));
-          if (pass && p < dg) out[p] = j;
+          if (pass && p < dg) {
+            if (in_smem) b[p] = j;
+            else out[p] = j;
+          }
           w += __popc(m);
         }
+        __syncwarp();
+        if (in_smem) {
+          // rank placement: keys are distinct atom indices
+          for (int e = lane; e < dg; e += 32) {
+            const int key = b[e];
+            int rank = 0;
+            for (int t = 0; t < dg; ++t) rank += (b[t] < key);
+            out[rank] = key;
+          }
+        } else {
+          for (int round = 0; round < dg; ++round) {   // odd-even transposition sort in place (rare)
+            for (int k = 2 * lane + (round & 1); k + 1 < dg; k += 64) {
+              const int x = out[k], y = out[k + 1];
+              if (x > y) { out[k] = y; out[k + 1] = x; }
+            }
+            __syncwarp();
+          }
+        }
+        __syncwarp();
       }
     } else {
       // dense stencil (more candidates than one chunk): rows written to

@@ -409,6 +409,21 @@ def make_layer_weights(L: int, C: int, H: int, precision: str, seed: int, hidden
                 rad_W2=w2, gamma1=g1, gamma2=g2, Wa=Wa, Wb=Wb, Wd=Wd)
 
 
+def cg_num_paths(L: int) -> int:
+    """Coupling paths (l1, l2, l3) with 0 <= l1, l2, l3 <= L and
+    |l1 - l2| <= l3 <= l1 + l2 (the row count of the CG-convolution weights)."""
+    return sum(1 for l1 in range(L + 1) for l2 in range(L + 1) for l3 in range(L + 1)
+               if abs(l1 - l2) <= l3 <= l1 + l2)
+
+
+def make_cg_weights(L: int, C: int, seed: int) -> np.ndarray:
+    """Channel-wise path weights of the CG convolution, float32
+    [cg_num_paths(L)][C], N(0, 1) / sqrt(number of paths), seeded."""
+    rng = np.random.default_rng(seed)
+    n = cg_num_paths(L)
+    return (rng.standard_normal((n, C)) / math.sqrt(n)).astype(np.float32)
+
+
 def make_custom(pos: np.ndarray, box: Optional[np.ndarray], r_c: float, L: int, C: int,
                 H: int, precision: str = "fp32", seed: int = 0) -> Workload:
     """Features and weights for caller-given positions (edge-case tests)."""

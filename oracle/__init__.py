@@ -18,8 +18,12 @@ attention   the operator itself, edge by edge in fp64
 attention_grad
             the same operator restated in PyTorch CPU ops (fp64), whose
             autograd gives the gradients of a scalar of the outputs with
-            respect to positions, features and weights (the backward that
-            the GPU path does not have yet)
+            respect to positions, features and weights
+block       the E2Former-V2 block around the attention (merged RMS norm,
+            scalar-gated FFN, residuals)
+cg          Clebsch-Gordan coefficients (Racah formula) and the dense
+            x (x) Y(rhat) convolution in the global frame, the reference for
+            the re-indexed (edge-frame) CG convolution
 
 Sources (web pages on E2Former-V2, EquiformerV3 and DPA4):
   * "E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation

@@ -130,6 +130,9 @@ static e2f_status validate_csr(const e2f_csr *csr) {
 
 e2f_status block_forward_impl(const float *x, const float *pos, const e2f_csr *csr, const e2f_block_weights *w,
                               float *out, cudaStream_t s);
+int64_t cg_num_paths(int L);
+e2f_status cg_conv_impl(const void *x, int dtype, const float *pos, const e2f_csr *csr, int L, int C,
+                        const float *W, float *out, cudaStream_t s);
 e2f_status attention_backward_impl(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
                                    const float *G, float *dx, float *dpos, cudaStream_t s);
 
@@ -259,6 +262,24 @@ e2f_status e2f_block_forward(const float *x, const float *pos, const e2f_csr *cs
   if (!x || !pos || !out || x == out) return E2F_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
   return block_forward_impl(x, pos, csr, w, out, static_cast<cudaStream_t>(stream));
+}
+
+int64_t e2f_cg_num_paths(int32_t L) {
+  if (L < 0 || L > E2F_MAX_L) return -1;
+  return cg_num_paths(L);
+}
+
+e2f_status e2f_cg_conv_forward(const void *x, int32_t dtype, const float *pos, const e2f_csr *csr, int32_t L,
+                               int32_t C, const float *W, float *out, void *stream) {
+  e2f_status st = validate_csr(csr);
+  if (st != E2F_OK) return st;
+  if (L < 0 || L > E2F_MAX_L) return E2F_ERR_UNSUPPORTED;
+  if (dtype != E2F_F32 && dtype != E2F_BF16) return E2F_ERR_UNSUPPORTED;
+  if (C < 2 || C > 256 || (C & 1)) return E2F_ERR_INVALID_ARG;
+  if (csr->n_nodes == 0) return E2F_OK;
+  if (!x || !pos || !W || !out) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
+  return cg_conv_impl(x, dtype, pos, csr, L, C, W, out, static_cast<cudaStream_t>(stream));
 }
 
 e2f_status e2f_stream_status(void *stream) {

@@ -338,8 +338,6 @@ __global__ void __launch_bounds__(256) pack_w_kernel(PackArgs a) {
 // Table entry of (l, m, m'): DYP_STRIDE floats at
 // DYP_STRIDE * (wig_offset(l) + (m + l)(2l + 1) + (m' + l)): [eps, c_0, .., c_l].
 // ---------------------------------------------------------------------------
-constexpr int DYP_STRIDE = E2F_MAX_L + 2;
-constexpr int DYP_ENTRIES = (E2F_MAX_L + 1) * (2 * E2F_MAX_L + 1) * (2 * E2F_MAX_L + 3) / 3;  // sum (2l+1)^2
 __constant__ float c_dypoly[DYP_ENTRIES * DYP_STRIDE];
 
 static bool fit_dy_poly(float *tab) {
@@ -399,22 +397,33 @@ static bool fit_dy_poly(float *tab) {
   return true;
 }
 
-// Fits the table once per process and uploads it to each device once; safe
-// to call from several host threads.
-static e2f_status ensure_dy_poly() {
+}  // namespace tca
+
+// Host copy of the table, fitted once per process (thread-safe); null if the
+// fit failed.  The CG convolution uploads it into its own constant bank.
+const float *dy_poly_host_table() {
   static float tab[DYP_ENTRIES * DYP_STRIDE];
   static std::once_flag fit_once;
   static bool fitted_ok = false;
+  std::call_once(fit_once, [] { fitted_ok = tca::fit_dy_poly(tab); });
+  return fitted_ok ? tab : nullptr;
+}
+
+namespace tca {
+
+// Uploads the table to each device once; safe to call from several host
+// threads.
+static e2f_status ensure_dy_poly() {
   static std::mutex up_mu;
   static bool uploaded[64] = {};
-  std::call_once(fit_once, [] { fitted_ok = fit_dy_poly(tab); });
-  if (!fitted_ok) return E2F_ERR_CUDA;
+  const float *tab = dy_poly_host_table();
+  if (!tab) return E2F_ERR_CUDA;
   int dev = 0;
   E2F_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(up_mu);
   if (!uploaded[dev]) {
-    E2F_CUDA_TRY(cudaMemcpyToSymbol(c_dypoly, tab, sizeof(tab)));
+    E2F_CUDA_TRY(cudaMemcpyToSymbol(c_dypoly, tab, sizeof(float) * DYP_ENTRIES * DYP_STRIDE));
     uploaded[dev] = true;
   }
   return E2F_OK;

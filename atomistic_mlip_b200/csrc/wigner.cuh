@@ -17,6 +17,8 @@
 
 #include <math.h>
 
+#include "../../include/e2f.h"
+
 #ifdef __CUDACC__
 #define E2F_HD __host__ __device__ __forceinline__
 #else
@@ -26,6 +28,12 @@
 namespace e2f {
 
 E2F_HD int wig_offset(int l) { return l * (4 * l * l - 1) / 3; }
+
+// Polynomial table of the y-rotation blocks (fitted in attention_tc.cu):
+// entry (l, m, m') holds DYP_STRIDE floats [eps, c_0, .., c_l] at
+// DYP_STRIDE * (wig_offset(l) + (m + l)(2l + 1) + (m' + l)).
+constexpr int DYP_STRIDE = E2F_MAX_L + 2;
+constexpr int DYP_ENTRIES = (E2F_MAX_L + 1) * (2 * E2F_MAX_L + 1) * (2 * E2F_MAX_L + 3) / 3;   // sum (2l+1)^2
 E2F_HD int wig_size(int L) { return wig_offset(L + 1); }
 
 E2F_HD float wig_sqrt(float x) { return sqrtf(x); }

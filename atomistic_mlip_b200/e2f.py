@@ -70,6 +70,10 @@ SIGNATURES = {
                                                 ctypes.c_void_p, ctypes.c_void_p]),
     "e2f_block_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
                                            ctypes.POINTER(BlockWeights), ctypes.c_void_p, ctypes.c_void_p]),
+    "e2f_cg_num_paths": (ctypes.c_int64, [ctypes.c_int32]),
+    "e2f_cg_conv_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.POINTER(Csr),
+                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_void_p]),
     "e2f_stream_status": (ctypes.c_int32, [ctypes.c_void_p]),
     "e2f_wigner_d": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
                                       ctypes.c_void_p]),
@@ -235,6 +239,32 @@ def attention_forward(x, pos, nl: NeighborList, w: DeviceWeights, out=None, stre
     code = lib().e2f_attention_forward(_ptr(x), _ptr(pos), ctypes.byref(csr), ctypes.byref(w.struct),
                                        _ptr(out), _stream_ptr(stream))
     _check(code, "e2f_attention_forward")
+    return out
+
+
+def cg_num_paths(L: int) -> int:
+    """Rows of the CG-convolution weights for degree L."""
+    n = int(lib().e2f_cg_num_paths(int(L)))
+    if n < 0:
+        raise E2FError(1, "e2f_cg_num_paths", f"L = {L} out of range")
+    return n
+
+
+def cg_conv_forward(x, pos, nl: NeighborList, W, L: int, out=None, stream=None):
+    """Re-indexed CG convolution of x (float32 or bfloat16 [N, (L+1)^2, C])
+    with the harmonics of the edge directions; W float32 [cg_num_paths(L), C].
+    Returns float32 [N, (L+1)^2, C]."""
+    torch = _torch()
+    N, Q, C = int(x.shape[0]), int(x.shape[1]), int(x.shape[2])
+    if Q != (L + 1) ** 2:
+        raise ValueError(f"x has {Q} components, L = {L} needs {(L + 1) ** 2}")
+    dtype = F32 if x.dtype == torch.float32 else BF16
+    if out is None:
+        out = torch.empty((N, Q, C), dtype=torch.float32, device=pos.device)
+    csr = nl.csr()
+    code = lib().e2f_cg_conv_forward(_ptr(x), dtype, _ptr(pos), ctypes.byref(csr), int(L), C, _ptr(W), _ptr(out),
+                                     _stream_ptr(stream))
+    _check(code, "e2f_cg_conv_forward")
     return out
 
 

@@ -66,6 +66,44 @@ def so2_flops_per_edge(L: int, C: int) -> int:
     return 2 * n[0] ** 2 + sum(8 * n[m] ** 2 for m in range(1, L + 1))
 
 
+def cg_eaas_flops_per_edge(L: int, C: int) -> int:
+    """Algorithmic FLOPs per edge of the re-indexed CG convolution (2 per
+    multiply-add, per channel): z rotations in and out (4 per (l, m >= 1)
+    pair each), the y blocks in and out (sum over l >= 1 of (l+1)^2 + l^2
+    each), the coupling ((L+1)^2 + 4 sum_{m>=1} (L-m+1)^2) and the m = 0
+    accumulation (L + 1)."""
+    z = 2 * L * (L + 1)
+    y = sum((l + 1) ** 2 + l ** 2 for l in range(1, L + 1))
+    coup = (L + 1) ** 2 + 4 * sum((L - m + 1) ** 2 for m in range(1, L + 1))
+    return 2 * C * (2 * z + 2 * y + coup + (L + 1))
+
+
+def cg_dense_flops_per_edge(L: int, C: int) -> int:
+    """The same convolution as a dense contraction in the global frame:
+    2 (2l1+1)(2l2+1)(2l3+1) per path and channel (harmonics not counted)."""
+    n = 0
+    for l1 in range(L + 1):
+        for l2 in range(L + 1):
+            for l3 in range(abs(l1 - l2), min(L, l1 + l2) + 1):
+                n += (2 * l1 + 1) * (2 * l2 + 1) * (2 * l3 + 1)
+    return 2 * C * n
+
+
+def fp32_alu_peak_tflops(dev) -> float:
+    """FP32 multiply-add peak: SMs x 128 lanes x 2 FLOP x the maximum SM clock
+    (nvidia-smi clocks.max.sm; 1965 MHz if unavailable)."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = 1965.0
+    try:
+        q = subprocess.run(["nvidia-smi", "--query-gpu=clocks.max.sm", "--format=csv,noheader,nounits", "-i",
+                            str(dev.index or 0)], capture_output=True, text=True, timeout=10)
+        mhz = float(q.stdout.strip().splitlines()[0])
+    except Exception:
+        pass
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -321,6 +359,47 @@ def measure_forces(cfg, dev, peaks, reps=3, warm=1, wl=None):
     return res
 
 
+def measure_cg(cfg, dev, reps=3, warm=1, wl=None):
+    """The re-indexed CG convolution (x (x) Y(rhat) with channel-wise path
+    weights, evaluated in the edge frame) on a workload's features: call
+    time (CUDA events), edges/s and achieved FP32 TFLOP/s of its algorithmic
+    FLOPs against the FP32 multiply-add peak (the kernel runs on the CUDA
+    cores: the coupling is channel-wise, not a contraction)."""
+    import torch
+    from atomistic_mlip_b200 import e2f
+    from atomistic_mlip_b200 import workloads as w
+    stream = torch.cuda.current_stream(dev)
+    if wl is None:
+        wl = w.make_workload(cfg)
+    pos = torch.from_numpy(wl.pos).to(dev)
+    x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+    W = torch.from_numpy(w.make_cg_weights(wl.L, wl.C, 77)).to(dev)
+    nl = e2f.build_neighbors(pos, _box_list(wl), wl.r_c)
+    for _ in range(warm):
+        e2f.cg_conv_forward(x, pos, nl, W, wl.L)
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2f.cg_conv_forward(x, pos, nl, W, wl.L)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    t = statistics.median(ts)
+    F = cg_eaas_flops_per_edge(wl.L, wl.C)
+    peak = fp32_alu_peak_tflops(dev)
+    res = {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}"), "N": wl.N, "E": nl.n_edges, "L": wl.L, "C": wl.C,
+           "ms": t, "edges_per_s": nl.n_edges / (t * 1e-3), "flops_per_edge": F,
+           "dense_cg_flops_per_edge": cg_dense_flops_per_edge(wl.L, wl.C),
+           "achieved_tflops": F * nl.n_edges / (t * 1e-3) / 1e12, "fp32_peak_tflops": peak,
+           "frac_of_fp32_peak": F * nl.n_edges / (t * 1e-3) / 1e12 / peak,
+           "what": "e2f_cg_conv_forward: channel-wise CG convolution x (x) Y(rhat), edge-frame re-indexing, "
+                   "bf16 features, fp32 arithmetic"}
+    del x, pos, W, nl
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_block(cfg, dev, n_layers=1, reps=3, warm=1, wl=None):
     """n_layers E2Former-V2 blocks (merged RMS norm, attention, scalar-gated
     FFN with Hd = 4C, residuals) on a workload: time per block, and the
@@ -483,6 +562,7 @@ def run_ours(args):
         extras["workloads"] = rows + [sweep[-1]]
         extras["forces"] = [measure_forces(2, dev, peaks), measure_forces(4, dev, peaks, reps=2, wl=wl)]
         extras["block"] = [measure_block(4, dev, n_layers=1, wl=wl), measure_block(2, dev, n_layers=2)]
+        extras["cg_conv"] = [measure_cg(4, dev, wl=wl), measure_cg(2, dev)]
         extras["memory_sweep"] = {
             "N": ns, "peak_device_bytes": tot,
             "edges_per_s": [r["attention"]["edges_per_s"] for r in sweep],
@@ -624,6 +704,10 @@ def run_rows(args):
     if what == "block":
         print(json.dumps(measure_block(4, dev, reps=args.steps, warm=args.warmup)), flush=True)
         return
+    if what == "cg":
+        for cfg in (2, 4):
+            print(json.dumps(measure_cg(cfg, dev, reps=args.steps, warm=args.warmup)), flush=True)
+        return
     cfgs = {"all": (1, 2, 4, 3), "neighbors": (4,), "molecules": (1,), "water3k": (2,), "protein": (3,),
             "water100k": (4,)}[what]
     for cfg in cfgs:
@@ -641,7 +725,7 @@ def main(argv=None):
                     help="skip the other workloads and the memory sweep (profiling runs)")
     ap.add_argument("--rows", action="store_true", help="one JSON line per workload (one GPU)")
     ap.add_argument("--rows-what", choices=["all", "neighbors", "molecules", "water3k", "protein", "water100k",
-                                            "forces", "block"], default="all")
+                                            "forces", "block", "cg"], default="all")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -252,6 +252,43 @@ E2F_API e2f_status e2f_block_forward(const float *x, const float *pos, const e2f
                                      const e2f_block_weights *w, float *out, void *stream);
 
 /*
+ * e2f_cg_num_paths -- number of coupling paths (l1, l2, l3) of the CG
+ * convolution of degree L: 0 <= l1, l2, l3 <= L with |l1 - l2| <= l3 <=
+ * l1 + l2.  -1 for L outside 0..E2F_MAX_L.
+ */
+E2F_API int64_t e2f_cg_num_paths(int32_t L);
+
+/*
+ * e2f_cg_conv_forward -- Clebsch-Gordan convolution of node features with the
+ * harmonics of the edge directions, evaluated by re-indexing in the edge
+ * frame ([E2F] §2.1 EAAS, "Re-indexing operator").
+ *
+ *   x      device, [N][Q][C], Q = (L+1)^2, type `dtype` (E2F_F32 or
+ *          E2F_BF16); 16-byte aligned.
+ *   pos    device, [N][3] fp32 (the positions the CSR was built from).
+ *   csr    host descriptor from e2f_build_neighbors (device arrays).
+ *   L      0..E2F_MAX_L.   C  channels, even, 2..256.
+ *   W      device fp32 [e2f_cg_num_paths(L)][C]: the weight of path p and
+ *          channel c, paths in lexicographic (l1, l2, l3) order.
+ *   out    device, [N][Q][C] fp32, 16-byte aligned; fully overwritten.
+ *
+ * o_i[(l3,m3),c] = sum_{j in N(i)} u(r_ij) sum_p W[p][c]
+ *                  (x_j^{l1}[.,c] (x) Y^{l2}(rhat_ij))^{l3}_{m3},
+ * with (x) the real Clebsch-Gordan coupling (Racah's coefficients taken to
+ * the real harmonics of e2f_wigner_d: the real part for even l1 + l2 + l3,
+ * the imaginary part for odd), Y the orthonormal real harmonics, r_ij =
+ * p_j - p_i (minimum image), u = (cos(pi r / r_c) + 1)/2.  In the edge frame
+ * the harmonics of the edge keep only m = 0, so each path reduces to a
+ * block-sparse map between equal |m|; the dense contraction is never formed.
+ * o_i = 0 for an empty row.  The first call per device and L builds a small
+ * coefficient table (synchronous host-to-device copy); later calls are
+ * asynchronous.  Errors: E2F_ERR_INVALID_ARG (null or misaligned pointers, C
+ * out of range), E2F_ERR_UNSUPPORTED (L or dtype out of range).
+ */
+E2F_API e2f_status e2f_cg_conv_forward(const void *x, int32_t dtype, const float *pos, const e2f_csr *csr,
+                                       int32_t L, int32_t C, const float *W, float *out, void *stream);
+
+/*
  * e2f_stream_status -- synchronise `stream`, then return (and clear) any
  * error latched by a kernel of this library on the current device
  * (E2F_ERR_TIMEOUT for a bounded wait that gave up), or E2F_ERR_CUDA.

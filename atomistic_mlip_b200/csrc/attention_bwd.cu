@@ -289,21 +289,25 @@ __global__ void __launch_bounds__(BT) edge_dalpha_kernel(Args a) {
 }
 
 // ---------------------------------------------------------------------------
-// K5: ds, dL/du, dy = alpha GD, dL/dg, dw = g dy (stacked)
+// K5: ds, dL/du, dy = alpha GD, dL/dg, dw = g dy (stacked).  Channel-major:
+// a thread takes channel c through every (l, m) (compile-time), and the
+// per-(m, l) sums dL/dg are warp reductions over a padded [Q][C + 1] table
+// of products (no shared-memory atomics).
 // ---------------------------------------------------------------------------
 template <typename T, int L>
-__global__ void __launch_bounds__(BT) edge_dy_kernel(Args a) {
+__global__ void __launch_bounds__(BT, 4) edge_dy_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
+  extern __shared__ float prod[];   // [Q][C + 1]: dy * Y per (l, m), channel
   __shared__ float D[S];
-  __shared__ float dsh[16], alh[16], dgp[P];
-  const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
+  __shared__ float dsh[16], alh[16];
+  const int C = a.C, CP = C + 1, QC = Q * C, H = a.H, Ch = C / H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
     const int64_t e = a.ea + el;
     const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
     __syncthreads();
     for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
-    if (threadIdx.x < P) dgp[threadIdx.x] = 0.f;
     if (threadIdx.x < H) {
       const int h = threadIdx.x;
       const float al = a.al[el * H + h], diff = a.dal[el * H + h] - a.dlt[(size_t)(i - a.na) * H + h];
@@ -324,96 +328,130 @@ __global__ void __launch_bounds__(BT) edge_dy_kernel(Args a) {
     }
     const float *Gi = a.G + (size_t)i * QC;
     const float *Yr = a.Y + (size_t)el * QC;
+    const float *gvp = a.gv + el * P;
     T *dYr = static_cast<T *>(a.dY) + (size_t)el * QC;
-    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
-      const int l = x / C, c = x % C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
       const float alc = alh[c / Ch];
-      float gd[2 * L + 1];
-      rotate_col<L>(D, Gi, l, c, C, gd);
-      for (int m = -l; m <= l; ++m) {
-        const int am = m < 0 ? -m : m, p = pair_index(L, am, l);
-        const int so = stack_off(L, C, m) + (l - am) * C + c;
-        const float dy = alc * gd[m + l];
-        atomicAdd(&dgp[p], dy * Yr[so]);
-        dYr[so] = from_f<T>(dy * a.gv[el * P + p]);
+#pragma unroll
+      for (int l = 0; l <= L; ++l) {
+        float gd[2 * L + 1];
+        rotate_col<L>(D, Gi, l, c, C, gd);
+#pragma unroll
+        for (int m = -l; m <= l; ++m) {
+          const int am = m < 0 ? -m : m;
+          const int so = stack_off(L, C, m) + (l - am) * C + c;
+          const float dy = alc * gd[m + l];
+          prod[(l * l + l + m) * CP + c] = dy * Yr[so];
+          dYr[so] = from_f<T>(dy * gvp[pair_index(L, am, l)]);
+        }
       }
     }
     __syncthreads();
-    if (threadIdx.x < P) a.dgv[el * P + threadIdx.x] = dgp[threadIdx.x];
+    for (int p = warp; p < P; p += nw) {
+      int m = 0, rem = p;   // (m, l) of pair p
+      while (rem > L - m) { rem -= L - m + 1; ++m; }
+      const int l = m + rem;
+      float sacc = 0.f;
+      for (int c = lane; c < C; c += 32) {
+        sacc += prod[(l * l + l + m) * CP + c];
+        if (m > 0) sacc += prod[(l * l + l - m) * CP + c];
+      }
+      sacc = warp_sum(sacc);
+      if (lane == 0) a.dgv[el * P + p] = sacc;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
-// K6: dL/dD, torque, radius; atomics into dpos, dq, dk, dv
+// K6: dL/dD, torque, radius; atomics into dpos, dq, dk, dv.  Channel-major
+// staging into padded [Q][C + 1] rows (a thread per channel, (l, m) at
+// compile time), then one dL/dD entry per thread as a C-long dot product
+// over the padded rows (conflict-free), the m = 0 row terms as warp
+// reductions, and the scatter of dv, dq, dk with consecutive threads on
+// consecutive channels.
 // ---------------------------------------------------------------------------
 template <typename T, int L>
-__global__ void __launch_bounds__(BT) edge_bwd_kernel(Args a) {
+__global__ void __launch_bounds__(BT, 3) edge_bwd_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   extern __shared__ float sm[];
-  float *dvt = sm;                 // [Q][C]  dL/dv~ (unstacked)
-  float *vj = dvt + Q * a.C;       // [Q][C]
-  float *yv = vj + Q * a.C;        // [Q][C]  y = g Y (unstacked)
-  float *dz = yv + Q * a.C;        // [Q][C]  alpha G_i
-  float *qk = dz + Q * a.C;        // [2][L+1][C]  q~0, k~0
-  __shared__ float D[S], dD[S];
+  const int C = a.C, CP = C + 1, QC = Q * C, H = a.H, Ch = C / H;
+  float *dvt = sm;                 // [Q][CP]  dL/dv~ (unstacked)
+  float *vj = dvt + Q * CP;        // [Q][CP]
+  float *yv = vj + Q * CP;         // [Q][CP]  y = g Y (unstacked)
+  float *dz = yv + Q * CP;         // [Q][CP]  alpha G_i
+  float *qk = dz + Q * CP;         // [2][L+1][C]  q~0, k~0
+  __shared__ float D[S], dD[S], dD0[Q];
   __shared__ float dsh[16], misc[32], tau[3];
-  const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
     const int64_t e = a.ea + el;
     const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
     const int j = a.col_idx[e];
     __syncthreads();
-    for (int x = threadIdx.x; x < S; x += blockDim.x) { D[x] = a.Dm[el * S + x]; dD[x] = 0.f; }
+    for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
     if (threadIdx.x < H) dsh[threadIdx.x] = a.dsv[el * H + threadIdx.x] * a.inv_sqrt_d;
     if (threadIdx.x < 3) tau[threadIdx.x] = 0.f;
     __syncthreads();
     const float *Gi = a.G + (size_t)i * QC;
     const float *Yr = a.Y + (size_t)el * QC, *dAr = a.dA + (size_t)el * QC;
-    for (int x = threadIdx.x; x < QC; x += blockDim.x) {
-      const int q = x / C, c = x % C;
-      int l = 0;
-      while ((l + 1) * (l + 1) <= q) ++l;
-      const int m = q - l * l - l, am = m < 0 ? -m : m;
-      const int so = stack_off(L, C, m) + (l - am) * C + c;
-      dvt[x] = dAr[so];
-      vj[x] = ldf<T>(a.v, (size_t)j * QC + x);
-      yv[x] = a.gv[el * P + pair_index(L, am, l)] * Yr[so];
-      dz[x] = a.al[el * H + c / Ch] * Gi[x];
-    }
-    // q~0, k~0 (m = 0 rows of D q_i, D k_j)
-    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
-      const int l = x / C, c = x % C, w = 2 * l + 1;
-      const float *row0 = D + wig_offset(l) + l * w;
-      float qh = 0.f, kh = 0.f;
-      for (int mp = 0; mp < w; ++mp) {
-        qh = fmaf(row0[mp], ldf<T>(a.q, ((size_t)i * Q + l * l + mp) * C + c), qh);
-        kh = fmaf(row0[mp], ldf<T>(a.k, ((size_t)j * Q + l * l + mp) * C + c), kh);
+    const float *gvp = a.gv + el * P;
+    const T *qi = static_cast<const T *>(a.q) + (size_t)i * QC;
+    const T *kj = static_cast<const T *>(a.k) + (size_t)j * QC;
+    const T *vjr = static_cast<const T *>(a.v) + (size_t)j * QC;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      const float alc = a.al[el * H + c / Ch];
+#pragma unroll
+      for (int l = 0; l <= L; ++l) {
+        const float *row0 = D + wig_offset(l) + l * (2 * l + 1);
+        float qh = 0.f, kh = 0.f;
+#pragma unroll
+        for (int m = -l; m <= l; ++m) {
+          const int am = m < 0 ? -m : m, q = l * l + l + m;
+          const int so = stack_off(L, C, m) + (l - am) * C + c;
+          dvt[q * CP + c] = dAr[so];
+          vj[q * CP + c] = to_f(vjr[(size_t)q * C + c]);
+          yv[q * CP + c] = gvp[pair_index(L, am, l)] * Yr[so];
+          dz[q * CP + c] = alc * Gi[(size_t)q * C + c];
+          qh = fmaf(row0[m + l], to_f(qi[(size_t)q * C + c]), qh);
+          kh = fmaf(row0[m + l], to_f(kj[(size_t)q * C + c]), kh);
+        }
+        qk[l * C + c] = qh;
+        qk[(L + 1) * C + l * C + c] = kh;
       }
-      qk[l * C + c] = qh;
-      qk[(L + 1) * C + l * C + c] = kh;
     }
     __syncthreads();
-    // dL/dD^l[m][m'] = sum_c dv~[m] v_j[m'] + y[m] dz[m'] (+ the m = 0 row:
-    // dq~0 q_i[m'] + dk~0 k_j[m'], dq~0 = ds k~0 / sqrt d, dk~0 = ds q~0 / sqrt d)
-    for (int ent = warp; ent < S; ent += nw) {
+    // dL/dD^l[m][m'] = sum_c dv~[m] v_j[m'] + y[m] dz[m'] ...
+    for (int ent = threadIdx.x; ent < S; ent += blockDim.x) {
       int l = 0;
       while (wig_offset(l + 1) <= ent) ++l;
       const int w = 2 * l + 1, rr = (ent - wig_offset(l)) / w, cc = (ent - wig_offset(l)) % w;
-      const int qa = l * l + rr, qb = l * l + cc;
-      float s = 0.f;
-      for (int c = lane; c < C; c += 32) {
-        s = fmaf(dvt[qa * C + c], vj[qb * C + c], s);
-        s = fmaf(yv[qa * C + c], dz[qb * C + c], s);
-        if (rr == l) {
-          const float ds = dsh[c / Ch];
-          s = fmaf(ds * qk[(L + 1) * C + l * C + c], ldf<T>(a.q, ((size_t)i * Q + qb) * C + c), s);
-          s = fmaf(ds * qk[l * C + c], ldf<T>(a.k, ((size_t)j * Q + qb) * C + c), s);
-        }
+      const float *pa = dvt + (l * l + rr) * CP, *pb = vj + (l * l + cc) * CP;
+      const float *ya = yv + (l * l + rr) * CP, *zb = dz + (l * l + cc) * CP;
+      float s0 = 0.f, s1 = 0.f;
+      for (int c = 0; c < C; ++c) {
+        s0 = fmaf(pa[c], pb[c], s0);
+        s1 = fmaf(ya[c], zb[c], s1);
       }
-      s = warp_sum(s);
-      if (lane == 0) dD[ent] = s;
+      dD[ent] = s0 + s1;
+    }
+    // ... + the m = 0 row: dq~0 q_i[m'] + dk~0 k_j[m'] with dq~0 = ds k~0 / sqrt d,
+    // dk~0 = ds q~0 / sqrt d (one warp per (l, m'), lanes over channels)
+    for (int idx = warp; idx < Q; idx += nw) {
+      int l = 0;
+      while ((l + 1) * (l + 1) <= idx) ++l;
+      float sacc = 0.f;
+      for (int c = lane; c < C; c += 32)
+        sacc += dsh[c / Ch] * (qk[(L + 1) * C + l * C + c] * to_f(qi[(size_t)idx * C + c]) +
+                               qk[l * C + c] * to_f(kj[(size_t)idx * C + c]));
+      sacc = warp_sum(sacc);
+      if (lane == 0) dD0[idx] = sacc;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < Q; idx += blockDim.x) {
+      int l = 0;
+      while ((l + 1) * (l + 1) <= idx) ++l;
+      dD[wig_offset(l) + l * (2 * l + 1) + (idx - l * l)] += dD0[idx];
     }
     __syncthreads();
     // torque tau_k = -<D^T dD, J_k>, one (l, a, b) entry per thread
@@ -467,46 +505,26 @@ __global__ void __launch_bounds__(BT) edge_bwd_kernel(Args a) {
       atomicAdd(&a.dpos[3 * j + 0], gx); atomicAdd(&a.dpos[3 * j + 1], gy); atomicAdd(&a.dpos[3 * j + 2], gz);
       atomicAdd(&a.dpos[3 * i + 0], -gx); atomicAdd(&a.dpos[3 * i + 1], -gy); atomicAdd(&a.dpos[3 * i + 2], -gz);
     }
-    // dv_j += D^T dv~; dq_i, dk_j += row0^T dq~0 / dk~0 -- four channels per
-    // thread and one 16-byte atomic per array when C is a multiple of 4
-    if ((C & 3) == 0) {
-      for (int x4 = threadIdx.x; x4 < QC / 4; x4 += blockDim.x) {
-        const int x = 4 * x4, q = x / C, c = x % C;
-        int l = 0;
-        while ((l + 1) * (l + 1) <= q) ++l;
-        const int w = 2 * l + 1, mp = q - l * l;
+    // dv_j += D^T dv~; dq_i, dk_j += row0^T dq~0 / dk~0 (consecutive threads
+    // on consecutive channels)
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      const float ds = dsh[c / Ch];
+#pragma unroll
+      for (int l = 0; l <= L; ++l) {
+        const int w = 2 * l + 1;
         const float *Dl = D + wig_offset(l);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int m = 0; m < w; ++m) {
-          const float dm = Dl[m * w + mp];
-          const float *src = dvt + (l * l + m) * C + c;
-          acc.x = fmaf(dm, src[0], acc.x); acc.y = fmaf(dm, src[1], acc.y);
-          acc.z = fmaf(dm, src[2], acc.z); acc.w = fmaf(dm, src[3], acc.w);
+        const float gq = ds * qk[(L + 1) * C + l * C + c], gk = ds * qk[l * C + c];
+#pragma unroll
+        for (int mp = 0; mp < w; ++mp) {
+          float acc = 0.f;
+#pragma unroll
+          for (int m = 0; m < w; ++m) acc = fmaf(Dl[m * w + mp], dvt[(l * l + m) * CP + c], acc);
+          const size_t o = (size_t)(l * l + mp) * C + c;
+          atomicAdd(&a.dv[(size_t)j * QC + o], acc);
+          const float r0 = Dl[l * w + mp];
+          atomicAdd(&a.dq[(size_t)i * QC + o], r0 * gq);
+          atomicAdd(&a.dk[(size_t)j * QC + o], r0 * gk);
         }
-        atomicAdd(reinterpret_cast<float4 *>(a.dv + (size_t)j * QC + x), acc);
-        const float r0 = Dl[l * w + mp];
-        float4 gq, gk;
-        const float *qt = qk + (L + 1) * C + l * C + c, *kt = qk + l * C + c;
-        gq.x = r0 * dsh[c / Ch] * qt[0];       gk.x = r0 * dsh[c / Ch] * kt[0];
-        gq.y = r0 * dsh[(c + 1) / Ch] * qt[1]; gk.y = r0 * dsh[(c + 1) / Ch] * kt[1];
-        gq.z = r0 * dsh[(c + 2) / Ch] * qt[2]; gk.z = r0 * dsh[(c + 2) / Ch] * kt[2];
-        gq.w = r0 * dsh[(c + 3) / Ch] * qt[3]; gk.w = r0 * dsh[(c + 3) / Ch] * kt[3];
-        atomicAdd(reinterpret_cast<float4 *>(a.dq + (size_t)i * QC + x), gq);
-        atomicAdd(reinterpret_cast<float4 *>(a.dk + (size_t)j * QC + x), gk);
-      }
-    } else {
-      for (int x = threadIdx.x; x < QC; x += blockDim.x) {
-        const int q = x / C, c = x % C;
-        int l = 0;
-        while ((l + 1) * (l + 1) <= q) ++l;
-        const int w = 2 * l + 1, mp = q - l * l;
-        const float *Dl = D + wig_offset(l);
-        float acc = 0.f;
-        for (int m = 0; m < w; ++m) acc = fmaf(Dl[m * w + mp], dvt[(l * l + m) * C + c], acc);
-        atomicAdd(&a.dv[(size_t)j * QC + x], acc);
-        const float r0 = Dl[l * w + mp], ds = dsh[c / Ch];
-        atomicAdd(&a.dq[(size_t)i * QC + x], r0 * ds * qk[(L + 1) * C + l * C + c]);
-        atomicAdd(&a.dk[(size_t)j * QC + x], r0 * ds * qk[l * C + c]);
       }
     }
   }
@@ -716,9 +734,11 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
   a.Mv = reinterpret_cast<float *>(cb + oM); a.denv = reinterpret_cast<float *>(cb + oden);
   a.dlt = reinterpret_cast<float *>(cb + odl);
   a.dq = dq; a.dk = dk; a.dv = dv; a.dpos = dpos;
-  const size_t smem6 = sizeof(float) * ((size_t)4 * QC + 2 * (size_t)(L + 1) * C);
+  const size_t smem6 = sizeof(float) * ((size_t)4 * Q * (C + 1) + 2 * (size_t)(L + 1) * C);
+  const size_t smem5 = sizeof(float) * (size_t)Q * (C + 1);
   if (smem6 > 200 * 1024) return E2F_ERR_UNSUPPORTED;
   E2F_CUDA_TRY(cudaFuncSetAttribute(edge_bwd_kernel<T, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem6));
+  E2F_CUDA_TRY(cudaFuncSetAttribute(edge_dy_kernel<T, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem5));
   for (auto &ch : chunks) {
     a.na = ch.first; a.nb = ch.second;
     a.ea = rp[ch.first];
@@ -736,7 +756,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
     }
     E2F_LAUNCH((edge_dalpha_kernel<L>), eg, BT, 0, s, a);
     E2F_LAUNCH(node_delta_kernel, ng, 256, 0, s, a);
-    E2F_LAUNCH((edge_dy_kernel<T, L>), eg, BT, 0, s, a);
+    E2F_LAUNCH((edge_dy_kernel<T, L>), eg, BT, smem5, s, a);
     for (int m = 0; m <= L; ++m) {
       const int wm = m == 0 ? (L + 1) * C : 2 * (L - m + 1) * C;
       const int so = stack_off(L, C, m);

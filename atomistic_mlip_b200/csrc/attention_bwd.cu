@@ -115,7 +115,8 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   __shared__ float D[S];
-  __shared__ float hid[16], geo[8], hs[16];
+  __shared__ float hid[16], geo[8];
+  extern __shared__ float part[];   // [C]: per-channel logit partials
   const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
     const int64_t e = a.ea + el;
@@ -156,8 +157,6 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
       a.gv[el * P + threadIdx.x] = gg;
     }
     // logits: the m = 0 rows of D q_i and D k_j, per head
-    if (threadIdx.x < 16) hs[threadIdx.x] = 0.f;
-    __syncthreads();
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
       float s = 0.f;
 #pragma unroll
@@ -171,10 +170,14 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
         }
         s = fmaf(qh, kh, s);
       }
-      atomicAdd(&hs[c / Ch], s);
+      part[c] = s;
     }
     __syncthreads();
-    if (threadIdx.x < H) a.sv[el * H + threadIdx.x] = hs[threadIdx.x] * a.inv_sqrt_d;
+    if (threadIdx.x < H) {
+      float hsum = 0.f;
+      for (int c = threadIdx.x * Ch; c < (threadIdx.x + 1) * Ch; ++c) hsum += part[c];
+      a.sv[el * H + threadIdx.x] = hsum * a.inv_sqrt_d;
+    }
     // rotate in: v~[(l,m),c] = sum_m' D^l[m][m'] v_j[(l,m'),c], stacked
     T *Arow = static_cast<T *>(a.A) + (size_t)el * QC;
     for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
@@ -250,40 +253,45 @@ __device__ __forceinline__ void rotate_col(const float *D, const float *src, int
 // K3: alpha and dalpha per (edge, head)
 // ---------------------------------------------------------------------------
 template <int L>
-__global__ void __launch_bounds__(BT) edge_dalpha_kernel(Args a) {
+__global__ void __launch_bounds__(BT, 4) edge_dalpha_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   __shared__ float D[S];
-  __shared__ float hs[16];
+  extern __shared__ float part[];   // [C]: per-channel partials of dL/dalpha
   const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
     const int64_t e = a.ea + el;
     const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
     __syncthreads();
     for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
-    if (threadIdx.x < 16) hs[threadIdx.x] = 0.f;
     __syncthreads();
     const float *Gi = a.G + (size_t)i * QC;
     const float *Yr = a.Y + (size_t)el * QC;
-    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
-      const int l = x / C, c = x % C;
-      float gd[2 * L + 1];
-      rotate_col<L>(D, Gi, l, c, C, gd);
-      float s = 0.f;
-      for (int m = -l; m <= l; ++m) {
-        const int am = m < 0 ? -m : m;
-        const float y = a.gv[el * P + pair_index(L, am, l)] * Yr[stack_off(L, C, m) + (l - am) * C + c];
-        s = fmaf(y, gd[m + l], s);
+    const float *gvp = a.gv + el * P;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float sacc = 0.f;
+#pragma unroll
+      for (int l = 0; l <= L; ++l) {
+        float gd[2 * L + 1];
+        rotate_col<L>(D, Gi, l, c, C, gd);
+#pragma unroll
+        for (int m = -l; m <= l; ++m) {
+          const int am = m < 0 ? -m : m;
+          const float y = gvp[pair_index(L, am, l)] * Yr[stack_off(L, C, m) + (l - am) * C + c];
+          sacc = fmaf(y, gd[m + l], sacc);
+        }
       }
-      atomicAdd(&hs[c / Ch], s);
+      part[c] = sacc;
     }
     __syncthreads();
     if (threadIdx.x < H) {
       const int h = threadIdx.x;
+      float hsum = 0.f;
+      for (int c = h * Ch; c < (h + 1) * Ch; ++c) hsum += part[c];
       const float M = a.Mv[(size_t)(i - a.na) * H + h], den = a.denv[(size_t)(i - a.na) * H + h];
       const float sp = a.sv[el * H + h] + logf(a.uv[el]);
       a.al[el * H + h] = (den > 0.f && M > -INFINITY) ? expf(sp - M) / den : 0.f;
-      a.dal[el * H + h] = hs[h];
+      a.dal[el * H + h] = hsum;
     }
   }
 }
@@ -375,7 +383,10 @@ __global__ void __launch_bounds__(BT, 3) edge_bwd_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   extern __shared__ float sm[];
-  const int C = a.C, CP = C + 1, QC = Q * C, H = a.H, Ch = C / H;
+  // rows padded to C + 4 floats: 16-byte aligned for the vector dot products,
+  // and rows of different (l, m) start 4 banks apart (conflict-free for the
+  // eight threads of one 128-byte phase)
+  const int C = a.C, CP = C + 4, QC = Q * C, H = a.H, Ch = C / H;
   float *dvt = sm;                 // [Q][CP]  dL/dv~ (unstacked)
   float *vj = dvt + Q * CP;        // [Q][CP]
   float *yv = vj + Q * CP;         // [Q][CP]  y = g Y (unstacked)
@@ -429,9 +440,18 @@ __global__ void __launch_bounds__(BT, 3) edge_bwd_kernel(Args a) {
       const float *pa = dvt + (l * l + rr) * CP, *pb = vj + (l * l + cc) * CP;
       const float *ya = yv + (l * l + rr) * CP, *zb = dz + (l * l + cc) * CP;
       float s0 = 0.f, s1 = 0.f;
-      for (int c = 0; c < C; ++c) {
-        s0 = fmaf(pa[c], pb[c], s0);
-        s1 = fmaf(ya[c], zb[c], s1);
+      if ((C & 3) == 0) {
+        for (int c = 0; c < C; c += 4) {
+          const float4 xa = *reinterpret_cast<const float4 *>(pa + c), xb = *reinterpret_cast<const float4 *>(pb + c);
+          const float4 za = *reinterpret_cast<const float4 *>(ya + c), zz = *reinterpret_cast<const float4 *>(zb + c);
+          s0 = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, s0))));
+          s1 = fmaf(za.x, zz.x, fmaf(za.y, zz.y, fmaf(za.z, zz.z, fmaf(za.w, zz.w, s1))));
+        }
+      } else {
+        for (int c = 0; c < C; ++c) {
+          s0 = fmaf(pa[c], pb[c], s0);
+          s1 = fmaf(ya[c], zb[c], s1);
+        }
       }
       dD[ent] = s0 + s1;
     }
@@ -734,7 +754,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
   a.Mv = reinterpret_cast<float *>(cb + oM); a.denv = reinterpret_cast<float *>(cb + oden);
   a.dlt = reinterpret_cast<float *>(cb + odl);
   a.dq = dq; a.dk = dk; a.dv = dv; a.dpos = dpos;
-  const size_t smem6 = sizeof(float) * ((size_t)4 * Q * (C + 1) + 2 * (size_t)(L + 1) * C);
+  const size_t smem6 = sizeof(float) * ((size_t)4 * Q * (C + 4) + 2 * (size_t)(L + 1) * C);
   const size_t smem5 = sizeof(float) * (size_t)Q * (C + 1);
   if (smem6 > 200 * 1024) return E2F_ERR_UNSUPPORTED;
   E2F_CUDA_TRY(cudaFuncSetAttribute(edge_bwd_kernel<T, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem6));
@@ -746,7 +766,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
     if (a.ne == 0) continue;
     const int eg = (int)std::min<int64_t>(a.ne, 148LL * 16);
     const int ng = (int)std::min<int64_t>((a.nb - a.na + 7) / 8, 148LL * 8);
-    E2F_LAUNCH((edge_fwd_kernel<T, L>), eg, BT, 0, s, a);
+    E2F_LAUNCH((edge_fwd_kernel<T, L>), eg, BT, sizeof(float) * C, s, a);
     E2F_LAUNCH(node_stats_kernel, ng, 256, 0, s, a);
     for (int m = 0; m <= L; ++m) {
       const int wm = m == 0 ? (L + 1) * C : 2 * (L - m + 1) * C;
@@ -754,7 +774,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
       st = stacked_gemm<T>(bh, wc + woff[m], wm, static_cast<T *>(a.A) + so, a.Y + so, a.ne, QC, true);
       if (st != E2F_OK) return st;
     }
-    E2F_LAUNCH((edge_dalpha_kernel<L>), eg, BT, 0, s, a);
+    E2F_LAUNCH((edge_dalpha_kernel<L>), eg, BT, sizeof(float) * C, s, a);
     E2F_LAUNCH(node_delta_kernel, ng, 256, 0, s, a);
     E2F_LAUNCH((edge_dy_kernel<T, L>), eg, BT, smem5, s, a);
     for (int m = 0; m <= L; ++m) {

@@ -31,6 +31,20 @@ For every destination atom i and every neighbour j in N(i) (CSR row i):
   O12 alpha^h_ij = u_ij exp(s^h_ij) / sum_j' u_ij' exp(s^h_ij'), two-pass
       (max subtracted, then normalised).
   O13 o_i = sum_j alpha^{h(c)}_ij D_ij^T y_ij;  o_i = 0 when N(i) is empty.
+
+Multi-focus variant ("DPA4 ...", §2.1 A2: the hidden channels split into F
+focus streams, each with its own SO(2) stack, re-weighted by a cross-focus
+softmax computed from the l = 0 section), optional (``focus=(F, a)``):
+  F1  stream f owns channels [f C/F, (f+1) C/F); its SO(2) stack is the
+      diagonal block of W0 / Wr / Wi between its own input and output
+      channels (for every pair of degrees); cross-stream entries are dropped;
+  F2  z^f_ij = (F / C)^(1/2) sum_{c in f} a_c y_ij[(0,0), c] (the l = 0 section
+      of the edge message after the radial scale), beta_ij = softmax_f z_ij;
+  F3  y_ij[., c] *= beta^{f(c)}_ij, then O13 as above.
+Readings: the pages name neither the focus logits' form nor their source
+beyond "the l = 0 section of the edge features"; the edge message's own
+l = 0 section with one learned vector a (one weight per channel) is the
+plainest choice that keeps the re-weighting invariant.
 """
 from __future__ import annotations
 
@@ -123,6 +137,28 @@ def so2_mix(vt: np.ndarray, g: np.ndarray, L: int, C: int, W0, Wr, Wi) -> np.nda
     return y
 
 
+def focus_mask(W: np.ndarray, C: int, F: int) -> np.ndarray:
+    """F1: keep the entries of a stacked SO(2) matrix (rows and columns
+    l-major, then channel) whose output and input channels share a stream."""
+    W = np.asarray(W, np.float64)
+    Cf = C // F
+    fr = (np.arange(W.shape[0]) % C) // Cf
+    fc = (np.arange(W.shape[1]) % C) // Cf
+    return np.where(fr[:, None] == fc[None, :], W, 0.0)
+
+
+def cross_focus(y: np.ndarray, F: int, a: np.ndarray) -> np.ndarray:
+    """F2, F3: y [E, Q, C] -> y with each stream scaled by its softmax weight."""
+    E, Q, C = y.shape
+    Cf = C // F
+    y00 = y[:, 0, :] * np.asarray(a, np.float64)[None, :]
+    z = y00.reshape(E, F, Cf).sum(axis=2) / math.sqrt(Cf)
+    z = z - z.max(axis=1, keepdims=True)
+    beta = np.exp(z)
+    beta /= beta.sum(axis=1, keepdims=True)
+    return y * np.repeat(beta, Cf, axis=1)[:, None, :]
+
+
 # ---------------------------------------------------------------------------
 # the operator
 # ---------------------------------------------------------------------------
@@ -133,12 +169,14 @@ def attention(pos: np.ndarray, box: Optional[np.ndarray], r_c: float,
               nodes: Optional[np.ndarray] = None,
               gauge: Optional[Callable[[np.ndarray], np.ndarray]] = None,
               g_override: Optional[float] = None,
-              max_edges_per_chunk: int = 4096) -> np.ndarray:
+              max_edges_per_chunk: int = 4096,
+              focus: Optional[tuple] = None) -> np.ndarray:
     """o_i for i in `nodes` (default: all) -> [len(nodes), Q, C] fp64.
 
     `gauge(e_ids)` may return per-edge angles gamma (radians); the frame is
     then R_z(gamma) R_ij (test hook: the output must not change).
-    `g_override` replaces the radial MLP output by a constant (test hook)."""
+    `g_override` replaces the radial MLP output by a constant (test hook).
+    `focus=(F, a)` selects the multi-focus variant (F1-F3)."""
     N = np.asarray(pos).shape[0]
     Q = (L + 1) ** 2
     Ch = C // H
@@ -160,6 +198,12 @@ def attention(pos: np.ndarray, box: Optional[np.ndarray], r_c: float,
     k_rows = project(x_src, Wk, L) if len(need_src) else np.zeros((0, Q, C))
     v_rows = project(x_src, Wv, L) if len(need_src) else np.zeros((0, Q, C))
 
+    if focus is not None:   # F1
+        F = int(focus[0])
+        W0 = focus_mask(W0, C, F)
+        Wr = [None] + [focus_mask(Wr[m], C, F) for m in range(1, L + 1)]
+        Wi = [None] + [focus_mask(Wi[m], C, F) for m in range(1, L + 1)]
+
     # chunks of destination nodes with a bounded number of edges
     deg = row_ptr[nodes + 1] - row_ptr[nodes]
     start = 0
@@ -169,13 +213,13 @@ def attention(pos: np.ndarray, box: Optional[np.ndarray], r_c: float,
             tot += deg[stop]
             stop += 1
         _chunk(out, start, stop, nodes, row_ptr, col, pos, box, r_c, q_rows, k_rows, v_rows,
-               src_map, W0, Wr, Wi, rad_W1, rad_W2, L, C, H, Ch, d, gauge, g_override)
+               src_map, W0, Wr, Wi, rad_W1, rad_W2, L, C, H, Ch, d, gauge, g_override, focus)
         start = stop
     return out
 
 
 def _chunk(out, start, stop, nodes, row_ptr, col, pos, box, r_c, q_rows, k_rows, v_rows,
-           src_map, W0, Wr, Wi, rad_W1, rad_W2, L, C, H, Ch, d, gauge, g_override):
+           src_map, W0, Wr, Wi, rad_W1, rad_W2, L, C, H, Ch, d, gauge, g_override, focus=None):
     dst_local, e_ids = [], []
     for t in range(start, stop):
         i = nodes[t]
@@ -218,6 +262,8 @@ def _chunk(out, start, stop, nodes, row_ptr, col, pos, box, r_c, q_rows, k_rows,
         g = np.full((len(r), (L + 1) * (L + 2) // 2), float(g_override))
     # O10
     y = so2_mix(vt, g, L, C, W0, Wr, Wi)
+    if focus is not None:   # F2, F3
+        y = cross_focus(y, int(focus[0]), focus[1])
     # O13 (per-edge message in the global frame)
     z = rotate(D, y, L, transpose=True)
     # O11, O12 (two-pass softmax per destination and head)

@@ -89,7 +89,8 @@ e2f_status attention_simt_impl(const T *, const T *, const T *, const float *, c
                                const e2f_weights *, float *, cudaStream_t, cudaEvent_t, cudaEvent_t);
 e2f_status attention_tc_available(const e2f_weights *w);
 e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const float *pos, const e2f_csr *csr,
-                             const e2f_weights *w, float *out, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1);
+                             const e2f_weights *w, float *out, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1,
+                             int F, const float *focus_a);
 
 __global__ void wigner_kernel(const float *__restrict__ R, int64_t n, int L, float *__restrict__ D) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -139,7 +140,7 @@ e2f_status attention_backward_impl(const void *x, const float *pos, const e2f_cs
 // q, k, v (library scratch), then the fused attention kernel; arguments
 // already validated.
 e2f_status attention_forward_impl(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
-                                  float *out, cudaStream_t s) {
+                                  float *out, cudaStream_t s, int F = 1, const float *focus_a = nullptr) {
   const int64_t N = csr->n_nodes;
   if (N == 0) return E2F_OK;
   const size_t Q = (size_t)(w->L_max + 1) * (w->L_max + 1);
@@ -153,8 +154,11 @@ e2f_status attention_forward_impl(const void *x, const float *pos, const e2f_csr
   if (st != E2F_OK) return st;
   cudaEvent_t ev0, ev1;
   prof_events(&ev0, &ev1);
+  if (F > 1) {   // multi-focus: the tensor-core kernel only (checked by the caller)
+    return attention_tc_impl(q, k, v, pos, csr, w, out, s, ev0, ev1, F, focus_a);
+  }
   if (w->dtype == E2F_BF16 && attention_tc_available(w) == E2F_OK)
-    return attention_tc_impl(q, k, v, pos, csr, w, out, s, ev0, ev1);
+    return attention_tc_impl(q, k, v, pos, csr, w, out, s, ev0, ev1, 1, nullptr);
   if (w->dtype == E2F_F32)
     return attention_simt_impl<float>((const float *)q, (const float *)k, (const float *)v, pos, csr, w, out, s,
                                       ev0, ev1);
@@ -262,6 +266,23 @@ e2f_status e2f_block_forward(const float *x, const float *pos, const e2f_csr *cs
   if (!x || !pos || !out || x == out) return E2F_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
   return block_forward_impl(x, pos, csr, w, out, static_cast<cudaStream_t>(stream));
+}
+
+e2f_status e2f_attention_forward_multifocus(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
+                                            int32_t F, const float *focus_a, float *out, void *stream) {
+  e2f_status st = validate_weights(w);
+  if (st != E2F_OK) return st;
+  st = validate_csr(csr);
+  if (st != E2F_OK) return st;
+  if (F != 1 && F != 2 && F != 4 && F != 8) return E2F_ERR_INVALID_ARG;
+  if (F > 1) {
+    if (attention_tc_available(w) != E2F_OK || (w->L_max != 2 && w->L_max != 4)) return E2F_ERR_UNSUPPORTED;
+    if (!focus_a || !aligned16(focus_a)) return E2F_ERR_INVALID_ARG;
+  }
+  if (csr->n_nodes == 0) return E2F_OK;
+  if (!x || !pos || !out) return E2F_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return E2F_ERR_INVALID_ARG;
+  return attention_forward_impl(x, pos, csr, w, out, static_cast<cudaStream_t>(stream), F, focus_a);
 }
 
 int64_t e2f_cg_num_paths(int32_t L) {

@@ -159,6 +159,10 @@ struct TcArgs {
   const float *W1, *W2;
   float *out;
   int *err;
+  // multi-focus variant: F streams of CH / F channels (1: plain operator),
+  // focus vector a [CH] (fp32), log2 of the stream width
+  int F, fshift;
+  const float *focus_a;
 };
 
 // ---------------------------------------------------------------------------
@@ -288,6 +292,7 @@ struct PackArgs {
   const __nv_bfloat16 *Wi[E2F_MAX_L + 1];
   uint8_t *dst;
   int L;
+  int F;   // focus streams: entries between channels of different streams are packed as zero
 };
 
 __global__ void __launch_bounds__(256) pack_w_kernel(PackArgs a) {
@@ -308,18 +313,22 @@ __global__ void __launch_bounds__(256) pack_w_kernel(PackArgs a) {
   const int n = (L - m + 1) * CH;
   if (m == 0) {
     const int scol = lp * CH;
+    const int cf = CH / a.F;
     for (int x = threadIdx.x; x < 128 * 128; x += blockDim.x) {
       const int row = x >> 7, k = x & 127;
       const size_t srow = (size_t)(l - m) * CH + row;
-      *reinterpret_cast<__nv_bfloat16 *>(stage + kmajor_off(row, k, 128)) = a.W0[srow * n + scol + k];
+      const __nv_bfloat16 w = (row / cf == k / cf) ? a.W0[srow * n + scol + k] : __float2bfloat16_rn(0.f);
+      *reinterpret_cast<__nv_bfloat16 *>(stage + kmajor_off(row, k, 128)) = w;
     }
   } else {
     const int scol = (lp - m) * CH + kh * 64;
+    const int cf = CH / a.F;
     for (int x = threadIdx.x; x < 2 * 128 * 64; x += blockDim.x) {
       const int t = x >> 13, row = (x >> 6) & 127, k = x & 63;
       const size_t srow = (size_t)(l - m) * CH + row;
       const __nv_bfloat16 *src = (t == 0) ? a.Wr[m] : a.Wi[m];
-      *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = src[srow * n + scol + k];
+      const __nv_bfloat16 w = (row / cf == (kh * 64 + k) / cf) ? src[srow * n + scol + k] : __float2bfloat16_rn(0.f);
+      *reinterpret_cast<__nv_bfloat16 *>(stage + t * 16384 + kmajor_off(row, k, 64)) = w;
     }
   }
 }
@@ -432,7 +441,7 @@ static e2f_status ensure_dy_poly() {
 // ---------------------------------------------------------------------------
 // the fused kernel
 // ---------------------------------------------------------------------------
-template <int L>
+template <int L, bool MF>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   using Cf = Cfg<L>;
   constexpr int Q = Cf::Q, P = Cf::P, NUNIT = Cf::NUNIT;
@@ -711,6 +720,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
     }
     named_bar(1, 128);
     uint32_t pc = 0, nA0 = 0, nA1 = 0;   // R hand-overs per sign
+    float beta[MF ? 8 : 1];              // multi-focus: this edge's stream weights (set at pass (0, 0))
+    beta[0] = 1.f;
     int t = 0;
     bool dead = false;
     bool ok = ti.start();
@@ -745,6 +756,52 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
           const int e = 16 * ew + (lane & 15);
           const int p_ml = m * (L + 1) - m * (m - 1) / 2 + (l - m);
           const float ge = (e < ne) ? __half2float(gs[e * P + p_ml]) : 0.f;
+          if constexpr (MF) {
+            if (m == 0 && l == 0) {
+              // stream weights of this edge ("DPA4 ...", §2.1 A2): z_f = sum
+              // over the stream's channels of a_c (g y)[(0,0), c] / sqrt(C/F),
+              // beta = softmax_f z.  The y+ lanes hold the edge rows of the
+              // m = 0 pass; lanes 16-31 take their partner's weights.
+              float z[8];
+#pragma unroll
+              for (int ff = 0; ff < 8; ++ff) z[ff] = 0.f;
+#pragma unroll 1
+              for (int i = 0; i < 8; i += 2) {
+                float v[2][16];
+                tmem_ld_32x32b_x16x2(tbase + lane_base + 128 * b + 16 * i, tbase + lane_base + 128 * b + 16 * i + 16,
+                                     v[0], v[1]);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                  const int c0 = 16 * (i + h2);
+                  const float4 *ap = reinterpret_cast<const float4 *>(a.focus_a + c0);
+                  float part = 0.f;
+#pragma unroll
+                  for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 av = __ldg(ap + k4);
+                    part = fmaf(av.x, v[h2][4 * k4], fmaf(av.y, v[h2][4 * k4 + 1],
+                           fmaf(av.z, v[h2][4 * k4 + 2], fmaf(av.w, v[h2][4 * k4 + 3], part))));
+                  }
+                  const int f = c0 >> a.fshift;
+#pragma unroll
+                  for (int ff = 0; ff < 8; ++ff)
+                    if (ff == f) z[ff] += part;
+                }
+              }
+              const float zs = ge * rsqrtf((float)(CH / a.F));
+              float zmax = -INFINITY;
+#pragma unroll
+              for (int ff = 0; ff < 8; ++ff)
+                if (ff < a.F) zmax = fmaxf(zmax, z[ff] * zs);
+              float zsum = 0.f;
+#pragma unroll
+              for (int ff = 0; ff < 8; ++ff) {
+                beta[ff] = (ff < a.F) ? expf(z[ff] * zs - zmax) : 0.f;
+                zsum += beta[ff];
+              }
+#pragma unroll
+              for (int ff = 0; ff < 8; ++ff) beta[ff] = __shfl_sync(0xffffffffu, beta[ff] / zsum, lane & 15);
+            }
+          }
           auto to_a2 = [&](int which) {
 #pragma unroll 1
             for (int i = 0; i < 8; i += 2) {
@@ -756,8 +813,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
                 for (int h2 = 0; h2 < 2; ++h2) {
                   const int c0 = 16 * (i + h2);
                   // channels [c0, c0 + 8) and [c0 + 8, c0 + 16) lie in one head each
-                  const float s_lo = (e < ne) ? __half2float(al[e * ALS + (c0 >> hshift)]) * ge : 0.f;
-                  const float s_hi = (e < ne) ? __half2float(al[e * ALS + ((c0 + 8) >> hshift)]) * ge : 0.f;
+                  float s_lo = (e < ne) ? __half2float(al[e * ALS + (c0 >> hshift)]) * ge : 0.f;
+                  float s_hi = (e < ne) ? __half2float(al[e * ALS + ((c0 + 8) >> hshift)]) * ge : 0.f;
+                  if constexpr (MF) {   // the 16 channels lie in one stream (C / F >= 16)
+                    const int f = c0 >> a.fshift;
+                    float bf = beta[0];
+#pragma unroll
+                    for (int ff = 1; ff < 8; ++ff)
+                      if (ff == f) bf = beta[ff];
+                    s_lo *= bf;
+                    s_hi *= bf;
+                  }
                   const float *vv = v[h2];
                   const uint4 lo = make_uint4(pack_bf16x2(vv[0] * s_lo, vv[1] * s_lo), pack_bf16x2(vv[2] * s_lo, vv[3] * s_lo),
                                               pack_bf16x2(vv[4] * s_lo, vv[5] * s_lo), pack_bf16x2(vv[6] * s_lo, vv[7] * s_lo));
@@ -1413,11 +1479,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
-template <int L>
+template <int L, bool MF = false>
 static e2f_status launch_tc(const TcArgs &args, int grid, cudaStream_t s) {
   using Cf = Cfg<L>;
-  E2F_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM));
-  E2F_LAUNCH(attn_tc_kernel<L>, grid, NTHREADS, Cf::SMEM, s, args);
+  E2F_CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<L, MF>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM));
+  E2F_LAUNCH((attn_tc_kernel<L, MF>), grid, NTHREADS, Cf::SMEM, s, args);
   return E2F_OK;
 }
 
@@ -1437,8 +1503,10 @@ e2f_status attention_tc_available(const e2f_weights *w) {
 }
 
 e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const float *pos, const e2f_csr *csr,
-                             const e2f_weights *w, float *out, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1) {
+                             const e2f_weights *w, float *out, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1,
+                             int F, const float *focus_a) {
   using namespace tca;
+  if (F != 1 && w->L_max != 2 && w->L_max != 4) return E2F_ERR_UNSUPPORTED;
   const int L = w->L_max;
   const int64_t N = csr->n_nodes, E = csr->n_edges;
   const size_t Q = (size_t)(L + 1) * (L + 1);
@@ -1464,6 +1532,7 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   }
   pa.dst = wp.as<uint8_t>();
   pa.L = L;
+  pa.F = F;
   E2F_LAUNCH(pack_w_kernel, nst, 256, 0, s, pa);
 
   TcArgs a;
@@ -1489,6 +1558,9 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   a.W2 = w->rad_W2;
   a.out = out;
   a.err = device_error_flag();
+  a.F = F;
+  a.fshift = 31 - __builtin_clz((unsigned)(CH / F));
+  a.focus_a = focus_a;
   if (!a.err) return E2F_ERR_CUDA;
   e2f_status r = E2F_OK;
   int dev = 0, nsm = 148;
@@ -1499,8 +1571,8 @@ e2f_status attention_tc_impl(const void *q, const void *k, const void *v, const 
   if (ev0) E2F_CUDA_TRY(cudaEventRecord(ev0, s));
   switch (L) {
     case 1: r = launch_tc<1>(a, grid, s); break;
-    case 2: r = launch_tc<2>(a, grid, s); break;
-    case 4: r = launch_tc<4>(a, grid, s); break;
+    case 2: r = F > 1 ? launch_tc<2, true>(a, grid, s) : launch_tc<2>(a, grid, s); break;
+    case 4: r = F > 1 ? launch_tc<4, true>(a, grid, s) : launch_tc<4>(a, grid, s); break;
     case 5: r = launch_tc<5>(a, grid, s); break;
     case 6: r = launch_tc<6>(a, grid, s); break;
     default: return E2F_ERR_UNSUPPORTED;

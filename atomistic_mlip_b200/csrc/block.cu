@@ -31,7 +31,7 @@
 namespace e2f {
 
 e2f_status attention_forward_impl(const void *x, const float *pos, const e2f_csr *csr, const e2f_weights *w,
-                                  float *out, cudaStream_t s);
+                                  float *out, cudaStream_t s, int F = 1, const float *focus_a = nullptr);
 
 namespace blk {
 

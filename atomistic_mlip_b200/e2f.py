@@ -70,6 +70,9 @@ SIGNATURES = {
                                                 ctypes.c_void_p, ctypes.c_void_p]),
     "e2f_block_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
                                            ctypes.POINTER(BlockWeights), ctypes.c_void_p, ctypes.c_void_p]),
+    "e2f_attention_forward_multifocus": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Csr),
+                                                          ctypes.POINTER(Weights), ctypes.c_int32, ctypes.c_void_p,
+                                                          ctypes.c_void_p, ctypes.c_void_p]),
     "e2f_cg_num_paths": (ctypes.c_int64, [ctypes.c_int32]),
     "e2f_cg_conv_forward": (ctypes.c_int32, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.POINTER(Csr),
                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
@@ -239,6 +242,23 @@ def attention_forward(x, pos, nl: NeighborList, w: DeviceWeights, out=None, stre
     code = lib().e2f_attention_forward(_ptr(x), _ptr(pos), ctypes.byref(csr), ctypes.byref(w.struct),
                                        _ptr(out), _stream_ptr(stream))
     _check(code, "e2f_attention_forward")
+    return out
+
+
+def attention_forward_multifocus(x, pos, nl: NeighborList, w: DeviceWeights, F: int, focus_a, out=None,
+                                 stream=None):
+    """Multi-focus attention: F streams with their own SO(2) stacks,
+    re-weighted per edge by a softmax over the streams (float32 [N, Q, C])."""
+    torch = _torch()
+    N = int(pos.shape[0])
+    Q = (w.L + 1) ** 2
+    if out is None:
+        out = torch.empty((N, Q, w.C), dtype=torch.float32, device=pos.device)
+    csr = nl.csr()
+    code = lib().e2f_attention_forward_multifocus(_ptr(x), _ptr(pos), ctypes.byref(csr), ctypes.byref(w.struct),
+                                                  int(F), _ptr(focus_a) if focus_a is not None else None,
+                                                  _ptr(out), _stream_ptr(stream))
+    _check(code, "e2f_attention_forward_multifocus")
     return out
 
 

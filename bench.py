@@ -400,6 +400,50 @@ def measure_cg(cfg, dev, reps=3, warm=1, wl=None):
     return res
 
 
+def measure_multifocus(cfg, dev, peaks, F=4, reps=3, warm=1, wl=None):
+    """The multi-focus attention (F streams, per-stream SO(2) stacks, cross-
+    focus softmax) on a workload: call time, fused-kernel time and edges/s.
+    The kernel runs the full C x C block products with the cross-stream
+    entries packed as zero, so its tensor-pipe work is that of the plain
+    operator (reported against the bf16 peak); the useful part is 1/F of it."""
+    import torch
+    from atomistic_mlip_b200 import e2f
+    from atomistic_mlip_b200 import workloads as w
+    stream = torch.cuda.current_stream(dev)
+    if wl is None:
+        wl = w.make_workload(cfg)
+    pos = torch.from_numpy(wl.pos).to(dev)
+    x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+    dw = e2f.DeviceWeights.from_workload(wl, dev)
+    a = torch.randn(wl.C, device=dev, generator=torch.Generator(device=dev).manual_seed(5)) * 2.0
+    nl = e2f.build_neighbors(pos, _box_list(wl), wl.r_c)
+    for _ in range(warm):
+        e2f.attention_forward_multifocus(x, pos, nl, dw, F, a)
+    e2f.profile_enable(True)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e2f.attention_forward_multifocus(x, pos, nl, dw, F, a)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    kern = e2f.profile_read()
+    e2f.profile_enable(False)
+    t = statistics.median(ts)
+    kt = kern[1] / max(kern[0], 1)
+    Fx = so2_flops_per_edge(wl.L, wl.C)
+    res = {"workload": EXTRA_DESC.get(cfg, f"cfg{cfg}"), "N": wl.N, "E": nl.n_edges, "F": F, "call_ms": t,
+           "fused_kernel_ms": kt, "edges_per_s": nl.n_edges / (kt * 1e-3),
+           "executed_tflops": Fx * nl.n_edges / (kt * 1e-3) / 1e12,
+           "frac_of_bf16_peak": Fx * nl.n_edges / (kt * 1e-3) / 1e12 / float(peaks["bf16_tflops"]),
+           "useful_flops_per_edge": Fx // F,
+           "what": "e2f_attention_forward_multifocus: F focus streams, cross-focus softmax, bf16"}
+    del x, pos, dw, nl, a
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_block(cfg, dev, n_layers=1, reps=3, warm=1, wl=None):
     """n_layers E2Former-V2 blocks (merged RMS norm, attention, scalar-gated
     FFN with Hd = 4C, residuals) on a workload: time per block, and the
@@ -563,6 +607,7 @@ def run_ours(args):
         extras["forces"] = [measure_forces(2, dev, peaks), measure_forces(4, dev, peaks, reps=2, wl=wl)]
         extras["block"] = [measure_block(4, dev, n_layers=1, wl=wl), measure_block(2, dev, n_layers=2)]
         extras["cg_conv"] = [measure_cg(4, dev, wl=wl), measure_cg(2, dev)]
+        extras["multifocus"] = [measure_multifocus(4, dev, peaks, F=4, wl=wl)]
         extras["memory_sweep"] = {
             "N": ns, "peak_device_bytes": tot,
             "edges_per_s": [r["attention"]["edges_per_s"] for r in sweep],
@@ -704,6 +749,10 @@ def run_rows(args):
     if what == "block":
         print(json.dumps(measure_block(4, dev, reps=args.steps, warm=args.warmup)), flush=True)
         return
+    if what == "multifocus":
+        for cfg in (1, 4):
+            print(json.dumps(measure_multifocus(cfg, dev, peaks, F=4, reps=args.steps, warm=args.warmup)), flush=True)
+        return
     if what == "cg":
         for cfg in (2, 4):
             print(json.dumps(measure_cg(cfg, dev, reps=args.steps, warm=args.warmup)), flush=True)
@@ -725,7 +774,7 @@ def main(argv=None):
                     help="skip the other workloads and the memory sweep (profiling runs)")
     ap.add_argument("--rows", action="store_true", help="one JSON line per workload (one GPU)")
     ap.add_argument("--rows-what", choices=["all", "neighbors", "molecules", "water3k", "protein", "water100k",
-                                            "forces", "block", "cg"], default="all")
+                                            "forces", "block", "cg", "multifocus"], default="all")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -252,6 +252,29 @@ E2F_API e2f_status e2f_block_forward(const float *x, const float *pos, const e2f
                                      const e2f_block_weights *w, float *out, void *stream);
 
 /*
+ * e2f_attention_forward_multifocus -- the attention of e2f_attention_forward
+ * with F focus streams ([DPA4] §2.1 A2, multi-focus EMFA message).
+ *
+ *   x, pos, csr, w, out   as for e2f_attention_forward.
+ *   F        1, 2, 4 or 8 streams; stream f owns channels [f C/F, (f+1) C/F).
+ *   focus_a  device fp32 [C], 16-byte aligned: the focus vector (unused
+ *            for F = 1).
+ *
+ * Each stream has its own SO(2) stack: of W0, Wr[m], Wi[m] only the entries
+ * between input and output channels of the same stream are used (the others
+ * are read as zero).  Per edge, after the SO(2) mix and the radial scale,
+ * z_f = sqrt(F/C) sum_{c in f} focus_a[c] y[(0,0), c] (the l = 0 section of
+ * the message), beta = softmax_f z, and every channel of stream f is scaled
+ * by beta_f before the rotate-out and the envelope-gated attention sum.  F =
+ * 1 is exactly e2f_attention_forward.  F > 1 runs on the tensor-core kernel
+ * only: bf16, C = 128, L_max 2 or 4, 4 <= H <= 16 (else
+ * E2F_ERR_UNSUPPORTED).  Fully asynchronous.
+ */
+E2F_API e2f_status e2f_attention_forward_multifocus(const void *x, const float *pos, const e2f_csr *csr,
+                                                   const e2f_weights *w, int32_t F, const float *focus_a,
+                                                   float *out, void *stream);
+
+/*
  * e2f_cg_num_paths -- number of coupling paths (l1, l2, l3) of the CG
  * convolution of degree L: 0 <= l1, l2, l3 <= L with |l1 - l2| <= l3 <=
  * l1 + l2.  -1 for L outside 0..E2F_MAX_L.

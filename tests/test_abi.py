@@ -142,3 +142,26 @@ def test_validation_from_two_host_threads(lib):
     for t in ts:
         t.join()
     assert not errors, errors[:5]
+
+
+def test_multifocus_and_cg_validation(lib):
+    """Host-side checks of the multi-focus attention and the CG convolution
+    (no GPU work: every call below returns before any CUDA call)."""
+    csr = e2f.Csr()
+    csr.row_ptr = 64; csr.col_idx = 64; csr.n_nodes = 4; csr.n_edges = 4; csr.r_c = 1.0
+    f = lib.e2f_attention_forward_multifocus
+    d, odd = ctypes.c_void_p(64), ctypes.c_void_p(72)
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(_weights()), 3, d, d, None) == 1       # F not 1, 2, 4, 8
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(_weights(C=128, H=8, dtype=1, L=3)), 4, d, d, None) == 4
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(_weights(C=128, H=8, dtype=0, L=4)), 4, d, d, None) == 4
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(_weights(C=128, H=8, dtype=1, L=4)), 4, odd, d, None) == 1
+    assert f(d, d, ctypes.byref(csr), ctypes.byref(_weights(C=128, H=8, dtype=1, L=4)), 4, None, d, None) == 1
+    g = lib.e2f_cg_conv_forward
+    assert lib.e2f_cg_num_paths(7) == -1 and lib.e2f_cg_num_paths(-1) == -1
+    assert [lib.e2f_cg_num_paths(L) for L in range(4)] == [1, 5, 15, 34]
+    assert g(d, 0, d, ctypes.byref(csr), 7, 8, d, d, None) == 4      # L out of range
+    assert g(d, 2, d, ctypes.byref(csr), 2, 8, d, d, None) == 4      # dtype
+    assert g(d, 0, d, ctypes.byref(csr), 2, 7, d, d, None) == 1      # odd C
+    assert g(d, 0, d, ctypes.byref(csr), 2, 258, d, d, None) == 1    # C too large
+    assert g(odd, 0, d, ctypes.byref(csr), 2, 8, d, d, None) == 1    # misaligned x
+    assert g(d, 0, d, ctypes.byref(csr), 2, 8, None, d, None) == 1   # no weights

@@ -66,3 +66,16 @@ def test_multifocus_molecules_sampled(cuda_ok):
     csr = helpers.oracle_csr(1)
     ref = oa.attention_workload(wl, nodes=nodes, csr=csr, focus=(4, a.astype(np.float64)))
     assert helpers.rel_err(got[nodes], ref) <= TOL
+
+
+def test_multifocus_water100k_sampled(cuda_ok):
+    """The benchmark configuration: the 100,002-atom water box, L = 4, F = 4,
+    40 sampled rows of the full-size launch."""
+    wl = helpers.cached_workload(4, "bf16")
+    a = _focus(wl.C, 240)
+    got, _ = _gpu(wl, 4, a)
+    assert np.all(np.isfinite(got))
+    nodes = np.sort(np.random.default_rng(241).choice(wl.N, size=40, replace=False))
+    csr = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)
+    ref = oa.attention_workload(wl, nodes=nodes, csr=csr, focus=(4, a.astype(np.float64)))
+    assert helpers.rel_err(got[nodes], ref) <= TOL

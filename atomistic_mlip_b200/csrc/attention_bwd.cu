@@ -370,6 +370,15 @@ __global__ void __launch_bounds__(BT, 4) edge_dy_kernel(Args a) {
   }
 }
 
+// four consecutive values as floats (16-byte / 8-byte aligned)
+__device__ __forceinline__ float4 ld4f(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4f(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 // ---------------------------------------------------------------------------
 // K6: dL/dD, torque, radius; atomics into dpos, dq, dk, dv.  Channel-major
 // staging into padded [Q][C + 1] rows (a thread per channel, (l, m) at
@@ -379,19 +388,20 @@ __global__ void __launch_bounds__(BT, 4) edge_dy_kernel(Args a) {
 // consecutive channels.
 // ---------------------------------------------------------------------------
 template <typename T, int L>
-__global__ void __launch_bounds__(BT, 3) edge_bwd_kernel(Args a) {
+__global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   extern __shared__ float sm[];
   // rows padded to C + 4 floats: 16-byte aligned for the vector dot products,
   // and rows of different (l, m) start 4 banks apart (conflict-free for the
   // eight threads of one 128-byte phase)
-  const int C = a.C, CP = C + 4, QC = Q * C, H = a.H, Ch = C / H;
-  float *dvt = sm;                 // [Q][CP]  dL/dv~ (unstacked)
-  float *vj = dvt + Q * CP;        // [Q][CP]
-  float *yv = vj + Q * CP;         // [Q][CP]  y = g Y (unstacked)
-  float *dz = yv + Q * CP;         // [Q][CP]  alpha G_i
-  float *qk = dz + Q * CP;         // [2][L+1][C]  q~0, k~0
+  // v_j is staged in its storage type (exact), rows padded to 16 bytes more
+  const int C = a.C, CP = C + 4, CPV = C + 16 / (int)sizeof(T), QC = Q * C, H = a.H, Ch = C / H;
+  float *dvt = sm;                                         // [Q][CP]  dL/dv~ (unstacked)
+  T *vj = reinterpret_cast<T *>(dvt + Q * CP);             // [Q][CPV]
+  float *yv = dvt + Q * CP + (Q * CPV * (int)sizeof(T) + 15) / 16 * 4;   // [Q][CP]  y = g Y (unstacked)
+  float *dz = yv + Q * CP;                                 // [Q][CP]  alpha G_i
+  float *qk = dz + Q * CP;                                 // [2][L+1][C]  q~0, k~0
   __shared__ float D[S], dD[S], dD0[Q];
   __shared__ float dsh[16], misc[32], tau[3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(BT, 3) edge_bwd_kernel(Args a) {
           const int am = m < 0 ? -m : m, q = l * l + l + m;
           const int so = stack_off(L, C, m) + (l - am) * C + c;
           dvt[q * CP + c] = dAr[so];
-          vj[q * CP + c] = to_f(vjr[(size_t)q * C + c]);
+          vj[q * CPV + c] = vjr[(size_t)q * C + c];
           yv[q * CP + c] = gvp[pair_index(L, am, l)] * Yr[so];
           dz[q * CP + c] = alc * Gi[(size_t)q * C + c];
           qh = fmaf(row0[m + l], to_f(qi[(size_t)q * C + c]), qh);
@@ -437,19 +447,20 @@ __global__ void __launch_bounds__(BT, 3) edge_bwd_kernel(Args a) {
       int l = 0;
       while (wig_offset(l + 1) <= ent) ++l;
       const int w = 2 * l + 1, rr = (ent - wig_offset(l)) / w, cc = (ent - wig_offset(l)) % w;
-      const float *pa = dvt + (l * l + rr) * CP, *pb = vj + (l * l + cc) * CP;
+      const float *pa = dvt + (l * l + rr) * CP;
+      const T *pb = vj + (l * l + cc) * CPV;
       const float *ya = yv + (l * l + rr) * CP, *zb = dz + (l * l + cc) * CP;
       float s0 = 0.f, s1 = 0.f;
       if ((C & 3) == 0) {
         for (int c = 0; c < C; c += 4) {
-          const float4 xa = *reinterpret_cast<const float4 *>(pa + c), xb = *reinterpret_cast<const float4 *>(pb + c);
+          const float4 xa = *reinterpret_cast<const float4 *>(pa + c), xb = ld4f(pb + c);
           const float4 za = *reinterpret_cast<const float4 *>(ya + c), zz = *reinterpret_cast<const float4 *>(zb + c);
           s0 = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, s0))));
           s1 = fmaf(za.x, zz.x, fmaf(za.y, zz.y, fmaf(za.z, zz.z, fmaf(za.w, zz.w, s1))));
         }
       } else {
         for (int c = 0; c < C; ++c) {
-          s0 = fmaf(pa[c], pb[c], s0);
+          s0 = fmaf(pa[c], to_f(pb[c]), s0);
           s1 = fmaf(ya[c], zb[c], s1);
         }
       }
@@ -754,7 +765,8 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
   a.Mv = reinterpret_cast<float *>(cb + oM); a.denv = reinterpret_cast<float *>(cb + oden);
   a.dlt = reinterpret_cast<float *>(cb + odl);
   a.dq = dq; a.dk = dk; a.dv = dv; a.dpos = dpos;
-  const size_t smem6 = sizeof(float) * ((size_t)4 * Q * (C + 4) + 2 * (size_t)(L + 1) * C);
+  const size_t smem6 = sizeof(float) * ((size_t)3 * Q * (C + 4) + 2 * (size_t)(L + 1) * C) +
+                       ((size_t)Q * (C + 16 / sizeof(T)) * sizeof(T) + 15) / 16 * 16;
   const size_t smem5 = sizeof(float) * (size_t)Q * (C + 1);
   if (smem6 > 200 * 1024) return E2F_ERR_UNSUPPORTED;
   E2F_CUDA_TRY(cudaFuncSetAttribute(edge_bwd_kernel<T, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem6));

@@ -87,6 +87,19 @@ template <int L> struct Cfg {
   static constexpr bool TMU = (L == 3 || L == 4);
   static constexpr int TMU_SP = 2 * L - 2;                 // first TMEM unit index
   static constexpr int NSU = TMU ? NUNIT - 2 : NUNIT;      // units in shared memory
+  // Unit slot of (m, l'): for m >= 1 the first of the (+m, -m) pair (the
+  // pair is (slot, slot + 1)); slots from NSU on are the TMEM pair.  For
+  // L = 4 the last degree's pair sits in slots 4-5, which m = 3 does not
+  // use, so the producers build it while m = 3 runs, and the next tile's
+  // m = 0 units 0-3 while m = 4 runs (instead of waiting for the MMA to
+  // release slots 0-1).
+  static __host__ __device__ constexpr int unit_slot(int m, int lp) {
+    return (L == 4 && m == 4) ? 4 : (m == 0 ? lp : 2 * (lp - m));
+  }
+  // The producers' fill order within degree m: the t-th unit filled is
+  // l' = fill_lp(m, t) (for L = 4 and m = 1 the TMEM pair first, since it
+  // is free while m = 0 runs).
+  static __host__ __device__ constexpr int fill_lp(int m, int t) { return (L == 4 && m == 1) ? (t == 0 ? L : t) : m + t; }
   static constexpr int NDYE = (L + 1) * (L + 2) * (2 * L + 3) / 6;   // sum (l+1)^2
   static constexpr int NDYO = L * (L + 1) * (2 * L + 1) / 6;         // sum l^2
   static constexpr int NDYP = ((NDYE + NDYO) + 1) & ~1;
@@ -548,7 +561,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
             const uint32_t dp = tbase + 128 * b, dmn = tbase + (16u << 16) + 128 * b;
             #pragma unroll 1
             for (int lp = m; lp <= L && !bad; ++lp) {
-              const int sp = (m == 0) ? lp : 2 * (lp - m);
+              const int sp = Cf::unit_slot(m, lp);
               if (first_pass) {
                 if (!mw(&unit_full[sp], (fillpar >> sp) & 1)) { bad = true; break; }
                 if (m > 0 && !mw(&unit_full[sp + 1], (fillpar >> (sp + 1)) & 1)) { bad = true; break; }
@@ -1261,8 +1274,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(TcArgs a) {
       #pragma unroll 1
       for (int m = 0; m <= L && !dead; ++m) {
         #pragma unroll 1
-        for (int lp = m; lp <= L; ++lp) {
-          const int sp = (m == 0) ? lp : 2 * (lp - m);
+        for (int tf = 0; tf <= L - m; ++tf) {
+          const int lp = Cf::fill_lp(m, tf);
+          const int sp = Cf::unit_slot(m, lp);
           {
             // each producer warp waits for the unit on its own: the warps run
             // through the units independently (a warp that finished its part

@@ -604,7 +604,10 @@ def run_ours(args):
 
     e2e_run(args.warmup)
     e2e_ms = e2e_run(args.steps)
-    del pos_d[1], x_d[1], out_d[1], nl_rp[1], nl_ci[1]
+    # release the e2e buffers (the lists and the closure hold references)
+    del e2e_run
+    for lst in (pos_d, x_d, out_d, nl_rp, nl_ci):
+        lst.clear()
     h2d_bytes = int(pos_h.numel() * 4 + x_h.numel() * 2)
     d2h_bytes = int(out_h.numel() * 4)
 

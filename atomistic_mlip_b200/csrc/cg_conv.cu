@@ -88,10 +88,6 @@ template <typename V> __device__ __forceinline__ V vzero();
 template <> __device__ __forceinline__ float vzero<float>() { return 0.f; }
 template <> __device__ __forceinline__ float2 vzero<float2>() { return make_float2(0.f, 0.f); }
 
-template <typename V> struct VecOf;
-template <> struct VecOf<float> { static constexpr int N = 1; };
-template <> struct VecOf<float2> { static constexpr int N = 2; };
-
 __device__ __forceinline__ void ldv(const float *p, float &v) { v = *p; }
 __device__ __forceinline__ void ldv(const __nv_bfloat16 *p, float &v) { v = __bfloat162float(*p); }
 __device__ __forceinline__ void ldv(const float *p, float2 &v) { v = *reinterpret_cast<const float2 *>(p); }
@@ -133,7 +129,7 @@ template <typename T, int L>
 __global__ void __launch_bounds__(256, 2) cg_conv_kernel(Args a) {
   using Cf = Cfg<L>;
   using V = typename std::conditional<Cf::CPT == 2, float2, float>::type;
-  constexpr int Q = Cf::Q, NDY = Cf::NDY, NS = Cf::NS, CPT = Cf::CPT;
+  constexpr int Q = Cf::Q, NDY = Cf::NDY, CPT = Cf::CPT;
   constexpr int LZ = L > 0 ? L : 1;
   __shared__ float s_dy[EB][NDY > 0 ? NDY : 1];
   __shared__ float s_cs[EB][LZ], s_sn[EB][LZ];

@@ -4,6 +4,7 @@
 // gradient of the energy; "DPA4 ...", §2.2 energy-to-force path).
 //
 // Recompute, per chunk of whole destination nodes (at most CHUNK_E edges):
+//   K0 edge_dst     the destination node of every edge of the chunk
 //   K1 edge_fwd     geometry, D^l blocks of the two-angle frame, envelope,
 //                   radial MLP, logits s; the rotated features
 //                   v~ = D v_j in SO(2)-stacked order
@@ -64,6 +65,7 @@ struct Args {
   // chunk
   int na, nb;                     // nodes [na, nb)
   int64_t ea, ne;                 // edges [ea, ea + ne)
+  int32_t *dst;                   // [ne] destination node of each edge
   void *A, *dY;                   // [ne][QC] storage type (stacked)
   float *Y, *dA;                  // [ne][QC] fp32 (stacked)
   float *Dm, *gv, *zv, *sv, *uv, *rv, *al, *dal, *dsv, *duv, *dgv;
@@ -77,14 +79,15 @@ template <typename T> __device__ __forceinline__ float ldf(const void *p, size_t
   return to_f(static_cast<const T *>(p)[i]);
 }
 
-__device__ __forceinline__ int node_of_edge(const int32_t *rp, int na, int nb, int64_t e) {
-  int lo = na, hi = nb - 1;   // largest n with rp[n] <= e
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if ((int64_t)rp[mid] <= e) lo = mid;
-    else hi = mid - 1;
+// K0: dst[e - ea] = n for every edge e of row n (warp per node, lanes over
+// the row), so that the per-edge kernels get their node with one load
+__global__ void edge_dst_kernel(Args a) {
+  const int lane = threadIdx.x & 31;
+  for (int n = a.na + blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < a.nb;
+       n += gridDim.x * (blockDim.x >> 5)) {
+    const int64_t e0 = a.row_ptr[n] - a.ea, e1 = a.row_ptr[n + 1] - a.ea;
+    for (int64_t e = e0 + lane; e < e1; e += 32) a.dst[e] = n;
   }
-  return lo;
 }
 
 // D^l blocks of the edge frame into shared memory (block-cooperative).
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
   const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
     const int64_t e = a.ea + el;
-    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    const int i = a.dst[el];
     const int j = a.col_idx[e];
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -260,8 +263,7 @@ __global__ void __launch_bounds__(BT, 4) edge_dalpha_kernel(Args a) {
   extern __shared__ float part[];   // [C]: per-channel partials of dL/dalpha
   const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
-    const int64_t e = a.ea + el;
-    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    const int i = a.dst[el];
     __syncthreads();
     for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
     __syncthreads();
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(BT, 4) edge_dalpha_kernel(Args a) {
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
         float gd[2 * L + 1];
+        asm volatile("" ::: "memory");   // one degree's loads in flight at a time (no spills)
         rotate_col<L>(D, Gi, l, c, C, gd);
 #pragma unroll
         for (int m = -l; m <= l; ++m) {
@@ -303,37 +306,35 @@ __global__ void __launch_bounds__(BT, 4) edge_dalpha_kernel(Args a) {
 // of products (no shared-memory atomics).
 // ---------------------------------------------------------------------------
 template <typename T, int L>
-__global__ void __launch_bounds__(BT, 4) edge_dy_kernel(Args a) {
+__global__ void __launch_bounds__(BT, 6) edge_dy_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   extern __shared__ float prod[];   // [Q][C + 1]: dy * Y per (l, m), channel
   __shared__ float D[S];
-  __shared__ float dsh[16], alh[16];
+  __shared__ float alh[16];
   const int C = a.C, CP = C + 1, QC = Q * C, H = a.H, Ch = C / H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
-    const int64_t e = a.ea + el;
-    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    const int i = a.dst[el];
     __syncthreads();
     for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
-    if (threadIdx.x < H) {
-      const int h = threadIdx.x;
-      const float al = a.al[el * H + h], diff = a.dal[el * H + h] - a.dlt[(size_t)(i - a.na) * H + h];
-      alh[h] = al;
-      dsh[h] = al * diff;
-      a.dsv[el * H + h] = al * diff;
+    if (warp == 0) {
+      // ds_h = alpha_h (dalpha_h - Delta_h); dL/du = sum_h e^(s - M) / den
+      // (dalpha_h - Delta_h)  (no division by u), summed over the lanes
+      float du = 0.f;
+      if (lane < H) {
+        const int h = lane;
+        const size_t nh = (size_t)(i - a.na) * H + h;
+        const float al = a.al[el * H + h], diff = a.dal[el * H + h] - a.dlt[nh];
+        alh[h] = al;
+        a.dsv[el * H + h] = al * diff;
+        const float M = a.Mv[nh], den = a.denv[nh];
+        if (den > 0.f && M > -INFINITY) du = expf(a.sv[el * H + h] - M) / den * diff;
+      }
+      du = warp_sum(du);
+      if (lane == 0) a.duv[el] = du;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      // dL/du = sum_h e^(s - M) / den (dalpha - Delta)  (no division by u)
-      float du = 0.f;
-      for (int h = 0; h < H; ++h) {
-        const float M = a.Mv[(size_t)(i - a.na) * H + h], den = a.denv[(size_t)(i - a.na) * H + h];
-        if (den > 0.f && M > -INFINITY)
-          du += expf(a.sv[el * H + h] - M) / den * (a.dal[el * H + h] - a.dlt[(size_t)(i - a.na) * H + h]);
-      }
-      a.duv[el] = du;
-    }
     const float *Gi = a.G + (size_t)i * QC;
     const float *Yr = a.Y + (size_t)el * QC;
     const float *gvp = a.gv + el * P;
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(BT, 4) edge_dy_kernel(Args a) {
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
         float gd[2 * L + 1];
+        asm volatile("" ::: "memory");   // one degree's loads in flight at a time (no spills)
         rotate_col<L>(D, Gi, l, c, C, gd);
 #pragma unroll
         for (int m = -l; m <= l; ++m) {
@@ -401,13 +403,13 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
   T *vj = reinterpret_cast<T *>(dvt + Q * CP);             // [Q][CPV]
   float *yv = dvt + Q * CP + (Q * CPV * (int)sizeof(T) + 15) / 16 * 4;   // [Q][CP]  y = g Y (unstacked)
   float *dz = yv + Q * CP;                                 // [Q][CP]  alpha G_i
-  float *qk = dz + Q * CP;                                 // [2][L+1][C]  q~0, k~0
+  float *qk = dz + Q * CP;                                 // [2][L+1][C]  ds q~0, ds k~0 (/ sqrt d)
   __shared__ float D[S], dD[S], dD0[Q];
   __shared__ float dsh[16], misc[32], tau[3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
     const int64_t e = a.ea + el;
-    const int i = node_of_edge(a.row_ptr, a.na, a.nb, e);
+    const int i = a.dst[el];
     const int j = a.col_idx[e];
     __syncthreads();
     for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
     const T *kj = static_cast<const T *>(a.k) + (size_t)j * QC;
     const T *vjr = static_cast<const T *>(a.v) + (size_t)j * QC;
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      const float alc = a.al[el * H + c / Ch];
+      const float alc = a.al[el * H + c / Ch], dsc = dsh[c / Ch];
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
         const float *row0 = D + wig_offset(l) + l * (2 * l + 1);
@@ -437,8 +439,8 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
           qh = fmaf(row0[m + l], to_f(qi[(size_t)q * C + c]), qh);
           kh = fmaf(row0[m + l], to_f(kj[(size_t)q * C + c]), kh);
         }
-        qk[l * C + c] = qh;
-        qk[(L + 1) * C + l * C + c] = kh;
+        qk[l * C + c] = dsc * qh;               // dk~0 = ds q~0 / sqrt d
+        qk[(L + 1) * C + l * C + c] = dsc * kh; // dq~0 = ds k~0 / sqrt d
       }
     }
     __syncthreads();
@@ -466,15 +468,16 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
       }
       dD[ent] = s0 + s1;
     }
-    // ... + the m = 0 row: dq~0 q_i[m'] + dk~0 k_j[m'] with dq~0 = ds k~0 / sqrt d,
-    // dk~0 = ds q~0 / sqrt d (one warp per (l, m'), lanes over channels)
+    // ... + the m = 0 row: dq~0 q_i[m'] + dk~0 k_j[m'] (one warp per (l, m'),
+    // lanes over channels)
     for (int idx = warp; idx < Q; idx += nw) {
       int l = 0;
       while ((l + 1) * (l + 1) <= idx) ++l;
       float sacc = 0.f;
+#pragma unroll 4
       for (int c = lane; c < C; c += 32)
-        sacc += dsh[c / Ch] * (qk[(L + 1) * C + l * C + c] * to_f(qi[(size_t)idx * C + c]) +
-                               qk[l * C + c] * to_f(kj[(size_t)idx * C + c]));
+        sacc += qk[(L + 1) * C + l * C + c] * to_f(qi[(size_t)idx * C + c]) +
+                qk[l * C + c] * to_f(kj[(size_t)idx * C + c]);
       sacc = warp_sum(sacc);
       if (lane == 0) dD0[idx] = sacc;
     }
@@ -539,12 +542,11 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
     // dv_j += D^T dv~; dq_i, dk_j += row0^T dq~0 / dk~0 (consecutive threads
     // on consecutive channels)
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      const float ds = dsh[c / Ch];
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
         const int w = 2 * l + 1;
         const float *Dl = D + wig_offset(l);
-        const float gq = ds * qk[(L + 1) * C + l * C + c], gk = ds * qk[l * C + c];
+        const float gq = qk[(L + 1) * C + l * C + c], gk = qk[l * C + c];
 #pragma unroll
         for (int mp = 0; mp < w; ++mp) {
           float acc = 0.f;
@@ -740,6 +742,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
   const size_t oz = carve(ce * 16 * 4), os = carve(ce * H * 4), ou = carve(ce * 4), orr = carve(ce * 16);
   const size_t oal = carve(ce * H * 4), odal = carve(ce * H * 4), ods = carve(ce * H * 4), odu = carve(ce * 4);
   const size_t odg = carve(ce * P * 4), oM = carve(cn * H * 4), oden = carve(cn * H * 4), odl = carve(cn * H * 4);
+  const size_t odst = carve(ce * 4);
   Scratch cs;
   E2F_CUDA_TRY(cs.alloc(off, s));
   char *cb = cs.as<char>();
@@ -764,6 +767,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
   a.dgv = reinterpret_cast<float *>(cb + odg);
   a.Mv = reinterpret_cast<float *>(cb + oM); a.denv = reinterpret_cast<float *>(cb + oden);
   a.dlt = reinterpret_cast<float *>(cb + odl);
+  a.dst = reinterpret_cast<int32_t *>(cb + odst);
   a.dq = dq; a.dk = dk; a.dv = dv; a.dpos = dpos;
   const size_t smem6 = sizeof(float) * ((size_t)3 * Q * (C + 4) + 2 * (size_t)(L + 1) * C) +
                        ((size_t)Q * (C + 16 / sizeof(T)) * sizeof(T) + 15) / 16 * 16;
@@ -778,6 +782,7 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
     if (a.ne == 0) continue;
     const int eg = (int)std::min<int64_t>(a.ne, 148LL * 16);
     const int ng = (int)std::min<int64_t>((a.nb - a.na + 7) / 8, 148LL * 8);
+    E2F_LAUNCH(edge_dst_kernel, ng, 256, 0, s, a);
     E2F_LAUNCH((edge_fwd_kernel<T, L>), eg, BT, sizeof(float) * C, s, a);
     E2F_LAUNCH(node_stats_kernel, ng, 256, 0, s, a);
     for (int m = 0; m <= L; ++m) {

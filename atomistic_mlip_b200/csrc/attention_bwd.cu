@@ -23,7 +23,7 @@
 //                   dL/dr_ij = (dL/dr) rhat + tau x rhat / r; atomics into
 //                   dL/dpos of both atoms and into dL/dq_i, dL/dk_j, dL/dv_j
 // then
-//   K7 dx           dL/dx = per degree dq Wq + dk Wk + dv Wv.
+//   GEMM            dL/dx = per degree dq Wq + dk Wk + dv Wv (cuBLAS, fp32).
 //
 // Per-edge tensors live only inside a chunk (bounded scratch); the SO(2)
 // products are dense GEMMs over the chunk's edges.
@@ -50,8 +50,9 @@ constexpr int JMAX = (E2F_MAX_L + 1) * (2 * E2F_MAX_L + 1) * (2 * E2F_MAX_L + 3)
 
 // J_k^l = d/dt D^l(exp(t K_k)) at t = 0, k = x, y, z (K_k v = e_k x v),
 // blocks laid out like the Wigner blocks; fitted on the host by a central
-// difference of the Ivanic-Ruedenberg construction.
-__constant__ float c_gen[3 * JMAX];
+// difference of the Ivanic-Ruedenberg construction.  Global memory, not
+// __constant__: the torque reads it at a different entry in every lane.
+__device__ float g_gen[3 * JMAX];
 
 struct Args {
   int L, C, H, N;
@@ -381,6 +382,55 @@ __device__ __forceinline__ float4 ld4f(const __nv_bfloat16 *p) {
   return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
+// One row (l, m) = q of dL/dD^l from the staged rows: this lane's partial over
+// the 4-channel chunks 4 qq, 4 qq + 16, ... (C a multiple of 16), summed over
+// the four lanes of the row (mask quad) and stored by the first of them.
+template <int LL, typename T>
+__device__ __forceinline__ void dd_row_l(int rr, int qq, unsigned quad, int C, int CP, int CPV, const float *dvt,
+                                         const T *vj, const float *yv, const float *dz, float *dD) {
+  constexpr int W = 2 * LL + 1;
+  const int q = LL * LL + rr;
+  const float *pa = dvt + q * CP, *ya = yv + q * CP;
+  const T *vb = vj + LL * LL * CPV;
+  const float *zb = dz + LL * LL * CP;
+  float acc[W];
+#pragma unroll
+  for (int cc = 0; cc < W; ++cc) acc[cc] = 0.f;
+  for (int c = 4 * qq; c < C; c += 16) {
+    const float4 xa = ld4f(pa + c), za = ld4f(ya + c);
+#pragma unroll
+    for (int cc = 0; cc < W; ++cc) {
+      const float4 xb = ld4f(vb + cc * CPV + c), zz = ld4f(zb + cc * CP + c);
+      acc[cc] = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, acc[cc]))));
+      acc[cc] = fmaf(za.x, zz.x, fmaf(za.y, zz.y, fmaf(za.z, zz.z, fmaf(za.w, zz.w, acc[cc]))));
+    }
+  }
+#pragma unroll
+  for (int cc = 0; cc < W; ++cc) {
+    acc[cc] += __shfl_xor_sync(quad, acc[cc], 1);
+    acc[cc] += __shfl_xor_sync(quad, acc[cc], 2);
+  }
+  if (qq == 0) {
+#pragma unroll
+    for (int cc = 0; cc < W; ++cc) dD[wig_offset(LL) + rr * W + cc] = acc[cc];
+  }
+}
+
+template <typename T, int L>
+__device__ __forceinline__ void dd_row(int q, int qq, unsigned quad, int C, int CP, int CPV, const float *dvt,
+                                       const T *vj, const float *yv, const float *dz, float *dD) {
+  int l = 0;
+  while ((l + 1) * (l + 1) <= q) ++l;
+  const int rr = q - l * l;
+  switch (l) {
+#define E2F_DD_ROW(LL) \
+  case LL: if (LL <= L) dd_row_l<(LL <= L ? LL : 0), T>(rr, qq, quad, C, CP, CPV, dvt, vj, yv, dz, dD); break;
+    E2F_DD_ROW(0) E2F_DD_ROW(1) E2F_DD_ROW(2) E2F_DD_ROW(3) E2F_DD_ROW(4) E2F_DD_ROW(5) E2F_DD_ROW(6)
+#undef E2F_DD_ROW
+    default: break;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // K6: dL/dD, torque, radius; atomics into dpos, dq, dk, dv.  Channel-major
 // staging into padded [Q][C + 1] rows (a thread per channel, (l, m) at
@@ -445,28 +495,26 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
     }
     __syncthreads();
     // dL/dD^l[m][m'] = sum_c dv~[m] v_j[m'] + y[m] dz[m'] ...
-    for (int ent = threadIdx.x; ent < S; ent += blockDim.x) {
-      int l = 0;
-      while (wig_offset(l + 1) <= ent) ++l;
-      const int w = 2 * l + 1, rr = (ent - wig_offset(l)) / w, cc = (ent - wig_offset(l)) % w;
-      const float *pa = dvt + (l * l + rr) * CP;
-      const T *pb = vj + (l * l + cc) * CPV;
-      const float *ya = yv + (l * l + rr) * CP, *zb = dz + (l * l + cc) * CP;
-      float s0 = 0.f, s1 = 0.f;
-      if ((C & 3) == 0) {
-        for (int c = 0; c < C; c += 4) {
-          const float4 xa = *reinterpret_cast<const float4 *>(pa + c), xb = ld4f(pb + c);
-          const float4 za = *reinterpret_cast<const float4 *>(ya + c), zz = *reinterpret_cast<const float4 *>(zb + c);
-          s0 = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, s0))));
-          s1 = fmaf(za.x, zz.x, fmaf(za.y, zz.y, fmaf(za.z, zz.z, fmaf(za.w, zz.w, s1))));
-        }
-      } else {
-        for (int c = 0; c < C; ++c) {
-          s0 = fmaf(pa[c], to_f(pb[c]), s0);
-          s1 = fmaf(ya[c], zb[c], s1);
-        }
+    if ((C & 15) == 0) {
+      // four lanes per row (l, m) of dD^l, each over every fourth 4-channel
+      // chunk and all 2l + 1 entries of the row, so that the row's dv~ and y
+      // chunks are read once; the four partials are then summed by shuffles
+      const int qq = threadIdx.x & 3;
+      const unsigned quad = 0xFu << (lane & ~3);
+      for (int q = threadIdx.x >> 2; q < Q; q += blockDim.x >> 2)
+        dd_row<T, L>(q, qq, quad, C, CP, CPV, dvt, vj, yv, dz, dD);
+    } else {
+      for (int ent = threadIdx.x; ent < S; ent += blockDim.x) {
+        int l = 0;
+        while (wig_offset(l + 1) <= ent) ++l;
+        const int w = 2 * l + 1, rr = (ent - wig_offset(l)) / w, cc = (ent - wig_offset(l)) % w;
+        const float *pa = dvt + (l * l + rr) * CP;
+        const T *pb = vj + (l * l + cc) * CPV;
+        const float *ya = yv + (l * l + rr) * CP, *zb = dz + (l * l + cc) * CP;
+        float s0 = 0.f;
+        for (int c = 0; c < C; ++c) s0 = fmaf(pa[c], to_f(pb[c]), fmaf(ya[c], zb[c], s0));
+        dD[ent] = s0;
       }
-      dD[ent] = s0 + s1;
     }
     // ... + the m = 0 row: dq~0 q_i[m'] + dk~0 k_j[m'] (one warp per (l, m'),
     // lanes over channels)
@@ -498,9 +546,9 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
         const float *Dl = D + wig_offset(l), *dDl = dD + wig_offset(l);
         float mab = 0.f;   // (D^T dD)[ra][cb]
         for (int m = 0; m < w; ++m) mab = fmaf(Dl[m * w + ra], dDl[m * w + cb], mab);
-        t0 = fmaf(mab, c_gen[ent], t0);
-        t1 = fmaf(mab, c_gen[JMAX + ent], t1);
-        t2 = fmaf(mab, c_gen[2 * JMAX + ent], t2);
+        t0 = fmaf(mab, __ldg(&g_gen[ent]), t0);
+        t1 = fmaf(mab, __ldg(&g_gen[JMAX + ent]), t1);
+        t2 = fmaf(mab, __ldg(&g_gen[2 * JMAX + ent]), t2);
       }
       t0 = warp_sum(t0); t1 = warp_sum(t1); t2 = warp_sum(t2);
       if (lane == 0) { atomicAdd(&tau[0], -t0); atomicAdd(&tau[1], -t1); atomicAdd(&tau[2], -t2); }
@@ -563,37 +611,11 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// K7: dx[n,(l,m),c] = sum_o dq[n,(l,m),o] Wq[l][o][c] + (k, v) alike
-// ---------------------------------------------------------------------------
+// fp32 copy of a weight matrix (the dL/dx GEMMs run in fp32)
 template <typename T>
-__global__ void dx_kernel(const float *dq, const float *dk, const float *dv, const e2f_weights w, int N,
-                          float *dx) {
-  extern __shared__ float sr[];   // [3][C] rows of one (node, l, m)
-  const int L = w.L_max, C = w.C, Q = (L + 1) * (L + 1);
-  for (int64_t row = blockIdx.x; row < (int64_t)N * Q; row += gridDim.x) {
-    const int q = (int)(row % Q);
-    int l = 0;
-    while ((l + 1) * (l + 1) <= q) ++l;
-    __syncthreads();
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      sr[c] = dq[row * C + c];
-      sr[C + c] = dk[row * C + c];
-      sr[2 * C + c] = dv[row * C + c];
-    }
-    __syncthreads();
-    const T *Wq = static_cast<const T *>(w.Wq[l]), *Wk = static_cast<const T *>(w.Wk[l]),
-            *Wv = static_cast<const T *>(w.Wv[l]);
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      float acc = 0.f;
-      for (int o = 0; o < C; ++o) {
-        acc = fmaf(sr[o], to_f(Wq[(size_t)o * C + c]), acc);
-        acc = fmaf(sr[C + o], to_f(Wk[(size_t)o * C + c]), acc);
-        acc = fmaf(sr[2 * C + o], to_f(Wv[(size_t)o * C + c]), acc);
-      }
-      dx[row * C + c] = acc;
-    }
-  }
+__global__ void to_f32_kernel(const T *src, int64_t n, float *dst) {
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x)
+    dst[x] = to_f(src[x]);
 }
 
 // Wc_m = [[Wr, -Wi], [Wi, Wr]] (2n x 2n, row-major), m >= 1
@@ -643,7 +665,7 @@ static e2f_status ensure_generators() {
   if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_gen_mu);
   if (!g_gen_up[dev]) {
-    E2F_CUDA_TRY(cudaMemcpyToSymbol(c_gen, g_gen_tab, sizeof(g_gen_tab)));
+    E2F_CUDA_TRY(cudaMemcpyToSymbol(g_gen, g_gen_tab, sizeof(g_gen_tab)));
     g_gen_up[dev] = true;
   }
   return E2F_OK;
@@ -802,8 +824,40 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
     }
     E2F_LAUNCH((edge_bwd_kernel<T, L>), eg, BT, smem6, s, a);
   }
-  const int rg = (int)std::min<int64_t>(N * Q, 148LL * 32);
-  E2F_LAUNCH(dx_kernel<T>, rg, 128, sizeof(float) * 3 * C, s, dq, dk, dv, *w, (int)N, dx);
+  // dL/dx[n, (l, m), :] = dq[n, (l, m), :] Wq[l] + dk Wk[l] + dv Wv[l]: per
+  // degree one strided-batched GEMM per projection over the 2l + 1 rows m
+  // (rows of one m are Q C apart), fp32 (weights converted once per call)
+  Scratch wf;
+  const float *Wf[3][L + 1];
+  if (std::is_same<T, float>::value) {
+    for (int l = 0; l <= L; ++l) {
+      Wf[0][l] = static_cast<const float *>(w->Wq[l]);
+      Wf[1][l] = static_cast<const float *>(w->Wk[l]);
+      Wf[2][l] = static_cast<const float *>(w->Wv[l]);
+    }
+  } else {
+    const int64_t cc = (int64_t)C * C;
+    E2F_CUDA_TRY(wf.alloc(sizeof(float) * 3 * (L + 1) * cc, s));
+    float *wb = wf.as<float>();
+    for (int t = 0; t < 3; ++t)
+      for (int l = 0; l <= L; ++l) {
+        const void *src = t == 0 ? w->Wq[l] : (t == 1 ? w->Wk[l] : w->Wv[l]);
+        float *d = wb + (t * (L + 1) + l) * cc;
+        E2F_LAUNCH(to_f32_kernel<T>, (int)std::min<int64_t>((cc + 255) / 256, 1024), 256, 0, s,
+                   static_cast<const T *>(src), cc, d);
+        Wf[t][l] = d;
+      }
+  }
+  const float *grads[3] = {dq, dk, dv};
+  for (int l = 0; l <= L; ++l)
+    for (int t = 0; t < 3; ++t) {
+      // column-major: dx^T[C x N] (ld QC) (+)= W^T[C x C] (the row-major W, ld C) * g^T[C x N] (ld QC)
+      const float one = 1.f, beta = t == 0 ? 0.f : 1.f;
+      const size_t o = (size_t)l * l * C;
+      if (cublasSgemmStridedBatched(bh, CUBLAS_OP_N, CUBLAS_OP_N, C, (int)N, C, &one, Wf[t][l], C, 0,
+                                    grads[t] + o, QC, C, &beta, dx + o, QC, C, 2 * l + 1) != CUBLAS_STATUS_SUCCESS)
+        return E2F_ERR_CUDA;
+    }
   return E2F_OK;
 }
 

@@ -48,8 +48,10 @@ def test_backward_fp32_cluster(cuda_ok):
     _check(wlmod.make_workload(0), "fp32", 1e-4)
 
 
-@pytest.mark.parametrize("L", [0, 1, 3])
+@pytest.mark.parametrize("L", [0, 1, 3, 4, 6])
 def test_backward_fp32_degrees(cuda_ok, L):
+    """C = 16 (the per-row dL/dD form, C a multiple of 16), every tile shape
+    of the degree loop up to the largest L."""
     wl = wlmod.make_workload(0, L=L, C=16, H=2)
     _check(wl, "fp32", 1e-4, seed=10 + L)
 

@@ -91,83 +91,110 @@ __global__ void edge_dst_kernel(Args a) {
   }
 }
 
-// D^l blocks of the edge frame into shared memory (block-cooperative).
-template <int L>
-__device__ void edge_wigner(float ux, float uy, float uz, float *D) {
-  if (threadIdx.x == 0) {
-    D[0] = 1.f;
-    if (L >= 1) {
-      float R[9];
-      edge_frame_two_angle(ux, uy, uz, R);
-      wig_l1_from_rotation(R, D + 1);
+// The next edge's destination node (and source node, D blocks), loaded one
+// iteration of the CTA's serial edge loop ahead into registers, so that the
+// dependent loads of an edge do not start with an index round trip.  The
+// CTA has BT threads.
+template <int S, bool J, bool DD>
+struct EdgePrefetch {
+  static constexpr int DPT = DD ? (S + BT - 1) / BT : 1;
+  int i = 0, j = 0;
+  float d[DPT];
+  __device__ __forceinline__ void load(const Args &a, int64_t el) {
+    if (el >= a.ne) return;
+    i = a.dst[el];
+    if (J) j = a.col_idx[a.ea + el];
+    if (DD) {
+#pragma unroll
+      for (int k = 0; k < DPT; ++k) {
+        const int x = threadIdx.x + k * BT;
+        if (x < S) d[k] = a.Dm[el * S + x];
+      }
     }
   }
-  __syncthreads();
-  for (int l = 2; l <= L; ++l) {
-    const int w = 2 * l + 1;
-    for (int x = threadIdx.x; x < w * w; x += blockDim.x)
-      D[wig_offset(l) + x] = wig_entry(l, x / w - l, x % w - l, D + 1, D + wig_offset(l - 1));
-    __syncthreads();
+  __device__ __forceinline__ void store_d(float *D) const {
+#pragma unroll
+    for (int k = 0; k < DPT; ++k) {
+      const int x = threadIdx.x + k * BT;
+      if (x < S) D[x] = d[k];
+    }
   }
-}
+};
 
 // ---------------------------------------------------------------------------
-// K1: geometry, D, envelope, radial MLP, logits; v~ = D v_j (stacked)
+// K1: geometry, D, envelope, radial MLP, logits; v~ = D v_j (stacked).  One
+// warp per edge (FWD_WARPS edges per CTA in flight, warp-level
+// synchronisation only): most steps of an edge use a few lanes, so one edge
+// per CTA would leave the CTA's other warps waiting at its barriers.
 // ---------------------------------------------------------------------------
+constexpr int FWD_WARPS = BT / 32;
+
 template <typename T, int L>
 __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
-  __shared__ float D[S];
-  __shared__ float hid[16], geo[8];
-  extern __shared__ float part[];   // [C]: per-channel logit partials
+  __shared__ float Dw[FWD_WARPS][S];
+  __shared__ float hidw[FWD_WARPS][16];
+  extern __shared__ float partw[];   // [FWD_WARPS][C]: per-channel logit partials
   const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
-  for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
-    const int64_t e = a.ea + el;
-    const int i = a.dst[el];
-    const int j = a.col_idx[e];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float dx, dy, dz;
-      pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dy, dz);
-      const float r = sqrtf(dx * dx + dy * dy + dz * dz);
-      geo[0] = dx; geo[1] = dy; geo[2] = dz; geo[3] = r;
-      geo[4] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float *D = Dw[warp], *hid = hidw[warp], *part = partw + warp * C;
+  for (int64_t el = (int64_t)blockIdx.x * FWD_WARPS + warp; el < a.ne; el += (int64_t)gridDim.x * FWD_WARPS) {
+    const int i = a.dst[el], j = a.col_idx[a.ea + el];
+    __syncwarp();   // the previous edge's readers of D, hid and part are done
+    // geometry (every lane; the two position loads are broadcasts)
+    float dx, dy, dz;
+    pair_disp(a.g, load_pos(a.pos, i), load_pos(a.pos, j), dx, dy, dz);
+    const float r = sqrtf(dx * dx + dy * dy + dz * dz);
+    if (lane == 0) {
       a.rv[el * 4 + 0] = dx; a.rv[el * 4 + 1] = dy; a.rv[el * 4 + 2] = dz; a.rv[el * 4 + 3] = r;
-      a.uv[el] = geo[4];
+      a.uv[el] = 0.5f * (cospif(r / a.g.rc) + 1.f);
+      // D^0, D^1 of the two-angle frame
+      float ux = 0.f, uy = 0.f, uz = 1.f;
+      if (r > 0.f) { ux = dx / r; uy = dy / r; uz = dz / r; }
+      D[0] = 1.f;
+      if (L >= 1) {
+        float R[9];
+        edge_frame_two_angle(ux, uy, uz, R);
+        wig_l1_from_rotation(R, D + 1);
+      }
     }
-    __syncthreads();
-    const float r = geo[3];
-    float ux = 0.f, uy = 0.f, uz = 1.f;
-    if (r > 0.f) { ux = geo[0] / r; uy = geo[1] / r; uz = geo[2] / r; }
-    edge_wigner<L>(ux, uy, uz, D);
-    for (int x = threadIdx.x; x < S; x += blockDim.x) a.Dm[el * S + x] = D[x];
     // radial MLP: 8 Gaussians (centres k r_c / 7, sigma 0.5) -> 16 SiLU -> P
-    if (threadIdx.x < 16) {
+    if (lane >= 16) {
+      const int h = lane - 16;
       float z = 0.f;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const float dd = r - (float)kk * (a.g.rc / 7.f);
-        z = fmaf(a.W1[threadIdx.x * 8 + kk], expf(-dd * dd * 2.f), z);
+        z = fmaf(a.W1[h * 8 + kk], expf(-dd * dd * 2.f), z);
       }
-      a.zv[el * 16 + threadIdx.x] = z;
-      hid[threadIdx.x] = z / (1.f + expf(-z));
+      a.zv[el * 16 + h] = z;
+      hid[h] = z / (1.f + expf(-z));
     }
-    __syncthreads();
-    if (threadIdx.x < P) {
+    __syncwarp();
+    // D^l, l >= 2, by the Ivanic-Ruedenberg recursion, a level at a time
+    for (int l = 2; l <= L; ++l) {
+      const int w = 2 * l + 1;
+      for (int x = lane; x < w * w; x += 32)
+        D[wig_offset(l) + x] = wig_entry(l, x / w - l, x % w - l, D + 1, D + wig_offset(l - 1));
+      __syncwarp();
+    }
+    for (int x = lane; x < S; x += 32) a.Dm[el * S + x] = D[x];
+    for (int p = lane; p < P; p += 32) {
       float gg = 0.f;
 #pragma unroll
-      for (int hh = 0; hh < 16; ++hh) gg = fmaf(a.W2[threadIdx.x * 16 + hh], hid[hh], gg);
-      a.gv[el * P + threadIdx.x] = gg;
+      for (int hh = 0; hh < 16; ++hh) gg = fmaf(a.W2[p * 16 + hh], hid[hh], gg);
+      a.gv[el * P + p] = gg;
     }
     // logits: the m = 0 rows of D q_i and D k_j, per head
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    for (int c = lane; c < C; c += 32) {
       float s = 0.f;
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
         const int w = 2 * l + 1;
         const float *row0 = D + wig_offset(l) + l * w;
         float qh = 0.f, kh = 0.f;
+#pragma unroll
         for (int mp = 0; mp < w; ++mp) {
           qh = fmaf(row0[mp], ldf<T>(a.q, ((size_t)i * Q + l * l + mp) * C + c), qh);
           kh = fmaf(row0[mp], ldf<T>(a.k, ((size_t)j * Q + l * l + mp) * C + c), kh);
@@ -176,15 +203,15 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
       }
       part[c] = s;
     }
-    __syncthreads();
-    if (threadIdx.x < H) {
+    __syncwarp();
+    if (lane < H) {
       float hsum = 0.f;
-      for (int c = threadIdx.x * Ch; c < (threadIdx.x + 1) * Ch; ++c) hsum += part[c];
-      a.sv[el * H + threadIdx.x] = hsum * a.inv_sqrt_d;
+      for (int c = lane * Ch; c < (lane + 1) * Ch; ++c) hsum += part[c];
+      a.sv[el * H + lane] = hsum * a.inv_sqrt_d;
     }
     // rotate in: v~[(l,m),c] = sum_m' D^l[m][m'] v_j[(l,m'),c], stacked
     T *Arow = static_cast<T *>(a.A) + (size_t)el * QC;
-    for (int x = threadIdx.x; x < (L + 1) * C; x += blockDim.x) {
+    for (int x = lane; x < (L + 1) * C; x += 32) {
       const int l = x / C, c = x % C, w = 2 * l + 1;
       float vv[2 * L + 1];
 #pragma unroll
@@ -263,10 +290,13 @@ __global__ void __launch_bounds__(BT, 4) edge_dalpha_kernel(Args a) {
   __shared__ float D[S];
   extern __shared__ float part[];   // [C]: per-channel partials of dL/dalpha
   const int C = a.C, QC = Q * C, H = a.H, Ch = C / H;
+  EdgePrefetch<S, false, true> pf;
+  pf.load(a, blockIdx.x);
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
-    const int i = a.dst[el];
+    const int i = pf.i;
     __syncthreads();
-    for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
+    pf.store_d(D);
+    pf.load(a, el + gridDim.x);
     __syncthreads();
     const float *Gi = a.G + (size_t)i * QC;
     const float *Yr = a.Y + (size_t)el * QC;
@@ -315,10 +345,13 @@ __global__ void __launch_bounds__(BT, 6) edge_dy_kernel(Args a) {
   __shared__ float alh[16];
   const int C = a.C, CP = C + 1, QC = Q * C, H = a.H, Ch = C / H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  EdgePrefetch<S, false, true> pf;
+  pf.load(a, blockIdx.x);
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
-    const int i = a.dst[el];
+    const int i = pf.i;
     __syncthreads();
-    for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
+    pf.store_d(D);
+    pf.load(a, el + gridDim.x);
     if (warp == 0) {
       // ds_h = alpha_h (dalpha_h - Delta_h); dL/du = sum_h e^(s - M) / den
       // (dalpha_h - Delta_h)  (no division by u), summed over the lanes
@@ -457,12 +490,13 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
   __shared__ float D[S], dD[S], dD0[Q];
   __shared__ float dsh[16], misc[32], tau[3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  EdgePrefetch<S, true, true> pf;
+  pf.load(a, blockIdx.x);
   for (int64_t el = blockIdx.x; el < a.ne; el += gridDim.x) {
-    const int64_t e = a.ea + el;
-    const int i = a.dst[el];
-    const int j = a.col_idx[e];
+    const int i = pf.i, j = pf.j;
     __syncthreads();
-    for (int x = threadIdx.x; x < S; x += blockDim.x) D[x] = a.Dm[el * S + x];
+    pf.store_d(D);
+    pf.load(a, el + gridDim.x);
     if (threadIdx.x < H) dsh[threadIdx.x] = a.dsv[el * H + threadIdx.x] * a.inv_sqrt_d;
     if (threadIdx.x < 3) tau[threadIdx.x] = 0.f;
     __syncthreads();
@@ -476,6 +510,7 @@ __global__ void __launch_bounds__(BT, 4) edge_bwd_kernel(Args a) {
       const float alc = a.al[el * H + c / Ch], dsc = dsh[c / Ch];
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
+        asm volatile("" ::: "memory");   // one degree's loads in flight at a time
         const float *row0 = D + wig_offset(l) + l * (2 * l + 1);
         float qh = 0.f, kh = 0.f;
 #pragma unroll
@@ -805,7 +840,8 @@ static e2f_status run(const void *x, const float *pos, const e2f_csr *csr, const
     const int eg = (int)std::min<int64_t>(a.ne, 148LL * 16);
     const int ng = (int)std::min<int64_t>((a.nb - a.na + 7) / 8, 148LL * 8);
     E2F_LAUNCH(edge_dst_kernel, ng, 256, 0, s, a);
-    E2F_LAUNCH((edge_fwd_kernel<T, L>), eg, BT, sizeof(float) * C, s, a);
+    const int fg = (int)std::min<int64_t>((a.ne + FWD_WARPS - 1) / FWD_WARPS, 148LL * 16);
+    E2F_LAUNCH((edge_fwd_kernel<T, L>), fg, BT, sizeof(float) * FWD_WARPS * C, s, a);
     E2F_LAUNCH(node_stats_kernel, ng, 256, 0, s, a);
     for (int m = 0; m <= L; ++m) {
       const int wm = m == 0 ? (L + 1) * C : 2 * (L - m + 1) * C;

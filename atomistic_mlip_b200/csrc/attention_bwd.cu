@@ -706,17 +706,18 @@ static e2f_status ensure_generators() {
   return E2F_OK;
 }
 
-static std::mutex g_blas_mu;
-static cublasHandle_t g_blas[64] = {};
+// One cuBLAS handle per (host thread, device): a handle carries the stream
+// it was last given, so calls from different threads on different streams
+// must not share one.
+static thread_local cublasHandle_t tl_blas[64] = {};
 
 static e2f_status blas_handle(cublasHandle_t *h, cudaStream_t s) {
   int dev = 0;
   E2F_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return E2F_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_blas_mu);
-  if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) return E2F_ERR_CUDA;
-  if (cublasSetStream(g_blas[dev], s) != CUBLAS_STATUS_SUCCESS) return E2F_ERR_CUDA;
-  *h = g_blas[dev];
+  if (!tl_blas[dev] && cublasCreate(&tl_blas[dev]) != CUBLAS_STATUS_SUCCESS) return E2F_ERR_CUDA;
+  if (cublasSetStream(tl_blas[dev], s) != CUBLAS_STATUS_SUCCESS) return E2F_ERR_CUDA;
+  *h = tl_blas[dev];
   return E2F_OK;
 }
 

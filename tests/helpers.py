@@ -3,6 +3,7 @@ run the library, and compare with the oracle under the error measure the
 tests use (max |gpu - ref| / max |ref| over the compared rows)."""
 from __future__ import annotations
 
+import dataclasses
 import functools
 
 import numpy as np
@@ -51,3 +52,24 @@ def oracle_csr(cfg: int):
 @functools.lru_cache(maxsize=None)
 def cached_workload(cfg: int, precision: str):
     return wlmod.make_workload(cfg, precision=precision)
+
+
+def local_gradients(wl, nodes, G):
+    """Oracle (dL/dpos, dL/dx) of the atoms `nodes` of a large system, from
+    the outputs that depend on them: rows S = nodes + their neighbours, over
+    the atoms U those rows read; every other output row is left out (it
+    does not depend on the sampled atoms)."""
+    from oracle import attention_grad as ag
+    from oracle import neighbors as nb
+    rp1, col1 = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)
+    S = np.unique(np.concatenate([nodes, col1.astype(np.int64)]))
+    rpS, colS = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, S)
+    U = np.unique(np.concatenate([S, colS.astype(np.int64)]))
+    idx = -np.ones(wl.N, np.int64)
+    idx[U] = np.arange(len(U))
+    rp = np.zeros(len(U) + 1, np.int64)
+    np.cumsum(np.diff(rpS)[U], out=rp[1:])
+    col = np.concatenate([idx[colS[rpS[u]:rpS[u + 1]]] for u in U]).astype(np.int32)
+    local = dataclasses.replace(wl, pos=wl.pos[U], x=wl.x[U])
+    ref = ag.gradients(local, (rp, col), G[U])
+    return ref["pos"][idx[nodes]], ref["x"][idx[nodes]]

@@ -127,3 +127,23 @@ def test_logit_gradient_recompute_form():
         G = np.random.default_rng(42).standard_normal((wl.N, (wl.L + 1) ** 2, wl.C))
         auto, formula = ag.logit_gradient(wl, csr, G)
         assert np.max(np.abs(auto - formula)) <= 1e-12 * np.max(np.abs(auto))
+
+
+def test_local_gradients_equal_full_gradients():
+    """The sampled form used on large systems (tests.helpers.local_gradients:
+    only the outputs of an atom and of its neighbours, over the atoms those
+    rows read) gives the atom's full dL/dpos and dL/dx: pinned against the
+    gradients of the whole system on a periodic box where the local region is
+    a strict subset of the atoms."""
+    from tests import helpers
+    rng = np.random.default_rng(21)
+    b = 16.0
+    pos = rng.uniform(0.0, b, (120, 3)).astype(np.float32)
+    wl = wlmod.make_custom(pos, np.array([b, b, b], np.float32), 3.5, L=2, C=8, H=2, seed=22)
+    G = rng.standard_normal(wl.x.shape)
+    full = ag.gradients(wl, nb.neighbors(wl.pos, wl.box, wl.r_c), G)
+    nodes = np.array([3, 57, 101])
+    gp, gx = helpers.local_gradients(wl, nodes, G)
+    assert np.max(np.abs(gp - full["pos"][nodes])) <= 1e-12 * np.max(np.abs(full["pos"][nodes]))
+    assert np.max(np.abs(gx - full["x"][nodes])) <= 1e-12 * np.max(np.abs(full["x"][nodes]))
+    assert np.max(np.abs(full["pos"][nodes])) > 0

@@ -54,22 +54,35 @@ def cached_workload(cfg: int, precision: str):
     return wlmod.make_workload(cfg, precision=precision)
 
 
+def local_rows(pos, box, r_c, rows):
+    """(U, (row_ptr, col), idx) for sampled rows of a large system: the atoms
+    U that the radius-graph rows `rows` read (the rows' own atoms and their
+    neighbours, sorted), the CSR over U that lists exactly those rows in
+    full (every other row empty), and idx mapping a global atom index to its
+    place in U (-1 outside).  An operator whose output row i reads only atom
+    i and its neighbours gives the same rows on this subsystem."""
+    from oracle import neighbors as nb
+    rows = np.unique(np.asarray(rows, np.int64))
+    rp, col = nb.neighbor_rows(pos, box, r_c, rows)
+    U = np.unique(np.concatenate([rows, col.astype(np.int64)]))
+    idx = -np.ones(len(pos), np.int64)
+    idx[U] = np.arange(len(U))
+    lrp = np.zeros(len(U) + 1, np.int64)
+    np.cumsum(np.diff(rp)[U], out=lrp[1:])
+    lcol = np.concatenate([idx[col[rp[u]:rp[u + 1]]] for u in U]).astype(np.int32)
+    return U, (lrp, lcol), idx
+
+
 def local_gradients(wl, nodes, G):
     """Oracle (dL/dpos, dL/dx) of the atoms `nodes` of a large system, from
-    the outputs that depend on them: rows S = nodes + their neighbours, over
-    the atoms U those rows read; every other output row is left out (it
-    does not depend on the sampled atoms)."""
+    the outputs that depend on them: the rows of the nodes and of their
+    neighbours, over the atoms those rows read; every other output row is
+    left out (it does not depend on the sampled atoms)."""
     from oracle import attention_grad as ag
     from oracle import neighbors as nb
-    rp1, col1 = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)
-    S = np.unique(np.concatenate([nodes, col1.astype(np.int64)]))
-    rpS, colS = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, S)
-    U = np.unique(np.concatenate([S, colS.astype(np.int64)]))
-    idx = -np.ones(wl.N, np.int64)
-    idx[U] = np.arange(len(U))
-    rp = np.zeros(len(U) + 1, np.int64)
-    np.cumsum(np.diff(rpS)[U], out=rp[1:])
-    col = np.concatenate([idx[colS[rpS[u]:rpS[u + 1]]] for u in U]).astype(np.int32)
+    col1 = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)[1]
+    S = np.unique(np.concatenate([np.asarray(nodes, np.int64), col1.astype(np.int64)]))
+    U, csr, idx = local_rows(wl.pos, wl.box, wl.r_c, S)
     local = dataclasses.replace(wl, pos=wl.pos[U], x=wl.x[U])
-    ref = ag.gradients(local, (rp, col), G[U])
+    ref = ag.gradients(local, csr, G[U])
     return ref["pos"][idx[nodes]], ref["x"][idx[nodes]]

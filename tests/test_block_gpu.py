@@ -88,3 +88,34 @@ def test_block_bf16_water_box_sampled(cuda_ok):
     csr = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)
     ref = ob.block_forward(wl.pos, wl.box, wl.r_c, csr, wl.x, lw, nodes=nodes, round_bf16=True)
     assert helpers.rel_err(got[nodes], ref) <= 2e-2
+
+
+def test_block_bf16_water100k_sampled(cuda_ok):
+    """The 100,002-atom water box, one block (the configuration the block is
+    timed on), 40 sampled rows of the full-size call against the oracle on
+    the rows' local subsystem (the rows' atoms and their neighbours)."""
+    wl = helpers.cached_workload(4, "bf16")
+    lw = wlmod.make_layer_weights(wl.L, wl.C, wl.H, "bf16", 72)
+    got = _run(wl, [lw], "bf16")
+    nodes = np.sort(np.random.default_rng(73).choice(wl.N, size=40, replace=False))
+    U, csr, idx = helpers.local_rows(wl.pos, wl.box, wl.r_c, nodes)
+    ref = ob.block_forward(wl.pos[U], wl.box, wl.r_c, csr, wl.x[U], lw, nodes=idx[nodes], round_bf16=True)
+    assert np.all(np.isfinite(got[nodes]))
+    assert helpers.rel_err(got[nodes], ref) <= 2e-2
+
+
+def test_two_layer_model_water_box_sampled(cuda_ok):
+    """Two blocks on the 3,000-atom water box (bf16, as timed), 8 sampled
+    rows: the second block's rows read the first block's outputs at the rows
+    and their neighbours, which the oracle computes on their own local
+    subsystem first."""
+    wl = helpers.cached_workload(2, "bf16")
+    layers = [wlmod.make_layer_weights(wl.L, wl.C, wl.H, "bf16", s) for s in (74, 75)]
+    got = _run(wl, layers, "bf16")
+    nodes = np.sort(np.random.default_rng(76).choice(wl.N, size=8, replace=False))
+    U1, csr2, idx1 = helpers.local_rows(wl.pos, wl.box, wl.r_c, nodes)
+    U2, csr1, idx2 = helpers.local_rows(wl.pos, wl.box, wl.r_c, U1)
+    x1 = ob.block_forward(wl.pos[U2], wl.box, wl.r_c, csr1, wl.x[U2], layers[0], nodes=idx2[U1],
+                          round_bf16=True)
+    ref = ob.block_forward(wl.pos[U1], wl.box, wl.r_c, csr2, x1, layers[1], nodes=idx1[nodes], round_bf16=True)
+    assert helpers.rel_err(got[nodes], ref) <= 2e-2

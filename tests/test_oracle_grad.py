@@ -147,3 +147,22 @@ def test_local_gradients_equal_full_gradients():
     assert np.max(np.abs(gp - full["pos"][nodes])) <= 1e-12 * np.max(np.abs(full["pos"][nodes]))
     assert np.max(np.abs(gx - full["x"][nodes])) <= 1e-12 * np.max(np.abs(full["x"][nodes]))
     assert np.max(np.abs(full["pos"][nodes])) > 0
+
+
+def test_local_rows_reproduce_the_attention_rows():
+    """tests.helpers.local_rows: the attention oracle on the subsystem of
+    some rows (their atoms and neighbours, only those rows listed) gives the
+    same rows as on the whole periodic system."""
+    from tests import helpers
+    rng = np.random.default_rng(23)
+    b = 16.0
+    pos = rng.uniform(0.0, b, (120, 3)).astype(np.float32)
+    wl = wlmod.make_custom(pos, np.array([b, b, b], np.float32), 3.5, L=2, C=8, H=2, seed=24)
+    rp, col = nb.neighbors(wl.pos, wl.box, wl.r_c)[:2]
+    args = (wl.Wq, wl.Wk, wl.Wv, wl.W0, wl.Wr, wl.Wi, wl.rad_W1, wl.rad_W2, wl.L, wl.C, wl.H)
+    full = oa.attention(wl.pos, wl.box, wl.r_c, rp, col, wl.x, *args)
+    nodes = np.array([5, 60, 99])
+    U, csr, idx = helpers.local_rows(wl.pos, wl.box, wl.r_c, nodes)
+    assert len(U) < wl.N
+    loc = oa.attention(wl.pos[U], wl.box, wl.r_c, csr[0], csr[1], wl.x[U], *args, nodes=idx[nodes])
+    assert np.max(np.abs(loc - full[nodes])) <= 1e-12 * np.max(np.abs(full[nodes]))

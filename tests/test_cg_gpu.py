@@ -108,15 +108,17 @@ def test_cg_num_paths_matches_oracle(cuda_ok):
         assert e2f.cg_num_paths(L) == len(cg.paths(L)) == wlmod.cg_num_paths(L)
 
 
-def test_cg_conv_water100k_sampled(cuda_ok):
-    """The benchmark configuration: the 100,002-atom water box, L = 4,
-    C = 128, the workload's bf16 features, 40 sampled rows of the full-size
-    launch against the oracle's brute-force rows."""
-    wl = helpers.cached_workload(4, "bf16")
+@pytest.mark.parametrize("cfg", [2, 4])
+def test_cg_conv_water_timed_configs(cuda_ok, cfg):
+    """The configurations the convolution is timed on: the 3,000- and
+    100,002-atom water boxes, L = 4, C = 128, the workload's bf16 features,
+    40 sampled rows of the full-size launch against the oracle's brute-force
+    rows."""
+    wl = helpers.cached_workload(cfg, "bf16")
     W = wlmod.make_cg_weights(4, 128, 77)
     got = _gpu(wl.pos, wl.box, wl.r_c, wl.x, W, 4, "bf16")
     assert np.all(np.isfinite(got))
-    nodes = np.sort(np.random.default_rng(160).choice(wl.N, size=40, replace=False))
+    nodes = np.sort(np.random.default_rng(160 + cfg).choice(wl.N, size=40, replace=False))
     rp, col = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)[:2]
     ref = cg.cg_conv(wl.pos, wl.box, wl.r_c, rp, col, _stored(wl.x, "bf16"), W, 4, nodes=nodes)
     assert helpers.rel_err(got[nodes], ref) <= TOL

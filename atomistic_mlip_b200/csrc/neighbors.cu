@@ -125,6 +125,7 @@ __global__ void cell_scatter_kernel(const float *__restrict__ pos, const int32_t
 // exact).  Otherwise every pair takes the branch test.
 // ---------------------------------------------------------------------------
 constexpr int CAND_CAP = 1024;      // candidates staged at a time
+constexpr int COUNT_HPW = 3;        // home atoms per warp and sweep in the count pass
 constexpr int CELL_THREADS = 256;
 
 struct Stencil {
@@ -234,19 +235,33 @@ __global__ void __launch_bounds__(CELL_THREADS) cell_count_kernel(int ncell, Cel
       __syncthreads();
       stage_candidates(st, c0, nc, spos, cp, cs);
       __syncthreads();
-      for (int a = wid; a < hn; a += nw) {
-        const float4 me = spos[h0 + a];
-        const int i = __float_as_int(me.w);
-        const float3 pi = make_float3(me.x, me.y, me.z);
-        int cnt = 0;
-        for (int k = lane; k < nc; k += 32) {
-          const float4 pj = cp[k];
-          if (__float_as_int(pj.w) != i && is_edge<FAST>(g, pi, pj, cs[k])) ++cnt;
+      // COUNT_HPW home atoms per warp in one sweep: each staged candidate is
+      // read from shared memory once for all of them
+      for (int a0 = wid; a0 < hn; a0 += nw * COUNT_HPW) {
+        float3 pi[COUNT_HPW];
+        int ii[COUNT_HPW], cnt[COUNT_HPW];
+#pragma unroll
+        for (int q = 0; q < COUNT_HPW; ++q) {
+          const int a = a0 + q * nw;
+          const float4 me = a < hn ? spos[h0 + a] : make_float4(0.f, 0.f, 0.f, __int_as_float(-1));
+          ii[q] = __float_as_int(me.w);
+          pi[q] = make_float3(me.x, me.y, me.z);
+          cnt[q] = 0;
         }
-        cnt = warp_sum_i(cnt);
-        if (lane == 0) {
-          if (c0 == 0) deg[i] = cnt;
-          else deg[i] += cnt;
+        for (int k = lane; k < nc; k += 32) {
+          const float4 pj = cp[k], sj = cs[k];
+          const int j = __float_as_int(pj.w);
+#pragma unroll
+          for (int q = 0; q < COUNT_HPW; ++q)
+            if (j != ii[q] && is_edge<FAST>(g, pi[q], pj, sj)) ++cnt[q];
+        }
+#pragma unroll
+        for (int q = 0; q < COUNT_HPW; ++q) {
+          const int c = warp_sum_i(cnt[q]);
+          if (lane == 0 && ii[q] >= 0) {
+            if (c0 == 0) deg[ii[q]] = c;
+            else deg[ii[q]] += c;
+          }
         }
       }
     }
@@ -389,7 +404,9 @@ static int cell_grid_blocks(long long ncell) {
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  return (int)std::max<long long>(1, std::min<long long>(ncell, (long long)nsm * 8));
+  // one CTA per cell (up to 16 waves of resident CTAs, grid-stride beyond):
+  // cells differ in cost, so the hardware's block scheduler balances them
+  return (int)std::max<long long>(1, std::min<long long>(ncell, (long long)nsm * 96));
 }
 
 static e2f_status launch_count(long long ncell, const CellGrid &cg, const Geom &g, const int32_t *cstart,

@@ -91,3 +91,17 @@ def test_backward_bf16_full_width(cuda_ok):
     wl0 = wlmod.make_workload(0)
     wl = wlmod.make_custom(wl0.pos, None, wl0.r_c, L=4, C=128, H=8, precision="bf16", seed=8)
     _check(wl, "bf16", 3e-2)
+
+
+def test_backward_isolated_atoms_and_no_edges(cuda_ok):
+    """Isolated atoms get zero gradients; a system with no edge at all gives
+    zero dL/dx and dL/dpos (every chunk is empty)."""
+    pos = np.array([[0, 0, 0], [1.1, 0.4, -0.3], [40, 40, 40], [80, 0, 0]], np.float32)
+    wl = wlmod.make_custom(pos, None, 3.0, L=2, C=16, H=2, precision="fp32", seed=500)
+    ex, ep = _check(wl, "fp32", 1e-4, seed=501)
+    G = np.random.default_rng(502).standard_normal(wl.x.shape)
+    gx, gp = _gpu_grads(wl, G, "fp32")
+    assert np.all(gx[2:] == 0) and np.all(gp[2:] == 0)
+    far = wlmod.make_custom(pos[2:], None, 3.0, L=2, C=16, H=2, precision="fp32", seed=503)
+    gx, gp = _gpu_grads(far, np.random.default_rng(504).standard_normal(far.x.shape), "fp32")
+    assert np.all(gx == 0) and np.all(gp == 0)

@@ -128,9 +128,10 @@ struct EdgePrefetch {
 // per CTA would leave the CTA's other warps waiting at its barriers.
 // ---------------------------------------------------------------------------
 constexpr int FWD_WARPS = BT / 32;
+constexpr int FWD_CPL = 2;   // channels per lane in the logits and the rotate-in
 
 template <typename T, int L>
-__global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
+__global__ void __launch_bounds__(BT, 6) edge_fwd_kernel(Args a) {
   constexpr int Q = (L + 1) * (L + 1), S = L * (4 * L * L - 1) / 3 + (2 * L + 1) * (2 * L + 1);
   constexpr int P = (L + 1) * (L + 2) / 2;
   __shared__ float Dw[FWD_WARPS][S];
@@ -186,22 +187,39 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
       for (int hh = 0; hh < 16; ++hh) gg = fmaf(a.W2[p * 16 + hh], hid[hh], gg);
       a.gv[el * P + p] = gg;
     }
-    // logits: the m = 0 rows of D q_i and D k_j, per head
-    for (int c = lane; c < C; c += 32) {
-      float s = 0.f;
+    // logits: the m = 0 rows of D q_i and D k_j, per head.  A lane takes
+    // FWD_CPL channels (32 apart) at once, so each D entry is read once for
+    // all of them.
+    for (int c0 = lane; c0 < C; c0 += 32 * FWD_CPL) {
+      float s[FWD_CPL];
+#pragma unroll
+      for (int r = 0; r < FWD_CPL; ++r) s[r] = 0.f;
 #pragma unroll
       for (int l = 0; l <= L; ++l) {
+        asm volatile("" ::: "memory");   // one degree's loads in flight at a time
         const int w = 2 * l + 1;
         const float *row0 = D + wig_offset(l) + l * w;
-        float qh = 0.f, kh = 0.f;
+        float qh[FWD_CPL], kh[FWD_CPL];
+#pragma unroll
+        for (int r = 0; r < FWD_CPL; ++r) qh[r] = kh[r] = 0.f;
 #pragma unroll
         for (int mp = 0; mp < w; ++mp) {
-          qh = fmaf(row0[mp], ldf<T>(a.q, ((size_t)i * Q + l * l + mp) * C + c), qh);
-          kh = fmaf(row0[mp], ldf<T>(a.k, ((size_t)j * Q + l * l + mp) * C + c), kh);
+          const float d = row0[mp];
+#pragma unroll
+          for (int r = 0; r < FWD_CPL; ++r) {
+            const int c = c0 + 32 * r;
+            if (c < C) {
+              qh[r] = fmaf(d, ldf<T>(a.q, ((size_t)i * Q + l * l + mp) * C + c), qh[r]);
+              kh[r] = fmaf(d, ldf<T>(a.k, ((size_t)j * Q + l * l + mp) * C + c), kh[r]);
+            }
+          }
         }
-        s = fmaf(qh, kh, s);
+#pragma unroll
+        for (int r = 0; r < FWD_CPL; ++r) s[r] = fmaf(qh[r], kh[r], s[r]);
       }
-      part[c] = s;
+#pragma unroll
+      for (int r = 0; r < FWD_CPL; ++r)
+        if (c0 + 32 * r < C) part[c0 + 32 * r] = s[r];
     }
     __syncwarp();
     if (lane < H) {
@@ -209,20 +227,38 @@ __global__ void __launch_bounds__(BT) edge_fwd_kernel(Args a) {
       for (int c = lane * Ch; c < (lane + 1) * Ch; ++c) hsum += part[c];
       a.sv[el * H + lane] = hsum * a.inv_sqrt_d;
     }
-    // rotate in: v~[(l,m),c] = sum_m' D^l[m][m'] v_j[(l,m'),c], stacked
+    // rotate in: v~[(l,m),c] = sum_m' D^l[m][m'] v_j[(l,m'),c], stacked; a
+    // lane takes FWD_CPL channels at once (each D entry read once for all)
     T *Arow = static_cast<T *>(a.A) + (size_t)el * QC;
-    for (int x = lane; x < (L + 1) * C; x += 32) {
-      const int l = x / C, c = x % C, w = 2 * l + 1;
-      float vv[2 * L + 1];
+    for (int c0 = lane; c0 < C; c0 += 32 * FWD_CPL) {
 #pragma unroll
-      for (int mp = 0; mp < 2 * L + 1; ++mp) vv[mp] = mp < w ? ldf<T>(a.v, ((size_t)j * Q + l * l + mp) * C + c) : 0.f;
-      const float *Dl = D + wig_offset(l);
-      for (int m = -l; m <= l; ++m) {
-        float acc = 0.f;
+      for (int l = 0; l <= L; ++l) {
+        asm volatile("" ::: "memory");   // one degree's loads in flight at a time
+        const int w = 2 * l + 1;
+        float vv[FWD_CPL][2 * L + 1];
 #pragma unroll
-        for (int mp = 0; mp < 2 * L + 1; ++mp)
-          if (mp < w) acc = fmaf(Dl[(m + l) * w + mp], vv[mp], acc);
-        Arow[stack_off(L, C, m) + (l - (m < 0 ? -m : m)) * C + c] = from_f<T>(acc);
+        for (int r = 0; r < FWD_CPL; ++r) {
+          const int c = c0 + 32 * r;
+#pragma unroll
+          for (int mp = 0; mp < w; ++mp) vv[r][mp] = c < C ? ldf<T>(a.v, ((size_t)j * Q + l * l + mp) * C + c) : 0.f;
+        }
+        const float *Dl = D + wig_offset(l);
+#pragma unroll
+        for (int m = -l; m <= l; ++m) {
+          float acc[FWD_CPL];
+#pragma unroll
+          for (int r = 0; r < FWD_CPL; ++r) acc[r] = 0.f;
+#pragma unroll
+          for (int mp = 0; mp < w; ++mp) {
+            const float d = Dl[(m + l) * w + mp];
+#pragma unroll
+            for (int r = 0; r < FWD_CPL; ++r) acc[r] = fmaf(d, vv[r][mp], acc[r]);
+          }
+          const int so = stack_off(L, C, m) + (l - (m < 0 ? -m : m)) * C;
+#pragma unroll
+          for (int r = 0; r < FWD_CPL; ++r)
+            if (c0 + 32 * r < C) Arow[so + c0 + 32 * r] = from_f<T>(acc[r]);
+        }
       }
     }
   }

@@ -122,3 +122,13 @@ def test_cg_conv_water_timed_configs(cuda_ok, cfg):
     rp, col = nb.neighbor_rows(wl.pos, wl.box, wl.r_c, nodes)[:2]
     ref = cg.cg_conv(wl.pos, wl.box, wl.r_c, rp, col, _stored(wl.x, "bf16"), W, 4, nodes=nodes)
     assert helpers.rel_err(got[nodes], ref) <= TOL
+
+
+@pytest.mark.parametrize("L", [4, 6])
+def test_cg_conv_cluster_fp32_full_width(cuda_ok, L):
+    """C = 128 in fp32 storage (two channels per thread), L = 4 and the
+    largest degree, on the 24-atom cluster."""
+    wl0 = wlmod.make_workload(0)
+    rng = np.random.default_rng(170 + L)
+    x = rng.standard_normal((wl0.N, (L + 1) ** 2, 128)).astype(np.float32)
+    _check(wl0.pos, wl0.box, wl0.r_c, x, wlmod.make_cg_weights(L, 128, 171 + L), L, "fp32")

@@ -47,15 +47,56 @@ __device__ __forceinline__ int degree_of(int q) {
   return l;
 }
 
+__device__ __forceinline__ void store4(float *p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float a, float b, float c, float d) {
+  *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+}
+
 // ---------------------------------------------------------------------------
 // merged RMS norm: one warp per node
 // ---------------------------------------------------------------------------
 template <typename TOUT>
 __global__ void __launch_bounds__(256) rms_norm_kernel(const float *__restrict__ x, const float *__restrict__ add,
                                                        float *__restrict__ x1, const float *__restrict__ gamma,
-                                                       int N, int L, int C, TOUT *__restrict__ out) {
+                                                       int N, int L, int C, TOUT *__restrict__ out, bool vec) {
   const int lane = threadIdx.x & 31;
   const int Q = (L + 1) * (L + 1), QC = Q * C;
+  if (vec) {
+    // C a multiple of 4, every pointer 16-byte aligned: rows (l, m) of four
+    // channels per lane, the degree found once per row
+    const int C4 = C >> 2;
+    for (int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += gridDim.x * (blockDim.x >> 5)) {
+      const size_t nb = (size_t)n * QC;
+      float ss = 0.f;
+      for (int q = 0; q < Q; ++q)
+        for (int c4 = lane; c4 < C4; c4 += 32) {
+          const size_t o = nb + (size_t)q * C + 4 * c4;
+          float4 v = *reinterpret_cast<const float4 *>(x + o);
+          if (add) {
+            const float4 t = *reinterpret_cast<const float4 *>(add + o);
+            v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
+            *reinterpret_cast<float4 *>(x1 + o) = v;
+          }
+          ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+        }
+      ss = warp_sum(ss);
+      const float inv = 1.f / sqrtf(ss / (float)QC + RMS_EPS);
+      const float *vr = add ? x1 : x;   // this lane wrote the x1 entries it reads back
+      int l = 0;
+      for (int q = 0; q < Q; ++q) {
+        if ((l + 1) * (l + 1) <= q) ++l;
+        for (int c4 = lane; c4 < C4; c4 += 32) {
+          const size_t o = nb + (size_t)q * C + 4 * c4;
+          const float4 v = *reinterpret_cast<const float4 *>(vr + o);
+          const float *gr = gamma + l * C + 4 * c4;
+          store4(out + o, gr[0] * v.x * inv, gr[1] * v.y * inv, gr[2] * v.z * inv, gr[3] * v.w * inv);
+        }
+      }
+    }
+    return;
+  }
   for (int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += gridDim.x * (blockDim.x >> 5)) {
     const float *xr = x + (size_t)n * QC;
     const float *ar = add ? add + (size_t)n * QC : nullptr;
@@ -335,7 +376,9 @@ static e2f_status run_norm(const float *x, const float *add, float *x1, const fl
                            TOUT *out, cudaStream_t s) {
   if (N == 0) return E2F_OK;
   const int grid = (int)std::min<long long>((N + 7) / 8, 148LL * 16);
-  E2F_LAUNCH(rms_norm_kernel<TOUT>, grid, 256, 0, s, x, add, x1, gamma, N, L, C, out);
+  auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  const bool vec = (C & 3) == 0 && al16(x) && al16(add) && al16(x1) && al16(out);
+  E2F_LAUNCH(rms_norm_kernel<TOUT>, grid, 256, 0, s, x, add, x1, gamma, N, L, C, out, vec);
   return E2F_OK;
 }
 
